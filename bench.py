@@ -1,0 +1,365 @@
+#!/usr/bin/env python
+"""Benchmark of the fused diagonal-GMM EM step on B200.
+
+One step = one full EM iteration through the C ABI (gmm_em_step: parameter
+prep, the fused E-step + statistics pass over all N rows, the deterministic
+reduction and the M-step) on the resident synthetic workload.  Default
+workload: uint8img (N=1e6, D=128, K=256, fp32 X), the configuration the
+throughput metric is quoted on.
+
+Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then exactly
+K steps between a barrier + synchronize on both sides, timed with CUDA events
+on the stream the library launches on; X (512 MB) is larger than the 126 MB
+L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (plain fp64 EM) on the host cores, on a
+bounded row sample of the same workload per step, scaled to the same unit.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from soft_clustering_em_b200 import synth  # noqa: E402
+
+METRIC = "EM iterations/s and fused E+M N·K·D/s on 1 B200, % of roofline"
+UNIT = "EM iterations/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FUSED_SOURCES = ["soft_clustering_em_b200/csrc/simt_em.cuh",
+                 "soft_clustering_em_b200/csrc/common.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="uint8img", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--rows", type=int, default=0, help="override N (0: the workload's N)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def fused_source_sha():
+    h = hashlib.sha256()
+    for f in FUSED_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """Per-launch DRAM bytes of the fused kernel from a committed ncu summary,
+    or None if there is none for the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    e = d.get(workload)
+    if not e or e.get("source_sha") != fused_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms during a region."""
+
+    Q = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9 or (self.uuid and f[0] != self.uuid):
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s, p in zip(sm, power) if p > 300.0] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded)}
+
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def oracle_sample(wl, X_np, theta, n):
+    """One teacher-forced oracle EM step on the first n rows; returns (seconds, result)."""
+    import oracle
+
+    X64 = synth.x_as_f64(wl, X_np[:n])
+    t0 = time.perf_counter()
+    res = oracle.em_step(X64, *theta, var_floor=wl.var_floor)
+    return time.perf_counter() - t0, res
+
+
+def size_sample(wl, X_np, theta, seconds):
+    """Rows of an oracle sample that takes about `seconds` on this host."""
+    n0 = min(len(X_np), max(256, 2_000_000 // max(1, wl.K * wl.D // 64)))
+    t0, _ = oracle_sample(wl, X_np, theta, n0)
+    n = int(n0 * seconds / max(t0, 1e-3))
+    return max(n0, min(len(X_np), n))
+
+
+def reference_arm(args):
+    """The CPU oracle on the host cores (rank 0 only)."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    import oracle
+
+    wl = synth.WORKLOADS[args.workload]
+    N = args.rows or wl.N
+    X_np, _ = synth.make_data(wl, N)
+    rows = synth.init_rows(N, wl.K, wl.init_seed)
+    mode = 0 if wl.var_init == "one" else 1
+    theta = oracle.init(synth.x_as_f64(wl, X_np), rows, wl.K, mode, wl.var_floor)
+    per_step = min(10.0, 150.0 / max(1, args.steps + args.warmup))
+    n = size_sample(wl, X_np, theta, per_step)
+    for _ in range(args.warmup):
+        oracle_sample(wl, X_np, theta, n)
+    t = 0.0
+    for _ in range(args.steps):
+        dt, _ = oracle_sample(wl, X_np, theta, n)
+        t += dt
+    sec_per_iter = (t / args.steps) * (N / n)
+    value = 1.0 / sec_per_iter
+    sample = (f"first {n} of {N} rows, one EM step per timed step from the data-variance init, "
+              f"time scaled by N/n = {N / n:.1f}")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": sec_per_iter * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl, N),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, N):
+    xb = N * wl.D * (2 if wl.dtype == "bf16" else 4)
+    return {"workload": wl.name, "N": N, "D": wl.D, "K": wl.K, "x_dtype": wl.dtype,
+            "x_bytes": xb, "em_iters_per_run": wl.iters,
+            "l2": "inputs larger than L2 (no flush)" if xb > 126e6 else "L2 flushed between steps"}
+
+
+def ours(args):
+    import torch
+
+    from soft_clustering_em_b200 import gmm as G
+
+    world, rank, local = dist_setup(args)
+    if world > 1:
+        raise SystemExit("multi-GPU row-sharded EM is not built yet")
+    dev = torch.device("cuda", local)
+    wl = synth.WORKLOADS[args.workload]
+    N = args.rows or wl.N
+    X_np, _ = synth.make_data(wl, N)
+    Xh = torch.from_numpy(X_np.view(np.int16) if wl.dtype == "bf16" else X_np)
+    if wl.dtype == "bf16":
+        Xh = Xh.view(torch.bfloat16)
+    Xh = Xh.pin_memory()
+    Xd = Xh.to(dev, non_blocking=False)
+    p = G.problem_for(Xd, wl.K, wl.var_floor)
+    ws = G.workspace(p, dev)
+    rows = synth.init_rows(N, wl.K, wl.init_seed)
+    mode = G.GMM_INIT_VAR_ONE if wl.var_init == "one" else G.GMM_INIT_VAR_DATA
+    w, mu, var = G.gmm_init(Xd, rows, wl.K, mode, wl.var_floor, ws=ws)
+    ll = torch.zeros(1, dtype=torch.float64, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    theta0 = (w.clone(), mu.clone(), var.clone())
+    flush = None if Xd.numel() * Xd.element_size() > 126e6 else torch.empty(
+        256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        G.gmm_em_step(Xd, w, mu, var, ll, wl.var_floor, ws=ws)
+
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else None)
+    time.sleep(0.5)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for e in starts + stops:
+        e.record(stream)
+    torch.cuda.synchronize(dev)
+    launches0 = G.gmm_launch_count()
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_begin.record(stream)
+    for i in range(args.steps):
+        G.gmm_trace_fused(starts[i], stops[i])
+        step()
+        if flush is not None:
+            flush.zero_()
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = G.gmm_launch_count() - launches0
+    G.gmm_trace_fused(None, None)
+    clocks = sampler.stop()
+    total_ms = t_begin.elapsed_time(t_end)
+    fused_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
+    rc, flags = G.gmm_device_status(ws)
+    if rc != 0:
+        raise SystemExit(f"device status {G.status_string(rc)} flags={flags:#x}")
+
+    # ---- end to end: X and parameters from pinned host memory every step ----
+    w_h = theta0[0].cpu().pin_memory()
+    mu_h = theta0[1].cpu().pin_memory()
+    var_h = theta0[2].cpu().pin_memory()
+    ll_h = torch.zeros(1, dtype=torch.float64).pin_memory()
+    Xd2 = torch.empty_like(Xd)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e2e_steps = args.steps
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        Xd2.copy_(Xh, non_blocking=True)
+        w.copy_(w_h, non_blocking=True)
+        mu.copy_(mu_h, non_blocking=True)
+        var.copy_(var_h, non_blocking=True)
+        G.gmm_em_step(Xd2, w, mu, var, ll, wl.var_floor, ws=ws)
+        w_h.copy_(w, non_blocking=True)
+        mu_h.copy_(mu, non_blocking=True)
+        var_h.copy_(var, non_blocking=True)
+        ll_h.copy_(ll, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    pbytes = (w.numel() + mu.numel() + var.numel()) * 4
+    h2d = Xd.numel() * Xd.element_size() + pbytes
+    d2h = pbytes + 8
+
+    ms = total_ms / args.steps
+    value = 1e3 / ms
+    nkd = float(N) * wl.K * wl.D
+    pk, pk_kind = peaks()
+    sustained = total_ms >= 1000.0
+    peak = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    fused_avg = statistics.mean(fused_ms)
+    achieved = 8.0 * nkd / (fused_avg * 1e-3) / 1e12
+    traffic = ncu_traffic(wl.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(wl, N),
+        "nkd_per_s": nkd * value,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "fused E-step + statistics pass",
+                     "algorithmic": "8*N*K*D flop per launch",
+                     "fused_ms_per_launch": fused_avg,
+                     "peak_source": f"{pk_kind} bf16 dense "
+                                    f"{'sustained' if sustained else 'burst'}"},
+        "e2e": {"value": 1e3 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        theta = tuple(t.double().cpu().numpy() for t in theta0)
+        n = size_sample(wl, X_np, theta, args.cpu_seconds)
+        t_cpu, ref = oracle_sample(wl, X_np, theta, n)
+        line["cpu_baseline"] = {
+            "value": 1.0 / (t_cpu * N / n), "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"first {n} of {N} rows, one EM step from the bench's starting "
+                      f"parameters ({t_cpu:.1f} s), time scaled by N/n"}
+        # parity on the same sample, same starting parameters, same kernels
+        from oracle import compare
+
+        ws_s = G.workspace(G.problem_for(Xd[:n], wl.K, wl.var_floor), dev)
+        tw, tmu, tvar = (t.clone() for t in theta0)
+        lls = torch.zeros(1, dtype=torch.float64, device=dev)
+        G.gmm_em_step(Xd[:n], tw, tmu, tvar, lls, wl.var_floor, ws=ws_s)
+        got = (tw.double().cpu().numpy(), tmu.double().cpu().numpy(),
+               tvar.double().cpu().numpy(), lls.item())
+        rep = compare.compare_step(ref[:4], got, ref[4])
+        line["parity"] = {"rows": n, **{k: rep[k] for k in ("ok", "w", "mu", "var", "ll")}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+    ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,172 @@
+/*
+ * gmm.h -- C ABI of the B200 (sm_100a) fused EM library for diagonal-covariance
+ * Gaussian mixtures.
+ *
+ * Method: "Flash-GMM: A Memory-Efficient Kernel for Scalable Soft Clustering"
+ * (abstract; review page sections 1 and 3).  One EM iteration is one pass over
+ * the data in tiles: each tile's E-step log-densities, its per-point
+ * log-sum-exp normalisation into responsibilities and its contribution to the
+ * M-step sufficient statistics are formed on chip, and only the O(K*D)
+ * statistics reach global memory.  The N x K responsibility matrix is never
+ * written anywhere (review page, section 2 and section 3; memory O(KD)
+ * independent of N).
+ *
+ * Model (the pages do not print formulas; this is the textbook diagonal GMM):
+ *   log p(x) = log sum_k pi_k prod_d Normal(x_d; mu_kd, var_kd)
+ *   E-step:  r_nk = pi_k N(x_n | k) / sum_j pi_j N(x_n | j)
+ *   M-step:  pi_k = N_k / N,  mu_k = sum_n r_nk x_n / N_k,
+ *            var_kd = max(sum_n r_nk (x_nd - mu_kd)^2 / N_k, var_floor)
+ *   with N_k = sum_n r_nk.  A component with N_k <= 1e-12 N keeps its mean and
+ *   variance and gets pi_k = N_k / N; a component with pi_k = 0 has
+ *   responsibility 0 everywhere.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All array pointers are DEVICE pointers owned by the caller unless stated.
+ *    The library never allocates or frees device memory and never copies data
+ *    between host and device, except where an entry point says so.
+ *  - X is N x D, row-major, contiguous, of type problem->xdtype (fp32 or bf16),
+ *    16-byte aligned, with D * sizeof(element) a multiple of 16 bytes.
+ *  - w is K floats; mu and var are K x D floats, row-major (component-major).
+ *    Parameters are in the data's own units.
+ *  - ws is a caller-owned device workspace of at least gmm_workspace_size()
+ *    bytes, 256-byte aligned.  Its size depends on D, K, the dtype and the
+ *    device, never on N.  Calls that share a workspace must be ordered on one
+ *    stream.
+ *  - stream is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Every entry point only enqueues work on it and returns without
+ *    waiting, except gmm_device_status.
+ *  - Errors found on the host (null pointers, sizes, alignment, a workspace
+ *    that is too small) are returned before anything is enqueued.  Errors found
+ *    on the device (a non-finite input, a bounded wait that gave up) are
+ *    recorded in a status word inside the workspace; gmm_device_status reads
+ *    and clears it.  No entry point aborts, traps or falls back to the CPU.
+ */
+#ifndef SCEM_GMM_H
+#define SCEM_GMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GMM_OK = 0,
+  GMM_ERR_INVALID_ARG = 1, /* null pointer, N < 1, D < 1, K < 1, m out of range, ... */
+  GMM_ERR_UNSUPPORTED = 2, /* alignment or a shape this build does not handle */
+  GMM_ERR_CUDA = 3,        /* a CUDA runtime call failed (no device, launch error, ...) */
+  GMM_ERR_NUMERIC = 4,     /* the device saw a NaN/Inf in X or an invalid parameter */
+  GMM_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
+  GMM_ERR_WORKSPACE = 6    /* workspace null, misaligned or smaller than required */
+} gmm_status;
+
+typedef enum { GMM_F32 = 0, GMM_BF16 = 1 } gmm_dtype;
+
+typedef enum {
+  GMM_INIT_VAR_ONE = 0, /* every variance starts at 1 */
+  GMM_INIT_VAR_DATA = 1 /* every component starts at the per-dimension (biased)
+                           sample variance of X, floored */
+} gmm_init_var;
+
+typedef struct {
+  int64_t N;       /* number of points, >= 1 */
+  int32_t D;       /* dimensions, >= 1 */
+  int32_t K;       /* mixture components, >= 1 */
+  int32_t xdtype;  /* gmm_dtype of X */
+  float var_floor; /* variance floor applied by the M-step and the data-variance init, >= 0 */
+} gmm_problem;
+
+/* Device status bits recorded in the workspace (see gmm_device_status). */
+#define GMM_DEVFLAG_NONFINITE_X 0x1u     /* a NaN or Inf element in X */
+#define GMM_DEVFLAG_BAD_PARAMS 0x2u      /* w < 0, var <= 0 or a non-finite parameter */
+#define GMM_DEVFLAG_WAIT_TIMEOUT 0x4u    /* a bounded spin on a barrier gave up */
+
+/*
+ * Bytes of device workspace needed for problem p on the CURRENT device.
+ * The value depends on (D, K, xdtype) and the device's SM count only: it is
+ * identical for every N (the O(K*D) memory bound of the review page, section 3).
+ * Returns GMM_ERR_INVALID_ARG for bad arguments, GMM_ERR_CUDA if no device.
+ */
+gmm_status gmm_workspace_size(const gmm_problem* p, size_t* bytes);
+
+/*
+ * Initial parameters.  mu_k = X[rows_host[k]] (K row indices chosen by the
+ * caller, e.g. uniformly without replacement; HOST array of K int64 in
+ * [0, N)), w_k = 1/K, and var = 1 (GMM_INIT_VAR_ONE) or the per-dimension
+ * biased sample variance of X, max(., var_floor), for every component
+ * (GMM_INIT_VAR_DATA).  Writes w, mu, var.  The review page (section 3) gives
+ * no initialisation; this one is the library's definition.
+ */
+gmm_status gmm_init(const gmm_problem* p, const void* X, const int64_t* rows_host,
+                    int32_t init_var, float* w, float* mu, float* var, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/*
+ * One fused EM iteration, in place: (w, mu, var) <- M-step(E-step(X; w, mu, var)).
+ * loglik (device, 1 double, may be NULL) receives LL of the INPUT parameters,
+ * sum_n log p(x_n), including the -D/2 log(2 pi) term.
+ * The N x K responsibilities exist only on chip (review page, sections 2-3).
+ */
+gmm_status gmm_em_step(const gmm_problem* p, const void* X, float* w, float* mu, float* var,
+                       double* loglik, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * iters EM iterations in place.  ll_history (device, iters doubles, may be
+ * NULL) receives LL(theta_t) for t = 0 .. iters-1, each of the parameters that
+ * iteration started from.
+ */
+gmm_status gmm_fit(const gmm_problem* p, const void* X, int32_t iters, float* w, float* mu,
+                   float* var, double* ll_history, void* ws, size_t ws_bytes, void* stream);
+
+/* LL(theta) of the given parameters into *loglik (device, 1 double).  Parameters unchanged. */
+gmm_status gmm_loglik(const gmm_problem* p, const void* X, const float* w, const float* mu,
+                      const float* var, double* loglik, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/*
+ * Multi-assignment of each point to its m most responsible components, for
+ * placing border vectors in several IVF lists (Flash-GMM abstract: the
+ * responsibilities decide which clusters a vector near a cluster border joins).
+ * idx (device, N x m int32) gets component indices ordered by responsibility,
+ * descending, equal responsibilities in ascending index order; resp (device,
+ * N x m float) gets those responsibilities.  1 <= m <= min(K, 8).
+ */
+gmm_status gmm_assign_topm(const gmm_problem* p, const void* X, const float* w,
+                           const float* mu, const float* var, int32_t m, int32_t* idx,
+                           float* resp, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Waits for stream, then reads the device status word of ws into *flags
+ * (GMM_DEVFLAG_* bits; may be NULL) and, if clear != 0, resets it to 0.
+ * Returns GMM_OK when no bit is set, GMM_ERR_NUMERIC for the data/parameter
+ * bits, GMM_ERR_TIMEOUT for the wait bit.  The only entry point that blocks.
+ */
+gmm_status gmm_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* flags,
+                             int32_t clear);
+
+/*
+ * Tracing hook.  While start_event and stop_event (cudaEvent_t handles passed
+ * as void*) are non-NULL, every later call that runs the fused E-step pass
+ * records start_event on its stream just before that kernel's launch and
+ * stop_event just after it, so the kernel's own duration can be read with
+ * cudaEventElapsedTime.  Passing NULL, NULL turns it off.  The setting is
+ * process-wide and not synchronised between host threads.
+ */
+gmm_status gmm_trace_fused(void* start_event, void* stop_event);
+
+/*
+ * Number of kernels this library has enqueued in this process so far (all
+ * entry points, all devices), into *count.  For tracing and benchmarking.
+ */
+gmm_status gmm_launch_count(uint64_t* count);
+
+/* Static, human-readable name of a status code. */
+const char* gmm_status_string(gmm_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SCEM_GMM_H */

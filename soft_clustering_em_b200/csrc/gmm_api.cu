@@ -1,0 +1,288 @@
+// gmm_api.cu -- host side of the C ABI declared in include/gmm.h: argument
+// checks, workspace layout and the launch sequence of each entry point.
+// Nothing here allocates device memory or synchronises, except
+// gmm_device_status.
+#include <stdio.h>
+
+#include "common.cuh"
+#include "gmm.h"
+#include "simt_em.cuh"
+
+using namespace scem;
+
+namespace {
+
+size_t elem_bytes(int32_t t) { return t == GMM_BF16 ? 2 : 4; }
+
+gmm_status check_problem(const gmm_problem* p) {
+  if (!p) return GMM_ERR_INVALID_ARG;
+  if (p->N < 1 || p->D < 1 || p->K < 1) return GMM_ERR_INVALID_ARG;
+  if (p->xdtype != GMM_F32 && p->xdtype != GMM_BF16) return GMM_ERR_INVALID_ARG;
+  if (!(p->var_floor >= 0.f) || !isfinite(p->var_floor)) return GMM_ERR_INVALID_ARG;
+  if (p->D > kMaxD || p->K > kMaxK) return GMM_ERR_UNSUPPORTED;
+  if ((size_t)p->N > ((size_t)1 << 40)) return GMM_ERR_UNSUPPORTED;
+  return GMM_OK;
+}
+
+gmm_status check_x(const gmm_problem* p, const void* X) {
+  if (!X) return GMM_ERR_INVALID_ARG;
+  if (((uintptr_t)X) % 16 != 0) return GMM_ERR_UNSUPPORTED;
+  if (((size_t)p->D * elem_bytes(p->xdtype)) % 16 != 0) return GMM_ERR_UNSUPPORTED;
+  return GMM_OK;
+}
+
+gmm_status device_sms(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GMM_ERR_CUDA;
+  }
+  if (cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GMM_ERR_CUDA;
+  }
+  return GMM_OK;
+}
+
+gmm_status get_layout(const gmm_problem* p, void* ws, size_t ws_bytes, WsLayout* L) {
+  int sms = 0;
+  gmm_status s = device_sms(&sms);
+  if (s != GMM_OK) return s;
+  *L = ws_layout(p->D, p->K, sms);
+  if (!ws || ((uintptr_t)ws) % 256 != 0 || ws_bytes < L->total) return GMM_ERR_WORKSPACE;
+  return GMM_OK;
+}
+
+unsigned long long g_launches = 0;  // kernels enqueued by this library
+
+gmm_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    fprintf(stderr, "gmm: CUDA launch failed: %s\n", cudaGetErrorString(e));
+    return GMM_ERR_CUDA;
+  }
+  return GMM_OK;
+}
+
+cudaEvent_t g_trace_start = nullptr, g_trace_stop = nullptr;
+
+void trace_begin(cudaStream_t st) {
+  if (g_trace_start) cudaEventRecord(g_trace_start, st);
+}
+void trace_end(cudaStream_t st) {
+  if (g_trace_stop) cudaEventRecord(g_trace_stop, st);
+}
+
+// Status after enqueuing n kernels (counted for gmm_launch_count).
+gmm_status launched(int n) {
+  g_launches += n;
+  return launch_status();
+}
+
+template <typename XT, int MODE>
+gmm_status launch_simt(const gmm_problem* p, const void* X, const WsPtrs& w, int m, int32_t* idx,
+                       float* resp, cudaStream_t st) {
+  const size_t smem = simt_smem_bytes(p->D);
+  auto kern = simt_fused_kernel<XT, MODE>;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return GMM_ERR_UNSUPPORTED;
+    }
+  }
+  trace_begin(st);
+  kern<<<w.P, kSimtThreads, smem, st>>>((const XT*)X, p->N, p->D, p->K, w, m, idx, resp);
+  trace_end(st);
+  return launched(1);
+}
+
+template <int MODE>
+gmm_status fused_pass(const gmm_problem* p, const void* X, const WsPtrs& w, int m, int32_t* idx,
+                      float* resp, cudaStream_t st) {
+  if (p->xdtype == GMM_BF16) return launch_simt<__nv_bfloat16, MODE>(p, X, w, m, idx, resp, st);
+  return launch_simt<float, MODE>(p, X, w, m, idx, resp, st);
+}
+
+gmm_status prep(const gmm_problem* p, const float* w, const float* mu, const float* var,
+                const WsPtrs& ws, cudaStream_t st) {
+  prep_kernel<<<p->K, 128, 0, st>>>(p->D, p->K, w, mu, var, ws);
+  return launched(1);
+}
+
+gmm_status em_step_impl(const gmm_problem* p, const void* X, float* w, float* mu, float* var,
+                        double* loglik, const WsPtrs& ws, cudaStream_t st) {
+  gmm_status s = prep(p, w, mu, var, ws, st);
+  if (s != GMM_OK) return s;
+  s = fused_pass<kModeStats>(p, X, ws, 0, nullptr, nullptr, st);
+  if (s != GMM_OK) return s;
+  const size_t KD = (size_t)p->K * p->D;
+  reduce_mstep_kernel<<<(unsigned)((KD + 255) / 256), 256, 0, st>>>(p->N, p->D, p->K, p->var_floor,
+                                                                    ws, w, mu, var, loglik);
+  return launched(1);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gmm_status_string(gmm_status s) {
+  switch (s) {
+    case GMM_OK: return "GMM_OK";
+    case GMM_ERR_INVALID_ARG: return "GMM_ERR_INVALID_ARG";
+    case GMM_ERR_UNSUPPORTED: return "GMM_ERR_UNSUPPORTED";
+    case GMM_ERR_CUDA: return "GMM_ERR_CUDA";
+    case GMM_ERR_NUMERIC: return "GMM_ERR_NUMERIC";
+    case GMM_ERR_TIMEOUT: return "GMM_ERR_TIMEOUT";
+    case GMM_ERR_WORKSPACE: return "GMM_ERR_WORKSPACE";
+  }
+  return "GMM_ERR_UNKNOWN";
+}
+
+gmm_status gmm_workspace_size(const gmm_problem* p, size_t* bytes) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if (!bytes) return GMM_ERR_INVALID_ARG;
+  int sms = 0;
+  s = device_sms(&sms);
+  if (s != GMM_OK) return s;
+  *bytes = ws_layout(p->D, p->K, sms).total;
+  return GMM_OK;
+}
+
+gmm_status gmm_init(const gmm_problem* p, const void* X, const int64_t* rows_host,
+                    int32_t init_var, float* w, float* mu, float* var, void* ws, size_t ws_bytes,
+                    void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if ((s = check_x(p, X)) != GMM_OK) return s;
+  if (!rows_host || !w || !mu || !var) return GMM_ERR_INVALID_ARG;
+  if (init_var != GMM_INIT_VAR_ONE && init_var != GMM_INIT_VAR_DATA) return GMM_ERR_INVALID_ARG;
+  for (int k = 0; k < p->K; k++)
+    if (rows_host[k] < 0 || rows_host[k] >= p->N) return GMM_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
+  WsPtrs wp = ws_ptrs(ws, L);
+  cudaStream_t st = (cudaStream_t)stream;
+  // the K row indices travel to the workspace (the one host->device copy of this call)
+  if (cudaMemcpyAsync(wp.scratch, rows_host, sizeof(int64_t) * p->K, cudaMemcpyHostToDevice, st) !=
+      cudaSuccess) {
+    launch_status();
+    return GMM_ERR_CUDA;
+  }
+  const bool bf = p->xdtype == GMM_BF16;
+  if (bf)
+    init_gather_kernel<__nv_bfloat16><<<p->K, 128, 0, st>>>((const __nv_bfloat16*)X, p->D, p->K,
+                                                           wp.scratch, init_var, w, mu, var);
+  else
+    init_gather_kernel<float><<<p->K, 128, 0, st>>>((const float*)X, p->D, p->K, wp.scratch,
+                                                    init_var, w, mu, var);
+  if ((s = launched(1)) != GMM_OK) return s;
+  if (init_var == GMM_INIT_VAR_DATA) {
+    double* part = wp.slots;
+    double* mean = part + (size_t)wp.P * p->D;
+    for (int pass = 0; pass < 2; pass++) {
+      const double* mptr = pass == 0 ? nullptr : mean;
+      if (bf)
+        col_partial_kernel<__nv_bfloat16><<<wp.P, 256, 0, st>>>((const __nv_bfloat16*)X, p->N,
+                                                                p->D, mptr, part);
+      else
+        col_partial_kernel<float><<<wp.P, 256, 0, st>>>((const float*)X, p->N, p->D, mptr, part);
+      col_finish_kernel<<<(p->D + 127) / 128, 128, 0, st>>>(p->N, p->D, p->K, wp.P, part, pass,
+                                                            p->var_floor, mean, var);
+      if ((s = launched(2)) != GMM_OK) return s;
+    }
+  }
+  return GMM_OK;
+}
+
+gmm_status gmm_em_step(const gmm_problem* p, const void* X, float* w, float* mu, float* var,
+                       double* loglik, void* ws, size_t ws_bytes, void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if ((s = check_x(p, X)) != GMM_OK) return s;
+  if (!w || !mu || !var) return GMM_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
+  return em_step_impl(p, X, w, mu, var, loglik, ws_ptrs(ws, L), (cudaStream_t)stream);
+}
+
+gmm_status gmm_fit(const gmm_problem* p, const void* X, int32_t iters, float* w, float* mu,
+                   float* var, double* ll_history, void* ws, size_t ws_bytes, void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if ((s = check_x(p, X)) != GMM_OK) return s;
+  if (!w || !mu || !var || iters < 0) return GMM_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
+  const WsPtrs wp = ws_ptrs(ws, L);
+  for (int t = 0; t < iters; t++) {
+    s = em_step_impl(p, X, w, mu, var, ll_history ? ll_history + t : nullptr, wp,
+                     (cudaStream_t)stream);
+    if (s != GMM_OK) return s;
+  }
+  return GMM_OK;
+}
+
+gmm_status gmm_loglik(const gmm_problem* p, const void* X, const float* w, const float* mu,
+                      const float* var, double* loglik, void* ws, size_t ws_bytes, void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if ((s = check_x(p, X)) != GMM_OK) return s;
+  if (!w || !mu || !var || !loglik) return GMM_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
+  const WsPtrs wp = ws_ptrs(ws, L);
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((s = prep(p, w, mu, var, wp, st)) != GMM_OK) return s;
+  if ((s = fused_pass<kModeLoglik>(p, X, wp, 0, nullptr, nullptr, st)) != GMM_OK) return s;
+  reduce_loglik_kernel<<<1, 1, 0, st>>>(p->D, p->K, wp, loglik);
+  return launched(1);
+}
+
+gmm_status gmm_assign_topm(const gmm_problem* p, const void* X, const float* w, const float* mu,
+                           const float* var, int32_t m, int32_t* idx, float* resp, void* ws,
+                           size_t ws_bytes, void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if ((s = check_x(p, X)) != GMM_OK) return s;
+  if (!w || !mu || !var || !idx || !resp) return GMM_ERR_INVALID_ARG;
+  if (m < 1 || m > kMaxTopM || m > p->K) return GMM_ERR_INVALID_ARG;
+  WsLayout L;
+  if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
+  const WsPtrs wp = ws_ptrs(ws, L);
+  cudaStream_t st = (cudaStream_t)stream;
+  if ((s = prep(p, w, mu, var, wp, st)) != GMM_OK) return s;
+  return fused_pass<kModeTopm>(p, X, wp, m, idx, resp, st);
+}
+
+gmm_status gmm_launch_count(uint64_t* count) {
+  if (!count) return GMM_ERR_INVALID_ARG;
+  *count = g_launches;
+  return GMM_OK;
+}
+
+gmm_status gmm_trace_fused(void* start_event, void* stop_event) {
+  if ((start_event == nullptr) != (stop_event == nullptr)) return GMM_ERR_INVALID_ARG;
+  g_trace_start = (cudaEvent_t)start_event;
+  g_trace_stop = (cudaEvent_t)stop_event;
+  return GMM_OK;
+}
+
+gmm_status gmm_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* flags,
+                             int32_t clear) {
+  if (!ws || ws_bytes < 16) return GMM_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  uint32_t f = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return launch_status(), GMM_ERR_CUDA;
+  if (cudaMemcpy(&f, ws, sizeof(f), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return launch_status(), GMM_ERR_CUDA;
+  if (clear && cudaMemset(ws, 0, sizeof(uint32_t)) != cudaSuccess)
+    return launch_status(), GMM_ERR_CUDA;
+  if (flags) *flags = f;
+  if (f & GMM_DEVFLAG_WAIT_TIMEOUT) return GMM_ERR_TIMEOUT;
+  if (f & (GMM_DEVFLAG_NONFINITE_X | GMM_DEVFLAG_BAD_PARAMS)) return GMM_ERR_NUMERIC;
+  return GMM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,203 @@
+"""Thin Python binding of the C ABI in include/gmm.h (argument marshalling only).
+
+Every entry point keeps its C name.  Arrays are torch CUDA tensors; the binding
+passes their device pointers and the current CUDA stream to the library and
+does no arithmetic of its own.  The library must be built
+(``python -m soft_clustering_em_b200.build``); if it is missing every call
+raises -- there is no fallback implementation.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libscem_gmm.so")
+
+GMM_OK, GMM_ERR_INVALID_ARG, GMM_ERR_UNSUPPORTED, GMM_ERR_CUDA = 0, 1, 2, 3
+GMM_ERR_NUMERIC, GMM_ERR_TIMEOUT, GMM_ERR_WORKSPACE = 4, 5, 6
+GMM_F32, GMM_BF16 = 0, 1
+GMM_INIT_VAR_ONE, GMM_INIT_VAR_DATA = 0, 1
+GMM_DEVFLAG_NONFINITE_X, GMM_DEVFLAG_BAD_PARAMS, GMM_DEVFLAG_WAIT_TIMEOUT = 0x1, 0x2, 0x4
+
+EXPORTS = ("gmm_workspace_size", "gmm_init", "gmm_em_step", "gmm_fit", "gmm_loglik",
+           "gmm_assign_topm", "gmm_device_status", "gmm_trace_fused", "gmm_launch_count",
+           "gmm_status_string")
+
+
+class gmm_problem(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("D", ctypes.c_int32), ("K", ctypes.c_int32),
+                ("xdtype", ctypes.c_int32), ("var_floor", ctypes.c_float)]
+
+
+class GmmError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load the CUDA library and declare its signatures (raises if not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library {path} is not built; run "
+                           "`python -m soft_clustering_em_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    PP = ctypes.POINTER(gmm_problem)
+    lib.gmm_workspace_size.argtypes = [PP, ctypes.POINTER(SZ)]
+    lib.gmm_init.argtypes = [PP, P, ctypes.POINTER(I64), I32, P, P, P, P, SZ, P]
+    lib.gmm_em_step.argtypes = [PP, P, P, P, P, P, P, SZ, P]
+    lib.gmm_fit.argtypes = [PP, P, I32, P, P, P, P, P, SZ, P]
+    lib.gmm_loglik.argtypes = [PP, P, P, P, P, P, P, SZ, P]
+    lib.gmm_assign_topm.argtypes = [PP, P, P, P, P, I32, P, P, P, SZ, P]
+    lib.gmm_device_status.argtypes = [P, SZ, P, ctypes.POINTER(ctypes.c_uint32), I32]
+    lib.gmm_trace_fused.argtypes = [P, P]
+    lib.gmm_launch_count.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
+    lib.gmm_status_string.argtypes = [ctypes.c_int]
+    lib.gmm_status_string.restype = ctypes.c_char_p
+    for name in EXPORTS[:-1]:
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(s: int) -> str:
+    return load_library().gmm_status_string(int(s)).decode()
+
+
+def _check(rc, what):
+    if rc != GMM_OK:
+        raise GmmError(rc, what)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def xdtype_of(X) -> int:
+    if X.dtype == torch.float32:
+        return GMM_F32
+    if X.dtype == torch.bfloat16:
+        return GMM_BF16
+    raise TypeError(f"X must be float32 or bfloat16, got {X.dtype}")
+
+
+def problem(N, D, K, xdtype=GMM_F32, var_floor=1e-6) -> gmm_problem:
+    return gmm_problem(int(N), int(D), int(K), int(xdtype), float(var_floor))
+
+
+def problem_for(X, K, var_floor=1e-6) -> gmm_problem:
+    N, D = X.shape
+    return problem(N, D, K, xdtype_of(X), var_floor)
+
+
+def gmm_workspace_size(p: gmm_problem) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().gmm_workspace_size(ctypes.byref(p), ctypes.byref(n)),
+           "gmm_workspace_size")
+    return int(n.value)
+
+
+def workspace(p: gmm_problem, device=None) -> torch.Tensor:
+    """A zero-filled device workspace for problem p (caller-owned, reusable)."""
+    return torch.zeros(gmm_workspace_size(p), dtype=torch.uint8, device=device or "cuda")
+
+
+def _ws(p, ws, device):
+    return workspace(p, device) if ws is None else ws
+
+
+def gmm_init(X, rows, K, init_var=GMM_INIT_VAR_DATA, var_floor=1e-6, ws=None, stream=None):
+    """Initial (w, mu, var) from the K chosen rows of X (host int64 indices)."""
+    p = problem_for(X, K, var_floor)
+    ws = _ws(p, ws, X.device)
+    rows = (ctypes.c_int64 * K)(*[int(r) for r in rows])
+    w = torch.empty(K, dtype=torch.float32, device=X.device)
+    mu = torch.empty(K, X.shape[1], dtype=torch.float32, device=X.device)
+    var = torch.empty_like(mu)
+    _check(load_library().gmm_init(ctypes.byref(p), _ptr(X), rows, int(init_var), _ptr(w),
+                                   _ptr(mu), _ptr(var), _ptr(ws), ws.numel(), _stream(stream)),
+           "gmm_init")
+    return w, mu, var
+
+
+def gmm_em_step(X, w, mu, var, loglik=None, var_floor=1e-6, ws=None, stream=None):
+    """One fused EM iteration in place; loglik (1 double, device) gets LL of the input."""
+    p = problem_for(X, w.numel(), var_floor)
+    ws = _ws(p, ws, X.device)
+    _check(load_library().gmm_em_step(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu), _ptr(var),
+                                      _ptr(loglik), _ptr(ws), ws.numel(), _stream(stream)),
+           "gmm_em_step")
+
+
+def gmm_fit(X, w, mu, var, iters, var_floor=1e-6, ws=None, stream=None):
+    """iters EM iterations in place; returns the device LL history (iters doubles)."""
+    p = problem_for(X, w.numel(), var_floor)
+    ws = _ws(p, ws, X.device)
+    ll = torch.zeros(max(int(iters), 1), dtype=torch.float64, device=X.device)
+    _check(load_library().gmm_fit(ctypes.byref(p), _ptr(X), int(iters), _ptr(w), _ptr(mu),
+                                  _ptr(var), _ptr(ll), _ptr(ws), ws.numel(), _stream(stream)),
+           "gmm_fit")
+    return ll[:iters]
+
+
+def gmm_loglik(X, w, mu, var, var_floor=1e-6, ws=None, stream=None):
+    """LL of the given parameters as a 1-element device double tensor."""
+    p = problem_for(X, w.numel(), var_floor)
+    ws = _ws(p, ws, X.device)
+    ll = torch.zeros(1, dtype=torch.float64, device=X.device)
+    _check(load_library().gmm_loglik(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu), _ptr(var),
+                                     _ptr(ll), _ptr(ws), ws.numel(), _stream(stream)),
+           "gmm_loglik")
+    return ll
+
+
+def gmm_assign_topm(X, w, mu, var, m, var_floor=1e-6, ws=None, stream=None):
+    """(idx N x m int32, resp N x m float32): the m most responsible components per point."""
+    p = problem_for(X, w.numel(), var_floor)
+    ws = _ws(p, ws, X.device)
+    N = X.shape[0]
+    idx = torch.empty(N, int(m), dtype=torch.int32, device=X.device)
+    resp = torch.empty(N, int(m), dtype=torch.float32, device=X.device)
+    _check(load_library().gmm_assign_topm(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu), _ptr(var),
+                                          int(m), _ptr(idx), _ptr(resp), _ptr(ws), ws.numel(),
+                                          _stream(stream)), "gmm_assign_topm")
+    return idx, resp
+
+
+def gmm_device_status(ws, clear=True, stream=None):
+    """(status, flags): waits for the stream and reads the workspace's device status word."""
+    f = ctypes.c_uint32(0)
+    rc = load_library().gmm_device_status(_ptr(ws), ws.numel(), _stream(stream), ctypes.byref(f),
+                                          int(bool(clear)))
+    return rc, int(f.value)
+
+
+def gmm_trace_fused(start=None, stop=None):
+    """Record torch.cuda.Event start/stop around every later fused-kernel launch (None: off)."""
+    if start is None:
+        _check(load_library().gmm_trace_fused(None, None), "gmm_trace_fused")
+        return
+    for e in (start, stop):
+        if not e.cuda_event:
+            e.record()  # torch creates the CUDA event lazily, on its first record
+    _check(load_library().gmm_trace_fused(ctypes.c_void_p(start.cuda_event),
+                                          ctypes.c_void_p(stop.cuda_event)), "gmm_trace_fused")
+
+
+def gmm_launch_count() -> int:
+    """Kernels the library has enqueued in this process so far."""
+    c = ctypes.c_uint64(0)
+    _check(load_library().gmm_launch_count(ctypes.byref(c)), "gmm_launch_count")
+    return int(c.value)

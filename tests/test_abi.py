@@ -1,0 +1,110 @@
+"""The C-ABI library loads, exports every symbol include/gmm.h declares, and
+rejects bad arguments on the host before touching the device (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from soft_clustering_em_b200 import gmm as G
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from soft_clustering_em_b200 import build
+
+    build.build()
+    return G.load_library()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "gmm.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gmm_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_calls():
+    names = declared_functions()
+    for n in ("gmm_init", "gmm_em_step", "gmm_fit", "gmm_loglik", "gmm_assign_topm",
+              "gmm_workspace_size", "gmm_device_status", "gmm_trace_fused",
+              "gmm_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    assert set(declared_functions()) <= set(G.EXPORTS)
+
+
+def test_status_strings(lib):
+    assert G.status_string(0) == "GMM_OK"
+    assert G.status_string(G.GMM_ERR_WORKSPACE) == "GMM_ERR_WORKSPACE"
+    assert G.status_string(99) == "GMM_ERR_UNKNOWN"
+
+
+def _call_em(lib, p, X=16, w=16, mu=16, var=16):
+    P = ctypes.c_void_p
+    return lib.gmm_em_step(ctypes.byref(p), P(X), P(w), P(mu), P(var), P(0), P(256), 1 << 30,
+                           P(0))
+
+
+@pytest.mark.parametrize("N,D,K,dt,floor,code", [
+    (0, 4, 2, 0, 1e-6, G.GMM_ERR_INVALID_ARG),
+    (10, 0, 2, 0, 1e-6, G.GMM_ERR_INVALID_ARG),
+    (10, 4, 0, 0, 1e-6, G.GMM_ERR_INVALID_ARG),
+    (10, 4, 2, 7, 1e-6, G.GMM_ERR_INVALID_ARG),
+    (10, 4, 2, 0, float("nan"), G.GMM_ERR_INVALID_ARG),
+    (10, 4, 2, 0, -1.0, G.GMM_ERR_INVALID_ARG),
+    (10, 2, 2, 0, 1e-6, G.GMM_ERR_UNSUPPORTED),   # 8-byte rows: not a TMA-legal row pitch
+    (10, 4, 2, 1, 1e-6, G.GMM_ERR_UNSUPPORTED),   # bf16 rows must be 16-byte multiples too
+    (10, 4096, 2, 0, 1e-6, G.GMM_ERR_UNSUPPORTED),
+])
+def test_em_step_rejects_bad_problems(lib, N, D, K, dt, floor, code):
+    assert _call_em(lib, G.problem(N, D, K, dt, floor)) == code
+
+
+def test_null_and_misaligned_pointers(lib):
+    p = G.problem(10, 4, 2)
+    assert _call_em(lib, p, X=0) == G.GMM_ERR_INVALID_ARG
+    assert _call_em(lib, p, X=8) == G.GMM_ERR_UNSUPPORTED
+    assert _call_em(lib, p, w=0) == G.GMM_ERR_INVALID_ARG
+    assert _call_em(lib, p, var=0) == G.GMM_ERR_INVALID_ARG
+    assert lib.gmm_workspace_size(ctypes.byref(p), None) == G.GMM_ERR_INVALID_ARG
+    assert lib.gmm_workspace_size(None, ctypes.byref(ctypes.c_size_t())) == G.GMM_ERR_INVALID_ARG
+
+
+def test_topm_and_init_argument_checks(lib):
+    P = ctypes.c_void_p
+    p = G.problem(10, 4, 3)
+    for m in (0, 4, 9):
+        rc = lib.gmm_assign_topm(ctypes.byref(p), P(16), P(16), P(16), P(16), m, P(16), P(16),
+                                 P(256), 1 << 30, P(0))
+        assert rc == G.GMM_ERR_INVALID_ARG, m
+    rows = (ctypes.c_int64 * 3)(0, 5, 10)  # 10 is out of range for N = 10
+    rc = lib.gmm_init(ctypes.byref(p), P(16), rows, 1, P(16), P(16), P(16), P(256), 1 << 30, P(0))
+    assert rc == G.GMM_ERR_INVALID_ARG
+    rows = (ctypes.c_int64 * 3)(0, 5, 9)
+    rc = lib.gmm_init(ctypes.byref(p), P(16), rows, 2, P(16), P(16), P(16), P(256), 1 << 30, P(0))
+    assert rc == G.GMM_ERR_INVALID_ARG
+    rc = lib.gmm_fit(ctypes.byref(p), P(16), -1, P(16), P(16), P(16), P(0), P(256), 1 << 30, P(0))
+    assert rc == G.GMM_ERR_INVALID_ARG
+
+
+def test_no_device_is_a_cuda_error_not_a_crash(lib):
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    p = G.problem(1000, 16, 8)
+    n = ctypes.c_size_t(0)
+    assert lib.gmm_workspace_size(ctypes.byref(p), ctypes.byref(n)) == G.GMM_ERR_CUDA
+    assert _call_em(lib, p) == G.GMM_ERR_CUDA
+
+
+def test_trace_hook_arguments(lib):
+    P = ctypes.c_void_p
+    assert lib.gmm_trace_fused(P(16), None) == G.GMM_ERR_INVALID_ARG
+    assert lib.gmm_trace_fused(None, None) == G.GMM_OK

@@ -1,0 +1,243 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Every EM step is teacher-forced: the oracle starts from exactly the fp32
+parameters the GPU started from, and the two results are compared under the
+rules in oracle/compare.py.  Inputs are the seeded synthetic workloads of
+soft_clustering_em_b200.synth, down-scaled in N so the oracle finishes in
+seconds, with ragged N (not a multiple of any tile) and the degenerate cases.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from oracle import compare
+from soft_clustering_em_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def G():
+    import torch
+
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from soft_clustering_em_b200 import build
+    from soft_clustering_em_b200 import gmm
+
+    build.build()
+    gmm.load_library()
+    return gmm
+
+
+def to_device(wl, X):
+    import torch
+
+    if wl.dtype == "bf16":
+        return torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(X).cuda()
+
+
+def params_np(w, mu, var):
+    return (w.double().cpu().numpy(), mu.double().cpu().numpy(), var.double().cpu().numpy())
+
+
+def run_teacher_forced(G, wl, N, K, iters, rows=None):
+    import torch
+
+    X, _ = synth.make_data(wl, N)
+    X64 = synth.x_as_f64(wl, X)
+    Xd = to_device(wl, X)
+    rows = synth.init_rows(N, K, wl.init_seed) if rows is None else rows
+    mode = G.GMM_INIT_VAR_ONE if wl.var_init == "one" else G.GMM_INIT_VAR_DATA
+    p = G.problem_for(Xd, K, wl.var_floor)
+    ws = G.workspace(p)
+    w, mu, var = G.gmm_init(Xd, rows, K, mode, wl.var_floor, ws=ws)
+    # init parity: gathered means exact, data variance to fp32 rounding
+    rw, rmu, rvar = oracle.init(X64, rows, K, mode, wl.var_floor)
+    gw, gmu, gvar = params_np(w, mu, var)
+    np.testing.assert_array_equal(gmu, rmu)
+    np.testing.assert_allclose(gw, rw, rtol=1e-7)
+    np.testing.assert_allclose(gvar, rvar, rtol=1e-6)
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    reports = []
+    for t in range(iters):
+        th = params_np(w, mu, var)
+        G.gmm_em_step(Xd, w, mu, var, ll, wl.var_floor, ws=ws)
+        torch.cuda.synchronize()
+        rc, flags = G.gmm_device_status(ws)
+        assert rc == 0 and flags == 0
+        w2, mu2, var2, ll_ref, Nk = oracle.em_step(X64, *th, var_floor=wl.var_floor)
+        got = (*params_np(w, mu, var), float(ll.item()))
+        rep = compare.compare_step((w2, mu2, var2, ll_ref), got, Nk)
+        reports.append(rep)
+        assert rep["ok"], (t, rep)
+    return Xd, X64, (w, mu, var), reports
+
+
+CASES = [
+    ("gauss8", 10_000, 8, 10),
+    ("gauss8", 10_007, 8, 3),
+    ("uint8img", 20_011, 256, 3),
+    ("sphere768", 3_001, 1024, 2),
+    ("gauss4096", 20_000, 4096, 2),
+    ("bf16stream", 50_001, 1024, 3),
+]
+
+
+@pytest.mark.parametrize("name,N,K,iters", CASES)
+def test_em_steps_match_oracle(G, name, N, K, iters):
+    run_teacher_forced(G, synth.WORKLOADS[name], N, K, iters)
+
+
+@pytest.mark.parametrize("name,N,K", [("sphere768", 2_003, 1024), ("bf16stream", 30_001, 1024),
+                                      ("gauss8", 1_001, 8)])
+def test_loglik_and_topm_match_oracle(G, name, N, K):
+    wl = synth.WORKLOADS[name]
+    Xd, X64, (w, mu, var), _ = run_teacher_forced(G, wl, N, K, 2)
+    th = params_np(w, mu, var)
+    ll = G.gmm_loglik(Xd, w, mu, var, wl.var_floor)
+    ll_ref = oracle.loglik(X64, *th)
+    assert abs(ll.item() - ll_ref) <= compare.LL_REL * abs(ll_ref)
+    for m in (1, 2, 3):
+        idx, resp = G.gmm_assign_topm(Xd, w, mu, var, m)
+        ridx, rresp = oracle.assign_topm(X64, *th, min(m + 1, K))
+        bad, worst = compare.compare_topm(ridx[:, :m], rresp[:, :m], idx.cpu().numpy(),
+                                          resp.cpu().numpy(), rresp)
+        assert bad == 0 and worst <= 1.0, (m, bad, worst)
+
+
+def _tiny(G, X, w, mu, var, floor=1e-6):
+    import torch
+
+    Xd = torch.tensor(X, dtype=torch.float32, device="cuda")
+    wd = torch.tensor(w, dtype=torch.float32, device="cuda")
+    mud = torch.tensor(mu, dtype=torch.float32, device="cuda")
+    vard = torch.tensor(var, dtype=torch.float32, device="cuda")
+    th = params_np(wd, mud, vard)
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    G.gmm_em_step(Xd, wd, mud, vard, ll, floor)
+    ref = oracle.em_step(np.asarray(X, dtype=np.float32).astype(np.float64), *th, var_floor=floor)
+    return ref, (*params_np(wd, mud, vard), ll.item())
+
+
+def test_single_point_single_component(G):
+    ref, got = _tiny(G, [[1.0, 2.0, 3.0, 4.0]], [1.0], [[0.0] * 4], [[1.0] * 4])
+    np.testing.assert_allclose(got[0], [1.0])
+    np.testing.assert_allclose(got[1], [[1, 2, 3, 4]], rtol=1e-6)
+    np.testing.assert_allclose(got[2], 1e-6, rtol=1e-6)  # one point: variance hits the floor
+    assert abs(got[3] - ref[3]) <= 1e-6 * abs(ref[3])
+
+
+def test_k1_closed_form_and_max_d(G):
+    rng = np.random.default_rng(3)
+    D = 1024
+    X = (rng.normal(size=(777, D)) * 3 + 1).astype(np.float32)
+    ref, got = _tiny(G, X, [1.0], rng.normal(size=(1, D)), np.ones((1, D)))
+    X64 = X.astype(np.float64)
+    np.testing.assert_allclose(got[1][0], X64.mean(0), rtol=0, atol=1e-3 * 3)
+    np.testing.assert_allclose(got[2][0], X64.var(0), rtol=1e-3)
+    assert compare.compare_step(ref[:4], got, ref[4])["ok"]
+
+
+def test_ragged_k_and_dead_component(G):
+    rng = np.random.default_rng(5)
+    K, D, N = 300, 8, 4_099
+    X = rng.normal(size=(N, D)).astype(np.float32) * 4
+    w = rng.dirichlet(np.ones(K))
+    w[7] = 0.0  # dead: responsibility 0 everywhere
+    w = w / w.sum()
+    mu = X[rng.choice(N, K, replace=False)]
+    ref, got = _tiny(G, X, w, mu, np.ones((K, D)))
+    assert got[0][7] == 0.0
+    assert compare.compare_step(ref[:4], got, ref[4])["ok"]
+
+
+def test_workspace_does_not_depend_on_n(G):
+    for D, K, dt in ((128, 256, 0), (96, 4096, 0), (32, 1024, 1), (768, 1024, 0)):
+        sizes = {G.gmm_workspace_size(G.problem(N, D, K, dt)) for N in (10_000, 10**6, 10**8)}
+        assert len(sizes) == 1
+
+
+def test_step_allocates_no_device_memory(G):
+    import torch
+
+    wl = synth.WORKLOADS["uint8img"]
+    X, _ = synth.make_data(wl, 200_000)
+    Xd = to_device(wl, X)
+    p = G.problem_for(Xd, wl.K)
+    ws = G.workspace(p)
+    w, mu, var = G.gmm_init(Xd, synth.init_rows(len(X), wl.K, 1), wl.K, ws=ws)
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    G.gmm_em_step(Xd, w, mu, var, ll, ws=ws)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        G.gmm_em_step(Xd, w, mu, var, ll, ws=ws)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free0 == free1
+
+
+def test_deterministic(G):
+    import torch
+
+    wl = synth.WORKLOADS["bf16stream"]
+    X, _ = synth.make_data(wl, 40_000)
+    Xd = to_device(wl, X)
+    ws = G.workspace(G.problem_for(Xd, wl.K))
+    w, mu, var = G.gmm_init(Xd, synth.init_rows(len(X), wl.K, 9), wl.K, ws=ws)
+    outs = []
+    for _ in range(2):
+        w2, mu2, var2 = w.clone(), mu.clone(), var.clone()
+        ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+        G.gmm_em_step(Xd, w2, mu2, var2, ll, ws=ws)
+        outs.append((w2.cpu(), mu2.cpu(), var2.cpu(), ll.cpu()))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
+def test_nonfinite_input_sets_device_flag(G):
+    import torch
+
+    rng = np.random.default_rng(1)
+    X = rng.normal(size=(1000, 16)).astype(np.float32)
+    X[123, 4] = np.nan
+    Xd = torch.tensor(X, device="cuda")
+    ws = G.workspace(G.problem_for(Xd, 4))
+    w = torch.full((4,), 0.25, device="cuda")
+    mu = torch.tensor(X[:4], device="cuda").nan_to_num()
+    var = torch.ones(4, 16, device="cuda")
+    G.gmm_em_step(Xd, w, mu, var, ws=ws)
+    rc, flags = G.gmm_device_status(ws)
+    assert rc == G.GMM_ERR_NUMERIC and flags & G.GMM_DEVFLAG_NONFINITE_X
+    rc, flags = G.gmm_device_status(ws)  # cleared by the previous read
+    assert rc == 0 and flags == 0
+    Xd = torch.tensor(np.nan_to_num(X), device="cuda")
+    var[2, 3] = 0.0
+    G.gmm_em_step(Xd, w, mu, var, ws=ws)
+    rc, flags = G.gmm_device_status(ws)
+    assert rc == G.GMM_ERR_NUMERIC and flags & G.GMM_DEVFLAG_BAD_PARAMS
+
+
+def test_fit_matches_repeated_steps(G):
+    import torch
+
+    wl = synth.WORKLOADS["gauss8"]
+    X, _ = synth.make_data(wl)
+    Xd = to_device(wl, X)
+    ws = G.workspace(G.problem_for(Xd, wl.K))
+    rows = synth.init_rows(len(X), wl.K, wl.init_seed)
+    w, mu, var = G.gmm_init(Xd, rows, wl.K, G.GMM_INIT_VAR_ONE, ws=ws)
+    w1, mu1, var1 = w.clone(), mu.clone(), var.clone()
+    hist = G.gmm_fit(Xd, w, mu, var, wl.iters, ws=ws)
+    lls = []
+    for _ in range(wl.iters):
+        ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+        G.gmm_em_step(Xd, w1, mu1, var1, ll, ws=ws)
+        lls.append(ll.item())
+    assert torch.equal(w, w1) and torch.equal(mu, mu1) and torch.equal(var, var1)
+    np.testing.assert_array_equal(hist.cpu().numpy(), np.array(lls))
+    # LL of the GPU trajectory is monotone up to fp32 rounding
+    h = hist.cpu().numpy()
+    assert np.all(np.diff(h) >= -1e-6 * np.abs(h[1:]))
