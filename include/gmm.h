@@ -113,6 +113,36 @@ gmm_status gmm_em_step(const gmm_problem* p, const void* X, float* w, float* mu,
                        double* loglik, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * gmm_em_step without a caller-provided workspace, for callers that are not
+ * allowed to obtain device memory themselves: for example a plug-in running
+ * inside a host application that owns the whole device-memory budget and
+ * exposes no allocator, or a latency-bound loop that must not call cudaMalloc
+ * because it blocks the whole device.  It performs no device allocation of
+ * any kind (no cudaMalloc, no cudaFree, no allocating library routine).
+ * The Flash-GMM pages have no counterpart to this entry point.
+ *
+ * Scratch: a fixed 32 MiB array compiled into this library, present on every
+ * device that loads the library until the process exits.  The first call on a
+ * device looks up that array's device address (cudaGetSymbolAddress) and
+ * caches it; make that first call before any stream capture.  When the
+ * statistics slots of the regular workspace do not all fit, fewer CTAs run the
+ * fused pass (one slot each), which is slower but gives the same result up to
+ * summation order; a problem for which not even one slot fits
+ * (K*(2D+1)+1 doubles plus the parameter tables, above 32 MiB) is rejected with
+ * GMM_ERR_UNSUPPORTED and a message on stderr.
+ *
+ * Every call on a device uses the same array and it keeps the previous call's
+ * contents; each call resets the status word and rewrites everything else it
+ * reads.  Calls whose work overlaps on the GPU (different streams, or several
+ * host threads) race on the array and give wrong results: order them on one
+ * stream.  dev_flags (device, 1 uint32, may be NULL) receives this call's
+ * GMM_DEVFLAG_* bits.  Arguments, loglik and in-place updates are as for
+ * gmm_em_step.
+ */
+gmm_status gmm_em_step_noalloc(const gmm_problem* p, const void* X, float* w, float* mu,
+                               float* var, double* loglik, uint32_t* dev_flags, void* stream);
+
+/*
  * iters EM iterations in place.  ll_history (device, iters doubles, may be
  * NULL) receives LL(theta_t) for t = 0 .. iters-1, each of the parameters that
  * iteration started from.

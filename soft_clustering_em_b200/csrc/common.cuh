@@ -58,6 +58,18 @@ inline WsLayout ws_layout(int D, int K, int num_sms) {
   return L;
 }
 
+// The same layout with the number of slots cut down until the whole layout
+// fits in cap bytes (P = 0 when not even one slot fits).
+inline WsLayout ws_layout_capped(int D, int K, int num_sms, size_t cap) {
+  WsLayout L = ws_layout(D, K, num_sms);
+  const size_t fixed = L.slots;
+  const size_t per = L.slot_stride * 8;
+  size_t fit = cap > fixed ? (cap - fixed) / per : 0;
+  if ((size_t)L.P > fit) L.P = (int)fit;
+  L.total = align_up(fixed + (size_t)L.P * per, 256);
+  return L;
+}
+
 // Pointers into one workspace, passed to kernels by value.
 struct WsPtrs {
   unsigned int* status;

@@ -4,6 +4,8 @@
 // gmm_device_status.
 #include <stdio.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "gmm.h"
 #include "simt_em.cuh"
@@ -122,6 +124,40 @@ gmm_status em_step_impl(const gmm_problem* p, const void* X, float* w, float* mu
   return launched(1);
 }
 
+// ---------------------------------------------------------------------------
+// Scratch for gmm_em_step_noalloc: a fixed array in the module's own device
+// memory, so that entry point never asks for memory.  It exists on every
+// device that loads this library, for the life of the process.  Host code only
+// sees a host-side stand-in under this name; the device address comes from
+// cudaGetSymbolAddress, looked up once per device and cached.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoallocScratchBytes = (size_t)32 << 20;
+constexpr int kNoallocMaxDevices = 64;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+gmm_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return GMM_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kNoallocMaxDevices) return GMM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return GMM_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return GMM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -205,6 +241,41 @@ gmm_status gmm_em_step(const gmm_problem* p, const void* X, float* w, float* mu,
   WsLayout L;
   if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
   return em_step_impl(p, X, w, mu, var, loglik, ws_ptrs(ws, L), (cudaStream_t)stream);
+}
+
+gmm_status gmm_em_step_noalloc(const gmm_problem* p, const void* X, float* w, float* mu,
+                               float* var, double* loglik, uint32_t* dev_flags, void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if ((s = check_x(p, X)) != GMM_OK) return s;
+  if (!w || !mu || !var) return GMM_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((s = device_sms(&sms)) != GMM_OK) return s;
+  const WsLayout L = ws_layout_capped(p->D, p->K, sms, kNoallocScratchBytes);
+  if (L.P < 1) {
+    fprintf(stderr,
+            "gmm_em_step_noalloc: K=%d, D=%d needs %zu bytes of scratch for one statistics "
+            "slot; the built-in scratch holds %zu bytes\n",
+            p->K, p->D, L.slots + L.slot_stride * 8, kNoallocScratchBytes);
+    return GMM_ERR_UNSUPPORTED;
+  }
+  void* ws = nullptr;
+  if ((s = noalloc_scratch(&ws)) != GMM_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const WsPtrs wp = ws_ptrs(ws, L);
+  // the scratch keeps the previous call's bytes: only the status word must start at zero
+  // (prep rewrites every parameter table and the fused kernel zeroes its own slot)
+  if (cudaMemsetAsync(wp.status, 0, sizeof(uint32_t), st) != cudaSuccess) {
+    launch_status();
+    return GMM_ERR_CUDA;
+  }
+  if ((s = em_step_impl(p, X, w, mu, var, loglik, wp, st)) != GMM_OK) return s;
+  if (dev_flags && cudaMemcpyAsync(dev_flags, wp.status, sizeof(uint32_t),
+                                   cudaMemcpyDeviceToDevice, st) != cudaSuccess) {
+    launch_status();
+    return GMM_ERR_CUDA;
+  }
+  return GMM_OK;
 }
 
 gmm_status gmm_fit(const gmm_problem* p, const void* X, int32_t iters, float* w, float* mu,

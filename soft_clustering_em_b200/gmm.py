@@ -20,7 +20,8 @@ GMM_F32, GMM_BF16 = 0, 1
 GMM_INIT_VAR_ONE, GMM_INIT_VAR_DATA = 0, 1
 GMM_DEVFLAG_NONFINITE_X, GMM_DEVFLAG_BAD_PARAMS, GMM_DEVFLAG_WAIT_TIMEOUT = 0x1, 0x2, 0x4
 
-EXPORTS = ("gmm_workspace_size", "gmm_init", "gmm_em_step", "gmm_fit", "gmm_loglik",
+EXPORTS = ("gmm_workspace_size", "gmm_init", "gmm_em_step", "gmm_em_step_noalloc", "gmm_fit",
+           "gmm_loglik",
            "gmm_assign_topm", "gmm_device_status", "gmm_trace_fused", "gmm_launch_count",
            "gmm_status_string")
 
@@ -53,6 +54,7 @@ def load_library(path: str = LIB_PATH):
     lib.gmm_workspace_size.argtypes = [PP, ctypes.POINTER(SZ)]
     lib.gmm_init.argtypes = [PP, P, ctypes.POINTER(I64), I32, P, P, P, P, SZ, P]
     lib.gmm_em_step.argtypes = [PP, P, P, P, P, P, P, SZ, P]
+    lib.gmm_em_step_noalloc.argtypes = [PP, P, P, P, P, P, P, P]
     lib.gmm_fit.argtypes = [PP, P, I32, P, P, P, P, P, SZ, P]
     lib.gmm_loglik.argtypes = [PP, P, P, P, P, P, P, SZ, P]
     lib.gmm_assign_topm.argtypes = [PP, P, P, P, P, I32, P, P, P, SZ, P]
@@ -139,6 +141,19 @@ def gmm_em_step(X, w, mu, var, loglik=None, var_floor=1e-6, ws=None, stream=None
     _check(load_library().gmm_em_step(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu), _ptr(var),
                                       _ptr(loglik), _ptr(ws), ws.numel(), _stream(stream)),
            "gmm_em_step")
+
+
+def gmm_em_step_noalloc(X, w, mu, var, loglik=None, dev_flags=None, var_floor=1e-6,
+                        stream=None):
+    """gmm_em_step on the library's built-in scratch: no workspace, no device allocation.
+
+    For callers that may not obtain device memory (see include/gmm.h).  dev_flags
+    (1 int32 device tensor, optional) receives the call's device status bits.
+    """
+    p = problem_for(X, w.numel(), var_floor)
+    _check(load_library().gmm_em_step_noalloc(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu),
+                                              _ptr(var), _ptr(loglik), _ptr(dev_flags),
+                                              _stream(stream)), "gmm_em_step_noalloc")
 
 
 def gmm_fit(X, w, mu, var, iters, var_floor=1e-6, ws=None, stream=None):

@@ -27,9 +27,9 @@ def declared_functions():
 
 def test_header_declares_the_calls():
     names = declared_functions()
-    for n in ("gmm_init", "gmm_em_step", "gmm_fit", "gmm_loglik", "gmm_assign_topm",
-              "gmm_workspace_size", "gmm_device_status", "gmm_trace_fused",
-              "gmm_status_string"):
+    for n in ("gmm_init", "gmm_em_step", "gmm_em_step_noalloc", "gmm_fit", "gmm_loglik",
+              "gmm_assign_topm", "gmm_workspace_size", "gmm_device_status", "gmm_trace_fused",
+              "gmm_launch_count", "gmm_status_string"):
         assert n in names
 
 
