@@ -82,6 +82,9 @@ typedef struct {
 #define GMM_DEVFLAG_NONFINITE_X 0x1u     /* a NaN or Inf element in X */
 #define GMM_DEVFLAG_BAD_PARAMS 0x2u      /* w < 0, var <= 0 or a non-finite parameter */
 #define GMM_DEVFLAG_WAIT_TIMEOUT 0x4u    /* a bounded spin on a barrier gave up */
+#define GMM_DEVFLAG_X_RANGE 0x8u         /* an element of X lies so far from the mixture mean
+                                            (over 240 scale units, about 480 mixture standard
+                                            deviations) that the tensor-core path clipped it */
 
 /*
  * Bytes of device workspace needed for problem p on the CURRENT device.
@@ -170,7 +173,7 @@ gmm_status gmm_assign_topm(const gmm_problem* p, const void* X, const float* w,
 /*
  * Waits for stream, then reads the device status word of ws into *flags
  * (GMM_DEVFLAG_* bits; may be NULL) and, if clear != 0, resets it to 0.
- * Returns GMM_OK when no bit is set, GMM_ERR_NUMERIC for the data/parameter
+ * Returns GMM_OK when no bit is set, GMM_ERR_NUMERIC for the data/parameter/range
  * bits, GMM_ERR_TIMEOUT for the wait bit.  The only entry point that blocks.
  */
 gmm_status gmm_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* flags,

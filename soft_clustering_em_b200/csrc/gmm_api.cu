@@ -3,12 +3,17 @@
 // Nothing here allocates device memory or synchronises, except
 // gmm_device_status.
 #include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
 #include "gmm.h"
 #include "simt_em.cuh"
+#include "tc_em.cuh"
+#include "tma_host.h"
 
 using namespace scem;
 
@@ -46,12 +51,41 @@ gmm_status device_sms(int* sms) {
   return GMM_OK;
 }
 
-gmm_status get_layout(const gmm_problem* p, void* ws, size_t ws_bytes, WsLayout* L) {
+// Which kernels a problem runs and where their data sits in the workspace.
+// The CUDA-core layout always exists (top-m and init use it); the tensor-core
+// layout exists when the shape fits that kernel.  Both start at offset 256,
+// after the shared status word, and the workspace covers the larger one.
+struct Plan {
+  WsLayout simt;
+  TcLayout tc;
+  bool use_tc;
+  size_t total;
+};
+
+bool force_cuda_core_path() {
+  const char* e = getenv("SCEM_GMM_PATH");
+  return e && strcmp(e, "simt") == 0;
+}
+
+Plan make_plan(const gmm_problem* p, int sms, size_t cap) {
+  Plan P;
+  P.simt = cap ? ws_layout_capped(p->D, p->K, sms, cap) : ws_layout(p->D, p->K, sms);
+  P.use_tc = tc_shape_ok(p->D, p->K) && !force_cuda_core_path();
+  if (P.use_tc) {
+    P.tc = tc_layout(p->D, p->K, sms, cap);
+    if (P.tc.P < 1) P.use_tc = false;
+  }
+  P.total = P.simt.P >= 1 ? P.simt.total : 0;
+  if (P.use_tc) P.total = std::max(P.total, P.tc.total);
+  return P;
+}
+
+gmm_status get_plan(const gmm_problem* p, void* ws, size_t ws_bytes, Plan* P) {
   int sms = 0;
   gmm_status s = device_sms(&sms);
   if (s != GMM_OK) return s;
-  *L = ws_layout(p->D, p->K, sms);
-  if (!ws || ((uintptr_t)ws) % 256 != 0 || ws_bytes < L->total) return GMM_ERR_WORKSPACE;
+  *P = make_plan(p, sms, 0);
+  if (!ws || ((uintptr_t)ws) % 256 != 0 || ws_bytes < P->total) return GMM_ERR_WORKSPACE;
   return GMM_OK;
 }
 
@@ -112,15 +146,137 @@ gmm_status prep(const gmm_problem* p, const float* w, const float* mu, const flo
   return launched(1);
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core path
+// ---------------------------------------------------------------------------
+constexpr uint64_t kWaitBudgetNs = 1000000000ull;  // 1 s per device-side wait
+
+// Tiles whose statistics accumulate in fp32 tensor memory before an fp64
+// drain (SCEM_GMM_DRAIN_TILES overrides the default, for tuning).
+int tc_drain_tiles() {
+  const char* e = getenv("SCEM_GMM_DRAIN_TILES");
+  const int v = e ? atoi(e) : 0;
+  return v >= 1 && v <= 1024 ? v : kTcDrainTiles;
+}
+
+gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const float* var,
+                   char* ws, const TcLayout& T, cudaStream_t st) {
+  float* m = (float*)(ws + T.m);
+  tc_center_kernel<<<(p->D + 127) / 128, 128, 0, st>>>(p->D, p->K, w, mu, var, m,
+                                                       (float*)(ws + T.isc), (float*)(ws + T.sc));
+  tc_prep_w_kernel<<<T.Kpad, 128, 0, st>>>(
+      p->N, p->D, p->K, T.Fpad, w, mu, var, m, (const float*)(ws + T.sc), (__half*)(ws + T.whi),
+      (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.cd), (float*)(ws + T.wsc),
+      (int*)(ws + T.sharp), (float*)(ws + T.muh), (float*)(ws + T.ph), (unsigned int*)ws);
+  return launched(2);
+}
+
+template <typename XT, int MODE>
+gmm_status tc_launch(const gmm_problem* p, const void* X, char* ws, const TcLayout& T,
+                     cudaStream_t st, int* nslots) {
+  CUtensorMap mhi, mlo;
+  memset(&mhi, 0, sizeof(mhi));
+  memset(&mlo, 0, sizeof(mlo));
+  if (!make_tmap_16b_sw128(&mhi, ws + T.whi, (uint64_t)T.Fpad, (uint64_t)T.Kpad,
+                            (uint64_t)T.Fpad * 2, kTcComps) ||
+      !make_tmap_16b_sw128(&mlo, ws + T.wlo, (uint64_t)T.Fpad, (uint64_t)T.Kpad,
+                            (uint64_t)T.Fpad * 2, kTcComps))
+    return GMM_ERR_CUDA;
+  const TcSmem S = tc_smem_layout(p->D, T.C, T.nchunks);
+  // at least 120 KB so that exactly one CTA (and one 512-column TMEM allocation) sits on an SM
+  const size_t smem = std::max<size_t>(S.total, 120 * 1024);
+  auto kern = tc_fused_kernel<XT, MODE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return GMM_ERR_UNSUPPORTED;
+  }
+  if (T.C > 8 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    cudaGetLastError();
+    return GMM_ERR_UNSUPPORTED;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)T.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.blockDim = dim3(kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.gridDim = dim3((unsigned)(T.C * T.P), 1, 1);
+  int max_clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&max_clusters, (void*)kern, &cfg) != cudaSuccess ||
+      max_clusters < 1) {
+    cudaGetLastError();
+    return GMM_ERR_UNSUPPORTED;
+  }
+  const int64_t ntiles = (p->N + kTcRows - 1) / kTcRows;
+  const int ncl = (int)std::min<int64_t>(std::min(T.P, max_clusters), ntiles);
+  cfg.gridDim = dim3((unsigned)(T.C * ncl), 1, 1);
+  TcArgs args;
+  args.X = X;
+  args.N = p->N;
+  args.D = p->D;
+  args.K = p->K;
+  args.C = T.C;
+  args.nchunks = T.nchunks;
+  args.m = (const float*)(ws + T.m);
+  args.isc = (const float*)(ws + T.isc);
+  args.c = (const float*)(ws + T.c);
+  args.cd = (const float*)(ws + T.cd);
+  args.wsc = (const float*)(ws + T.wsc);
+  args.sharp = (const int*)(ws + T.sharp);
+  args.muh = (const float*)(ws + T.muh);
+  args.ph = (const float*)(ws + T.ph);
+  args.slots = (double*)(ws + T.slots);
+  args.slot_stride = T.slot_stride;
+  args.status = (unsigned int*)ws;
+  args.drain_tiles = tc_drain_tiles();
+  args.wait_ns = kWaitBudgetNs;
+  trace_begin(st);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args, mhi, mlo);
+  trace_end(st);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "gmm: tensor-core launch failed: %s\n", cudaGetErrorString(e));
+    cudaGetLastError();
+    return GMM_ERR_CUDA;
+  }
+  *nslots = ncl;
+  return launched(1);
+}
+
+template <int MODE>
+gmm_status tc_pass(const gmm_problem* p, const void* X, char* ws, const TcLayout& T,
+                   cudaStream_t st, int* nslots) {
+  if (p->xdtype == GMM_BF16) return tc_launch<__nv_bfloat16, MODE>(p, X, ws, T, st, nslots);
+  return tc_launch<float, MODE>(p, X, ws, T, st, nslots);
+}
+
 gmm_status em_step_impl(const gmm_problem* p, const void* X, float* w, float* mu, float* var,
-                        double* loglik, const WsPtrs& ws, cudaStream_t st) {
-  gmm_status s = prep(p, w, mu, var, ws, st);
-  if (s != GMM_OK) return s;
-  s = fused_pass<kModeStats>(p, X, ws, 0, nullptr, nullptr, st);
-  if (s != GMM_OK) return s;
+                        double* loglik, void* ws_base, const Plan& P, cudaStream_t st) {
+  char* ws = (char*)ws_base;
+  gmm_status s;
+  if (P.use_tc) {
+    const TcLayout& T = P.tc;
+    if ((s = tc_prep(p, w, mu, var, ws, T, st)) != GMM_OK) return s;
+    int nslots = 0;
+    if ((s = tc_pass<kTcStats>(p, X, ws, T, st, &nslots)) != GMM_OK) return s;
+    const size_t KD = (size_t)p->K * p->D;
+    tc_reduce_mstep_kernel<<<(unsigned)((KD + 255) / 256), 256, 0, st>>>(
+        p->N, p->D, p->K, p->var_floor, (const float*)(ws + T.m), (const float*)(ws + T.sc),
+        (const double*)(ws + T.slots), T.slot_stride, nslots, w, mu, var, loglik);
+    return launched(1);
+  }
+  const WsPtrs wp = ws_ptrs(ws_base, P.simt);
+  if ((s = prep(p, w, mu, var, wp, st)) != GMM_OK) return s;
+  if ((s = fused_pass<kModeStats>(p, X, wp, 0, nullptr, nullptr, st)) != GMM_OK) return s;
   const size_t KD = (size_t)p->K * p->D;
   reduce_mstep_kernel<<<(unsigned)((KD + 255) / 256), 256, 0, st>>>(p->N, p->D, p->K, p->var_floor,
-                                                                    ws, w, mu, var, loglik);
+                                                                    wp, w, mu, var, loglik);
   return launched(1);
 }
 
@@ -182,7 +338,7 @@ gmm_status gmm_workspace_size(const gmm_problem* p, size_t* bytes) {
   int sms = 0;
   s = device_sms(&sms);
   if (s != GMM_OK) return s;
-  *bytes = ws_layout(p->D, p->K, sms).total;
+  *bytes = make_plan(p, sms, 0).total;
   return GMM_OK;
 }
 
@@ -196,9 +352,9 @@ gmm_status gmm_init(const gmm_problem* p, const void* X, const int64_t* rows_hos
   if (init_var != GMM_INIT_VAR_ONE && init_var != GMM_INIT_VAR_DATA) return GMM_ERR_INVALID_ARG;
   for (int k = 0; k < p->K; k++)
     if (rows_host[k] < 0 || rows_host[k] >= p->N) return GMM_ERR_INVALID_ARG;
-  WsLayout L;
-  if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
-  WsPtrs wp = ws_ptrs(ws, L);
+  Plan P;
+  if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  WsPtrs wp = ws_ptrs(ws, P.simt);
   cudaStream_t st = (cudaStream_t)stream;
   // the K row indices travel to the workspace (the one host->device copy of this call)
   if (cudaMemcpyAsync(wp.scratch, rows_host, sizeof(int64_t) * p->K, cudaMemcpyHostToDevice, st) !=
@@ -238,9 +394,9 @@ gmm_status gmm_em_step(const gmm_problem* p, const void* X, float* w, float* mu,
   if (s != GMM_OK) return s;
   if ((s = check_x(p, X)) != GMM_OK) return s;
   if (!w || !mu || !var) return GMM_ERR_INVALID_ARG;
-  WsLayout L;
-  if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
-  return em_step_impl(p, X, w, mu, var, loglik, ws_ptrs(ws, L), (cudaStream_t)stream);
+  Plan P;
+  if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  return em_step_impl(p, X, w, mu, var, loglik, ws, P, (cudaStream_t)stream);
 }
 
 gmm_status gmm_em_step_noalloc(const gmm_problem* p, const void* X, float* w, float* mu,
@@ -251,26 +407,26 @@ gmm_status gmm_em_step_noalloc(const gmm_problem* p, const void* X, float* w, fl
   if (!w || !mu || !var) return GMM_ERR_INVALID_ARG;
   int sms = 0;
   if ((s = device_sms(&sms)) != GMM_OK) return s;
-  const WsLayout L = ws_layout_capped(p->D, p->K, sms, kNoallocScratchBytes);
-  if (L.P < 1) {
+  const Plan P = make_plan(p, sms, kNoallocScratchBytes);
+  if (!P.use_tc && P.simt.P < 1) {
     fprintf(stderr,
             "gmm_em_step_noalloc: K=%d, D=%d needs %zu bytes of scratch for one statistics "
             "slot; the built-in scratch holds %zu bytes\n",
-            p->K, p->D, L.slots + L.slot_stride * 8, kNoallocScratchBytes);
+            p->K, p->D, P.simt.slots + P.simt.slot_stride * 8, kNoallocScratchBytes);
     return GMM_ERR_UNSUPPORTED;
   }
   void* ws = nullptr;
   if ((s = noalloc_scratch(&ws)) != GMM_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
-  const WsPtrs wp = ws_ptrs(ws, L);
+  unsigned int* status = (unsigned int*)ws;
   // the scratch keeps the previous call's bytes: only the status word must start at zero
   // (prep rewrites every parameter table and the fused kernel zeroes its own slot)
-  if (cudaMemsetAsync(wp.status, 0, sizeof(uint32_t), st) != cudaSuccess) {
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) {
     launch_status();
     return GMM_ERR_CUDA;
   }
-  if ((s = em_step_impl(p, X, w, mu, var, loglik, wp, st)) != GMM_OK) return s;
-  if (dev_flags && cudaMemcpyAsync(dev_flags, wp.status, sizeof(uint32_t),
+  if ((s = em_step_impl(p, X, w, mu, var, loglik, ws, P, st)) != GMM_OK) return s;
+  if (dev_flags && cudaMemcpyAsync(dev_flags, status, sizeof(uint32_t),
                                    cudaMemcpyDeviceToDevice, st) != cudaSuccess) {
     launch_status();
     return GMM_ERR_CUDA;
@@ -284,11 +440,10 @@ gmm_status gmm_fit(const gmm_problem* p, const void* X, int32_t iters, float* w,
   if (s != GMM_OK) return s;
   if ((s = check_x(p, X)) != GMM_OK) return s;
   if (!w || !mu || !var || iters < 0) return GMM_ERR_INVALID_ARG;
-  WsLayout L;
-  if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
-  const WsPtrs wp = ws_ptrs(ws, L);
+  Plan P;
+  if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
   for (int t = 0; t < iters; t++) {
-    s = em_step_impl(p, X, w, mu, var, ll_history ? ll_history + t : nullptr, wp,
+    s = em_step_impl(p, X, w, mu, var, ll_history ? ll_history + t : nullptr, ws, P,
                      (cudaStream_t)stream);
     if (s != GMM_OK) return s;
   }
@@ -301,10 +456,20 @@ gmm_status gmm_loglik(const gmm_problem* p, const void* X, const float* w, const
   if (s != GMM_OK) return s;
   if ((s = check_x(p, X)) != GMM_OK) return s;
   if (!w || !mu || !var || !loglik) return GMM_ERR_INVALID_ARG;
-  WsLayout L;
-  if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
-  const WsPtrs wp = ws_ptrs(ws, L);
+  Plan P;
+  if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
+  if (P.use_tc) {
+    char* wsb = (char*)ws;
+    const TcLayout& T = P.tc;
+    if ((s = tc_prep(p, w, mu, var, wsb, T, st)) != GMM_OK) return s;
+    int nslots = 0;
+    if ((s = tc_pass<kTcLoglik>(p, X, wsb, T, st, &nslots)) != GMM_OK) return s;
+    tc_reduce_loglik_kernel<<<1, 1, 0, st>>>(p->D, p->K, (const double*)(wsb + T.slots),
+                                             T.slot_stride, nslots, loglik);
+    return launched(1);
+  }
+  const WsPtrs wp = ws_ptrs(ws, P.simt);
   if ((s = prep(p, w, mu, var, wp, st)) != GMM_OK) return s;
   if ((s = fused_pass<kModeLoglik>(p, X, wp, 0, nullptr, nullptr, st)) != GMM_OK) return s;
   reduce_loglik_kernel<<<1, 1, 0, st>>>(p->D, p->K, wp, loglik);
@@ -319,9 +484,9 @@ gmm_status gmm_assign_topm(const gmm_problem* p, const void* X, const float* w, 
   if ((s = check_x(p, X)) != GMM_OK) return s;
   if (!w || !mu || !var || !idx || !resp) return GMM_ERR_INVALID_ARG;
   if (m < 1 || m > kMaxTopM || m > p->K) return GMM_ERR_INVALID_ARG;
-  WsLayout L;
-  if ((s = get_layout(p, ws, ws_bytes, &L)) != GMM_OK) return s;
-  const WsPtrs wp = ws_ptrs(ws, L);
+  Plan P;
+  if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  const WsPtrs wp = ws_ptrs(ws, P.simt);
   cudaStream_t st = (cudaStream_t)stream;
   if ((s = prep(p, w, mu, var, wp, st)) != GMM_OK) return s;
   return fused_pass<kModeTopm>(p, X, wp, m, idx, resp, st);
@@ -352,7 +517,8 @@ gmm_status gmm_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* 
     return launch_status(), GMM_ERR_CUDA;
   if (flags) *flags = f;
   if (f & GMM_DEVFLAG_WAIT_TIMEOUT) return GMM_ERR_TIMEOUT;
-  if (f & (GMM_DEVFLAG_NONFINITE_X | GMM_DEVFLAG_BAD_PARAMS)) return GMM_ERR_NUMERIC;
+  if (f & (GMM_DEVFLAG_NONFINITE_X | GMM_DEVFLAG_BAD_PARAMS | GMM_DEVFLAG_X_RANGE))
+    return GMM_ERR_NUMERIC;
   return GMM_OK;
 }
 

@@ -104,20 +104,37 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
-// Bounded wait: spins at most `limit` times (each try_wait also suspends in
-// hardware for a while); on expiry sets the abort word (if not already set)
-// and returns false.  A set abort word makes every later wait give up at once.
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on phase `parity` of `bar`.  Gives up after budget_ns of wall
+// time, or as soon as another thread has set any bit of `abort_mask` in
+// *status (abort_mask = 0: wait out the full budget regardless); on its own
+// expiry it sets `expire_bit` in *status.  Returns true iff the phase completed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile unsigned int* abort_word,
-                                                  unsigned int abort_value, uint32_t limit,
-                                                  bool cluster_scope = false) {
-  for (uint32_t i = 0; i < limit; i++) {
-    const bool done = cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+                                                  volatile unsigned int* status,
+                                                  unsigned int abort_mask, uint64_t budget_ns,
+                                                  bool cluster_scope = false,
+                                                  unsigned int expire_bit = 0x4u) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 0;; i++) {
+    const bool done =
+        cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
     if (done) return true;
-    if ((i & 63) == 63 && *abort_word != 0u) return false;
+    if ((i & 15) == 0) {
+      if (*status & abort_mask) return false;
+      const uint64_t now = globaltimer_ns();
+      if (i == 0) {
+        t0 = now;
+      } else if (now - t0 > budget_ns) {
+        atomicOr(const_cast<unsigned int*>(status), expire_bit);
+        return false;
+      }
+    }
   }
-  atomicOr(const_cast<unsigned int*>(abort_word), abort_value);
-  return false;
 }
 
 // ---------------------------------------------------------------- proxies / fences
@@ -191,6 +208,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; i++) v[i] = __uint_as_float(r[i]);
 }
 
+// Each thread of the warp writes one 32-bit value to column `taddr`'s column
+// of its own lane (32 lanes x 1 column), and waits for the store to land.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "r"(__float_as_uint(v))
+      : "memory");
+}
+
 // ---------------------------------------------------------------- MMA
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand (tcgen05
 // format: start address, leading and stride byte offsets in 16-byte units,
@@ -218,6 +245,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
          | ((b_mn ? 1u : 0u) << 16)        // B major-ness
          | ((uint32_t)(N >> 3) << 17)      // N / 8
          | ((uint32_t)(M >> 4) << 24);     // M / 16
+}
+
+// Instruction descriptor for kind::f16 with FP16 A and B and an FP32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4)                         // D format: F32 (A, B format fields 0 = F16)
+         | ((a_mn ? 1u : 0u) << 15)
+         | ((b_mn ? 1u : 0u) << 16)
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
 }
 
 // D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread; accumulate = false

@@ -1,0 +1,818 @@
+// tc_em.cuh -- the fused EM pass on the 5th-generation tensor cores (sm_100a).
+//
+// Method: "Flash-GMM: A Memory-Efficient Kernel for Scalable Soft Clustering"
+// (review page, section 3): per data tile, the E-step log-densities, the
+// per-point log-sum-exp into responsibilities and the tile's share of the
+// M-step statistics are formed on chip; only O(K*D) statistics reach memory.
+//
+// Expanded E-step.  With a centring vector m (the mixture mean) and a
+// power-of-two scale s_d (about twice the mixture's standard deviation, so the
+// scaling is exact), x^ = (x - m)/s, mu^ = (mu - m)/s, var^ = var/s^2, every
+// log-joint is one dense contraction over the 2D features F = [x^, x^^2]:
+//   l_nk = c_k + sum_d x^_nd a_kd + sum_d x^_nd^2 b_kd,
+//   a_kd = mu^_kd / var^_kd,  b_kd = -1 / (2 var^_kd),
+//   c_k  = log pi_k - 1/2 sum_d (log(2 pi var_kd) + mu^_kd^2 / var^_kd).
+// F and W = [a, b] are split into fp16 pairs (hi + lo, 22 significant bits;
+// each W row carries its own power-of-two scale so it sits in fp16 range) and
+// the contraction takes F_hi W_hi + F_lo W_hi + F_hi W_lo (the lo*lo term is
+// below fp32 rounding), accumulated in fp32 in tensor memory.
+//
+// Sharp components.  The expanded form cancels: its fp32 error grows with
+// kappa_k = sum_d (mu^_kd^2 + 1) / var^_kd, up to ~1e-3 nat at kappa ~ 1e5.
+// A component with kappa_k > 1e7 (in practice one collapsed onto a few points,
+// at the variance floor), or with kappa_k > 3e3 while it expects fewer than 20
+// points (pi_k N < 20, where such an error moves its weight by ~1e-3), gets its
+// log-joints recomputed in direct form, sum_d (x^ - mu^)^2 / var^, on the CUDA
+// cores and written over the tensor-core value in tensor memory.
+//
+// Statistics.  r is scaled by 2^15 and split into an fp16 pair r^ = r_hi +
+// r_lo (about 22 significant bits; fp16 alone leaves components that hold a
+// point or two with weight errors near 1e-3); the same r^ gives
+//   N_k = sum_n r^_nk,  S1_kd = sum_n r^_nk x^_nd,  S2_kd = sum_n r^_nk x^_nd^2
+// as r_hi^T (F_hi + F_lo) + r_lo^T F_hi and r^T 1 on the tensor cores,
+// accumulated in fp32 in tensor memory over a few tiles and then added into
+// fp64 per-cluster slots.  The M-step undoes the scales exactly.  r^ passes
+// through one 32 KB buffer in two 64-row halves: rows 0-63 first, then rows
+// 64-127 once the MMAs of the first half have released it.
+//
+// Work split.  A cluster of C = ceil(K/128) CTAs takes one 128-row tile at a
+// time; CTA `rank` owns components [128 rank, 128 rank + 128).  Per tile each
+// CTA converts X into F (shared memory), runs the E-step MMAs for its 128
+// components (W streamed by TMA through a 3-stage ring), reduces each row's
+// max / sum-exp over its components, exchanges those with the other CTAs of
+// the cluster through distributed shared memory, forms r^ and runs the
+// statistics MMAs.  Warps 0-3: conversion, epilogue, drains (warp w owns
+// tensor-memory lanes 32w..32w+31); warp 4: MMA issue; warp 5: TMA issue.
+//
+// Tensor memory (512 columns): L logits [0,128); S statistics
+// [128, 128 + 64*nchunks); N_k [128 + 64*nchunks, +16).
+#pragma once
+
+#include <math.h>
+
+#include "common.cuh"
+#include "sm100_prims.cuh"
+
+namespace scem {
+
+constexpr int kTcRows = 128;      // rows per tile (= tensor-memory lanes)
+constexpr int kTcComps = 128;     // components per CTA
+constexpr int kTcChunk = 64;      // features per operand chunk (one swizzled 128-byte row)
+constexpr int kTcStages = 3;      // depth of the W ring
+constexpr int kTcMaxChunks = 4;   // 2D <= 256
+constexpr int kTcMaxCluster = 16;
+constexpr int kTcThreads = 192;
+constexpr int kTcDrainTiles = 8;  // tiles accumulated in fp32 before an fp64 drain
+constexpr uint32_t kTcChunkBytes = 128u * 128u;  // one [128 x 64] 16-bit operand chunk
+constexpr float kTcRScale = 32768.0f;            // r is stored as fp16(r * 2^15)
+constexpr double kTcSharpKappa = 1e7;            // direct form above this kappa_k ...
+constexpr double kTcSmallKappa = 3e3;            // ... or above this one for a component
+constexpr double kTcSmallPoints = 20.0;          //     expecting fewer points than this
+constexpr float kTcXMax = 240.0f;                // |x^| beyond this cannot be split into fp16
+
+enum TcMode { kTcStats = 0, kTcLoglik = 1 };
+
+inline int tc_nchunks(int D) { return (2 * D + kTcChunk - 1) / kTcChunk; }
+inline int tc_cluster(int K) { return (K + kTcComps - 1) / kTcComps; }
+
+// Byte offsets of the kernel's shared-memory regions (from a 1024-aligned base).
+struct TcSmem {
+  uint32_t F, W, R, ONES, msm, iscs, csm, wscs, cds, shl, xchg, bars, tslot, total;
+};
+
+__host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
+  TcSmem L;
+  uint32_t off = 0;
+  L.F = off;
+  off += 2u * nchunks * kTcChunkBytes;
+  L.W = off;
+  off += kTcStages * kTcChunkBytes;
+  L.R = off;
+  off += 2u * kTcChunkBytes;
+  L.ONES = off;
+  off += 4096;
+  L.msm = off;
+  off += ((uint32_t)D * 4 + 15) & ~15u;
+  L.iscs = off;
+  off += ((uint32_t)D * 4 + 15) & ~15u;
+  L.csm = off;
+  off += kTcComps * 4;
+  L.wscs = off;
+  off += kTcComps * 4;
+  L.cds = off;
+  off += kTcComps * 4;
+  L.shl = off;
+  off += (kTcComps + 4) * 4;
+  L.xchg = off;
+  off += 2u * C * kTcRows * 8;
+  L.bars = off;
+  off += 8 * (2 * kTcStages + 10);
+  L.tslot = off;
+  off += 16;
+  L.total = off + 1024;  // slack for aligning the dynamic base to 1024
+  return L;
+}
+
+// Workspace layout of the tensor-core path (after the 256-byte status block).
+//   m, isc, sc : D f32 centring vector, 1/s and s (powers of two)
+//   c    : C*128 f32 per-component constants of the expanded form (0 if sharp)
+//   cd   : C*128 f32 per-component constants of the direct form
+//   wsc  : C*128 f32 power-of-two scale of each W row (1 if sharp)
+//   sharp: C*128 int32 1 if the component's log-joints are computed in direct form
+//   muh, ph : [C*128 x D] f32 mu^ and 1/var^ for the direct form
+//   whi, wlo : [C*128 x 64*nchunks] fp16 operand W (hi and lo parts)
+//   slots: P per-cluster slots of slot_stride doubles:
+//          [(2D+1) x K] feature-major statistics (S1 rows 0..D-1, S2 rows
+//          D..2D-1, N_k row 2D) followed by the cluster's LL.
+struct TcLayout {
+  size_t m, isc, sc, c, cd, wsc, sharp, muh, ph, whi, wlo, slots, total, slot_stride;
+  int C, nchunks, Kpad, Fpad, P;
+};
+
+inline bool tc_shape_ok(int D, int K) {
+  if (!(D >= 4 && D <= 128 && D % 4 == 0 && K >= 1 && K <= kTcComps * kTcMaxCluster))
+    return false;
+  return tc_smem_layout(D, tc_cluster(K), tc_nchunks(D)).total <= 232448;  // 227 KB per CTA
+}
+
+inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
+  TcLayout L;
+  L.C = tc_cluster(K);
+  L.nchunks = tc_nchunks(D);
+  L.Kpad = L.C * kTcComps;
+  L.Fpad = L.nchunks * kTcChunk;
+  size_t off = 256;
+  L.m = off;
+  off = align_up(off + (size_t)D * 4, 256);
+  L.isc = off;
+  off = align_up(off + (size_t)D * 4, 256);
+  L.sc = off;
+  off = align_up(off + (size_t)D * 4, 256);
+  L.c = off;
+  off = align_up(off + (size_t)L.Kpad * 4, 256);
+  L.cd = off;
+  off = align_up(off + (size_t)L.Kpad * 4, 256);
+  L.wsc = off;
+  off = align_up(off + (size_t)L.Kpad * 4, 256);
+  L.sharp = off;
+  off = align_up(off + (size_t)L.Kpad * 4, 256);
+  L.muh = off;
+  off = align_up(off + (size_t)L.Kpad * D * 4, 256);
+  L.ph = off;
+  off = align_up(off + (size_t)L.Kpad * D * 4, 256);
+  L.whi = off;
+  off = align_up(off + (size_t)L.Kpad * L.Fpad * 2, 256);
+  L.wlo = off;
+  off = align_up(off + (size_t)L.Kpad * L.Fpad * 2, 256);
+  L.slot_stride = align_up((size_t)(2 * D + 1) * K + 1, 32);
+  L.slots = off;
+  L.P = num_sms / L.C;
+  if (cap) {
+    const size_t per = L.slot_stride * 8;
+    const size_t fit = cap > off ? (cap - off) / per : 0;
+    if ((size_t)L.P > fit) L.P = (int)fit;
+  }
+  L.total = align_up(off + (size_t)L.P * L.slot_stride * 8, 256);
+  return L;
+}
+
+struct TcArgs {
+  const void* X;
+  int64_t N;
+  int D, K, C, nchunks;
+  const float* m;       // centring vector, D
+  const float* isc;     // 1/s, D
+  const float* c;       // expanded-form constants, C*128 (-inf for padding / pi = 0)
+  const float* cd;      // direct-form constants, C*128
+  const float* wsc;     // W row scales, C*128
+  const int* sharp;     // direct-form flags, C*128
+  const float* muh;     // mu^, C*128 x D
+  const float* ph;      // 1/var^, C*128 x D
+  double* slots;        // per-cluster statistic slots
+  size_t slot_stride;   // doubles per slot: (2D+1)*K statistics + LL
+  unsigned int* status;
+  int drain_tiles;
+  uint64_t wait_ns;
+};
+
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float round_half(float a) { return __half2float(__float2half_rn(a)); }
+
+template <typename XT>
+__device__ __forceinline__ void load4(const XT* X, size_t i, float (&x)[4]);
+template <>
+__device__ __forceinline__ void load4<float>(const float* X, size_t i, float (&x)[4]) {
+  const float4 v = __ldg(reinterpret_cast<const float4*>(X + i));
+  x[0] = v.x;
+  x[1] = v.y;
+  x[2] = v.z;
+  x[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* X, size_t i,
+                                                      float (&x)[4]) {
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(X + i));
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+  x[0] = __low2float(a);
+  x[1] = __high2float(a);
+  x[2] = __low2float(b);
+  x[3] = __high2float(b);
+}
+
+template <typename XT, int MODE>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    tc_fused_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tm_whi,
+                    const __grid_constant__ CUtensorMap tm_wlo) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const int D = a.D, K = a.K, C = a.C, nch = a.nchunks;
+  const TcSmem L = tc_smem_layout(D, C, nch);
+  uint8_t* sF = sm + L.F;  // [hi|lo][chunk] x [128 rows x 64 features]
+  uint8_t* sW = sm + L.W;  // ring of [128 components x 64 features]
+  uint8_t* sR = sm + L.R;  // r_hi | r_lo, each [64 rows] x [128 components] (two 64-wide MN atoms)
+  uint8_t* sOnes = sm + L.ONES;
+  float* msm = reinterpret_cast<float*>(sm + L.msm);
+  float* iscs = reinterpret_cast<float*>(sm + L.iscs);
+  float* csm = reinterpret_cast<float*>(sm + L.csm);
+  float* wscs = reinterpret_cast<float*>(sm + L.wscs);
+  float* cds = reinterpret_cast<float*>(sm + L.cds);
+  int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = local indices
+  float2* xchg = reinterpret_cast<float2*>(sm + L.xchg);  // [2][C][128] (row max, row sum-exp)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kTcStages;
+  uint64_t* f_full = bars + 2 * kTcStages;
+  uint64_t* l_full = f_full + 1;
+  uint64_t* r_full = f_full + 2;
+  uint64_t* s_done = f_full + 3;
+  uint64_t* drained = f_full + 4;
+  uint64_t* xbar = f_full + 5;  // [2]
+  uint64_t* final_bar = f_full + 7;
+  uint64_t* r_full1 = f_full + 8;  // second 64-row half of r^ written
+  uint64_t* r_free = f_full + 9;   // MMAs of the first half done with the r^ buffer
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tslot);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t cid = cluster_id_x(), ncl = nclusters_x();
+  const int64_t ntiles = (a.N + kTcRows - 1) / kTcRows;
+  const int64_t my_tiles = ((int64_t)cid < ntiles) ? (ntiles - 1 - (int64_t)cid) / ncl + 1 : 0;
+  const int k0 = (int)rank * kTcComps;
+  volatile unsigned int* status = a.status;
+  constexpr unsigned int kAbort = GMM_DEVFLAG_WAIT_TIMEOUT;
+  double* slot = a.slots + (size_t)cid * a.slot_stride;
+  const size_t ll_index = (size_t)(2 * D + 1) * K;
+
+  // ---------------------------------------------------------------- set-up
+  if (tid == 0) {
+    for (int s = 0; s < kTcStages; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(f_full, 128);
+    mbar_init(l_full, 1);
+    mbar_init(r_full, 64);
+    mbar_init(r_full1, 64);
+    mbar_init(r_free, 1);
+    mbar_init(s_done, 1);
+    mbar_init(drained, 128);
+    mbar_init(&xbar[0], (uint32_t)C * 128);
+    mbar_init(&xbar[1], (uint32_t)C * 128);
+    mbar_init(final_bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  for (int i = tid; i < D; i += kTcThreads) {
+    msm[i] = a.m[i];
+    iscs[i] = a.isc[i];
+  }
+  for (int i = tid; i < kTcComps; i += kTcThreads) {
+    csm[i] = a.c[k0 + i];
+    wscs[i] = a.wsc[k0 + i];
+    cds[i] = a.cd[k0 + i];
+  }
+  if (tid == 0) {
+    int n = 0;
+    for (int j = 0; j < kTcComps; j++)
+      if (a.sharp[k0 + j]) shl[1 + n++] = j;
+    shl[0] = n;
+  }
+  for (int i = tid; i < 2048; i += kTcThreads)
+    reinterpret_cast<__half*>(sOnes)[i] = __float2half_rn(1.0f);
+  // padding features of F must read as zero in every MMA
+  for (uint32_t i = tid; i < 2u * nch * kTcChunkBytes / 16; i += kTcThreads)
+    reinterpret_cast<uint4*>(sF)[i] = make_uint4(0, 0, 0, 0);
+  if (MODE == kTcStats) {
+    for (int f = 0; f <= 2 * D; f++)
+      for (int kk = tid; kk < kTcComps; kk += kTcThreads)
+        if (k0 + kk < K) slot[(size_t)f * K + k0 + kk] = 0.0;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before_sync();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tslot;
+  const uint32_t tL = tmem;
+  const uint32_t tS = tmem + 128;
+  const uint32_t tNK = tmem + 128 + 64 * (uint32_t)nch;
+
+  if (warp == 5) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_whi);
+      tma_prefetch_desc(&tm_wlo);
+      uint32_t stage = 0, phase = 0;
+      int64_t issued = 0;
+      for (int64_t li = 0; li < my_tiles; li++) {
+        bool ok = true;
+        for (int c = 0; c < nch && ok; c++)
+          for (int part = 0; part < 2 && ok; part++) {
+            ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, status, kAbort, a.wait_ns);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&full[stage], kTcChunkBytes);
+            tma_load_2d(sW + stage * kTcChunkBytes, part ? &tm_wlo : &tm_whi, c * kTcChunk, k0,
+                        &full[stage]);
+            issued++;
+            if (++stage == kTcStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        if (!ok) break;
+      }
+      // every load issued must have landed before the CTA may exit
+      for (int s = 0; s < kTcStages && s < issued; s++) {
+        const int64_t uses = (issued - s + kTcStages - 1) / kTcStages;  // loads into stage s
+        mbar_wait_bounded(&full[s], (uint32_t)((uses - 1) & 1), status, 0u, a.wait_ns);
+      }
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idE = idesc_f16_f32(128, 128, false, false);
+      const uint32_t idS = idesc_f16_f32(128, 64, true, true);
+      const uint32_t idN = idesc_f16_f32(128, 16, true, false);
+      const uint32_t fb = smem_u32(sF), wb = smem_u32(sW), rb = smem_u32(sR);
+      const uint32_t ob = smem_u32(sOnes);
+      uint32_t stage = 0, phase = 0, ndrain = 0;
+      for (int64_t li = 0; li < my_tiles; li++) {
+        if (!mbar_wait_bounded(f_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) break;
+        tc_fence_after_sync();
+        bool ok = true;
+        for (int c = 0; c < nch && ok; c++) {
+          const uint32_t fhi = fb + (uint32_t)c * kTcChunkBytes;
+          const uint32_t flo = fb + (uint32_t)(nch + c) * kTcChunkBytes;
+          for (int part = 0; part < 2; part++) {
+            ok = mbar_wait_bounded(&full[stage], phase, status, kAbort, a.wait_ns);
+            if (!ok) break;
+            tc_fence_after_sync();
+            const uint32_t w = wb + stage * kTcChunkBytes;
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++) {
+              const uint64_t bd = sw128_desc(w + 32u * ks, 16, 1024);
+              mma_bf16(tL, sw128_desc(fhi + 32u * ks, 16, 1024), bd, idE,
+                       !(part == 0 && c == 0 && ks == 0));
+              if (part == 0) mma_bf16(tL, sw128_desc(flo + 32u * ks, 16, 1024), bd, idE, true);
+            }
+            mma_commit(&empty[stage]);
+            if (++stage == kTcStages) {
+              stage = 0;
+              phase ^= 1u;
+            }
+          }
+        }
+        if (!ok) break;
+        mma_commit(l_full);
+        if (!mbar_wait_bounded(r_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) break;
+        tc_fence_after_sync();
+        bool ok2 = true;
+        if (MODE == kTcStats) {
+          const bool first = (li % a.drain_tiles) == 0;
+          if (first && li > 0) {
+            if (!mbar_wait_bounded(drained, ndrain & 1u, status, kAbort, a.wait_ns)) break;
+            ndrain++;
+            tc_fence_after_sync();
+          }
+          for (int half = 0; half < 2 && ok2; half++) {
+            if (half == 1) {
+              mma_commit(r_free);
+              ok2 = mbar_wait_bounded(r_full1, (uint32_t)(li & 1), status, kAbort, a.wait_ns);
+              if (!ok2) break;
+              tc_fence_after_sync();
+            }
+#pragma unroll 1
+            for (int ks = 0; ks < 4; ks++) {
+              const uint64_t ahi = sw128_desc(rb + 2048u * ks, 8192, 1024);
+              const uint64_t alo = sw128_desc(rb + 16384u + 2048u * ks, 8192, 1024);
+              const bool acc = !(first && half == 0 && ks == 0);
+              const uint32_t kr = 2048u * (uint32_t)(4 * half + ks);  // F rows of this K-step
+              for (int c = 0; c < nch; c++) {
+                const uint64_t fhi = sw128_desc(fb + (uint32_t)c * kTcChunkBytes + kr, 16384, 1024);
+                const uint64_t flo =
+                    sw128_desc(fb + (uint32_t)(nch + c) * kTcChunkBytes + kr, 16384, 1024);
+                mma_bf16(tS + 64u * c, ahi, fhi, idS, acc);
+                mma_bf16(tS + 64u * c, ahi, flo, idS, true);
+                mma_bf16(tS + 64u * c, alo, fhi, idS, true);
+              }
+              const uint64_t od = sw128_desc(ob, 16, 1024);
+              mma_bf16(tNK, ahi, od, idN, acc);
+              mma_bf16(tNK, alo, od, idN, true);
+            }
+          }
+        } else {
+          mma_commit(r_free);
+          ok2 = mbar_wait_bounded(r_full1, (uint32_t)(li & 1), status, kAbort, a.wait_ns);
+        }
+        if (!ok2) break;
+        mma_commit(s_done);
+      }
+      // every MMA issued must be complete before tensor memory is released
+      mma_commit(final_bar);
+      mbar_wait_bounded(final_bar, 0, status, 0u, a.wait_ns);
+    }
+  } else {
+    // ------------------------------------------------------------ compute warps
+    const int t = tid;  // row of the tile in the epilogue, component lane in drains
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    double ll = 0.0;
+    bool ok = true;
+    const int G = D / 4;
+
+    auto drain = [&]() {
+      const int k = k0 + t;
+      for (int c = 0; c < nch; c++) {
+        float v0[32], v1[32];
+        tmem_ld32(tS + lane_base + 64u * c, v0);
+        tmem_ld32(tS + lane_base + 64u * c + 32u, v1);
+        if (k < K) {
+#pragma unroll
+          for (int j = 0; j < 32; j++) {
+            const int f0 = 64 * c + j, f1 = 64 * c + 32 + j;
+            if (f0 < 2 * D) slot[(size_t)f0 * K + k] += (double)v0[j];
+            if (f1 < 2 * D) slot[(size_t)f1 * K + k] += (double)v1[j];
+          }
+        }
+      }
+      float vn[32];
+      tmem_ld32(tNK + lane_base, vn);
+      if (k < K) slot[(size_t)(2 * D) * K + k] += (double)vn[0];
+    };
+
+    for (int64_t li = 0; li < my_tiles && ok; li++) {
+      const int64_t row0 = ((int64_t)cid + li * ncl) * kTcRows;
+      if (li > 0) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait_bounded(s_done, (uint32_t)((li - 1) & 1), status, kAbort,
+                                          a.wait_ns));
+        if (!ok) break;
+        tc_fence_after_sync();
+        if (MODE == kTcStats && (li % a.drain_tiles) == 0) {
+          drain();
+          tc_fence_before_sync();
+          mbar_arrive(drained);
+        }
+      }
+      // ---- X tile -> F = [x^, x^^2] as fp16 hi/lo in the swizzled layout
+      bool bad = false, wide = false;
+      for (int u = t; u < kTcRows * G; u += 128) {
+        const int n = u / G, g = u - n * G;
+        const int64_t row = row0 + n;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (row < a.N) {
+          load4<XT>(reinterpret_cast<const XT*>(a.X), (size_t)row * D + 4 * g, x);
+#pragma unroll
+          for (int j = 0; j < 4; j++) {
+            if (!isfinite(x[j])) bad = true;
+            x[j] = (x[j] - msm[4 * g + j]) * iscs[4 * g + j];
+            if (fabsf(x[j]) > kTcXMax) {
+              wide = true;
+              x[j] = copysignf(kTcXMax, x[j]);
+            }
+          }
+        }
+        float sq[4];
+        uint32_t hx[2], lx[2], hs[2], ls[2];
+#pragma unroll
+        for (int j = 0; j < 4; j++) sq[j] = x[j] * x[j];
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+          const float x0 = x[2 * h], x1 = x[2 * h + 1], s0 = sq[2 * h], s1 = sq[2 * h + 1];
+          const float x0h = round_half(x0), x1h = round_half(x1);
+          const float s0h = round_half(s0), s1h = round_half(s1);
+          hx[h] = pack_half2(x0h, x1h);
+          lx[h] = pack_half2(x0 - x0h, x1 - x1h);
+          hs[h] = pack_half2(s0h, s1h);
+          ls[h] = pack_half2(s0 - s0h, s1 - s1h);
+        }
+        const int f1 = 4 * g, f2 = D + 4 * g;
+        const uint32_t o1 = (uint32_t)(f1 >> 6) * kTcChunkBytes + sw128_offset(n, f1 & 63);
+        const uint32_t o2 = (uint32_t)(f2 >> 6) * kTcChunkBytes + sw128_offset(n, f2 & 63);
+        const uint32_t lo_off = (uint32_t)nch * kTcChunkBytes;
+        *reinterpret_cast<uint2*>(sF + o1) = make_uint2(hx[0], hx[1]);
+        *reinterpret_cast<uint2*>(sF + lo_off + o1) = make_uint2(lx[0], lx[1]);
+        *reinterpret_cast<uint2*>(sF + o2) = make_uint2(hs[0], hs[1]);
+        *reinterpret_cast<uint2*>(sF + lo_off + o2) = make_uint2(ls[0], ls[1]);
+      }
+      if (bad) atomicOr(a.status, GMM_DEVFLAG_NONFINITE_X);
+      if (wide) atomicOr(a.status, GMM_DEVFLAG_X_RANGE);
+      fence_proxy_async_smem();
+      mbar_arrive(f_full);
+
+      // ---- epilogue: logits -> row max / sum-exp -> cluster exchange -> r^
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait_bounded(l_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns));
+      if (!ok) break;
+      tc_fence_after_sync();
+      // sharp components: direct-form log-joints of this row, written over the
+      // tensor-core values (their expanded-form constant is 0 and scale 1)
+      const int nsh = shl[0];
+      for (int si = 0; si < nsh; si++) {
+        const int j = shl[1 + si];
+        const float* mk = a.muh + (size_t)(k0 + j) * D;
+        const float* pk = a.ph + (size_t)(k0 + j) * D;
+        float q = 0.f;
+        for (int d = 0; d < D; d += 4) {
+          const uint32_t off = (uint32_t)(d >> 6) * kTcChunkBytes + sw128_offset(t, d & 63);
+          const uint2 hv = *reinterpret_cast<const uint2*>(sF + off);
+          const uint2 lv = *reinterpret_cast<const uint2*>(sF + (uint32_t)nch * kTcChunkBytes + off);
+          const float4 m4 = __ldg(reinterpret_cast<const float4*>(mk + d));
+          const float4 p4 = __ldg(reinterpret_cast<const float4*>(pk + d));
+          const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
+          const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
+          const float2 l0 = __half22float2(*reinterpret_cast<const __half2*>(&lv.x));
+          const float2 l1 = __half22float2(*reinterpret_cast<const __half2*>(&lv.y));
+          float e0 = (h0.x + l0.x) - m4.x, e1 = (h0.y + l0.y) - m4.y;
+          float e2 = (h1.x + l1.x) - m4.z, e3 = (h1.y + l1.y) - m4.w;
+          q = fmaf(e0 * e0, p4.x, q);
+          q = fmaf(e1 * e1, p4.y, q);
+          q = fmaf(e2 * e2, p4.z, q);
+          q = fmaf(e3 * e3, p4.w, q);
+        }
+        tmem_st1(tL + lane_base + (uint32_t)j, cds[j] - 0.5f * q);
+      }
+      float e[128];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 4; q++) {
+        float v[32];
+        tmem_ld32(tL + lane_base + 32u * q, v);
+#pragma unroll
+        for (int j = 0; j < 32; j++) {
+          e[32 * q + j] = fmaf(v[j], wscs[32 * q + j], csm[32 * q + j]);
+          mx = fmaxf(mx, e[32 * q + j]);
+        }
+      }
+      float se = 0.f;
+      if (mx > -INFINITY) {
+#pragma unroll
+        for (int j = 0; j < 128; j++) {
+          e[j] = __expf(e[j] - mx);
+          se += e[j];
+        }
+      }
+      const uint32_t par = (uint32_t)(li & 1);
+      const uint32_t my_x = smem_u32(&xchg[(par * C + rank) * kTcRows + t]);
+      for (int r2 = 0; r2 < C; r2++) st_cluster_f32x2(map_to_rank(my_x, r2), mx, se);
+      const uint32_t xb = smem_u32(&xbar[par]);
+      for (int r2 = 0; r2 < C; r2++) mbar_arrive_cluster(map_to_rank(xb, r2));
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&xbar[par], (uint32_t)((li >> 1) & 1),
+                                                     status, kAbort, a.wait_ns, true));
+      if (!ok) break;
+      float M = -INFINITY;
+      for (int j = 0; j < C; j++) M = fmaxf(M, xchg[(par * C + j) * kTcRows + t].x);
+      float S = 0.f;
+      for (int j = 0; j < C; j++) {
+        const float2 p = xchg[(par * C + j) * kTcRows + t];
+        if (p.x > -INFINITY) S += p.y * __expf(p.x - M);
+      }
+      const float lse = M + __logf(S);
+      const bool valid = row0 + t < a.N;
+      if (valid && rank == 0) ll += (double)lse;
+      const float scale = (valid && mx > -INFINITY) ? __expf(mx - lse) * kTcRScale : 0.f;
+      const int half = t >> 6, rr = t & 63;
+      if (MODE == kTcStats) {
+        if (half == 1) {
+          // the first half's MMAs must be done with the buffer
+          ok = __all_sync(0xffffffffu, mbar_wait_bounded(r_free, (uint32_t)(li & 1), status,
+                                                         kAbort, a.wait_ns));
+          if (!ok) break;
+        }
+#pragma unroll
+        for (int q8 = 0; q8 < 16; q8++) {
+          float v[8], h[8];
+#pragma unroll
+          for (int i = 0; i < 8; i++) {
+            v[i] = e[8 * q8 + i] * scale;
+            h[i] = round_half(v[i]);
+          }
+          const uint4 ph4 = make_uint4(pack_half2(h[0], h[1]), pack_half2(h[2], h[3]),
+                                       pack_half2(h[4], h[5]), pack_half2(h[6], h[7]));
+          const uint4 pl4 = make_uint4(pack_half2(v[0] - h[0], v[1] - h[1]),
+                                       pack_half2(v[2] - h[2], v[3] - h[3]),
+                                       pack_half2(v[4] - h[4], v[5] - h[5]),
+                                       pack_half2(v[6] - h[6], v[7] - h[7]));
+          const uint32_t off = (uint32_t)(q8 >> 3) * 8192u + (uint32_t)rr * 128u +
+                               ((((uint32_t)(q8 & 7)) ^ ((uint32_t)rr & 7u)) << 4);
+          *reinterpret_cast<uint4*>(sR + off) = ph4;
+          *reinterpret_cast<uint4*>(sR + 16384u + off) = pl4;
+        }
+        fence_proxy_async_smem();
+      }
+      tc_fence_before_sync();
+      mbar_arrive(half == 0 ? r_full : r_full1);
+    }
+    if (ok && my_tiles > 0) {
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(s_done, (uint32_t)((my_tiles - 1) & 1),
+                                                     status, kAbort, a.wait_ns));
+      tc_fence_after_sync();
+      if (ok && MODE == kTcStats) drain();
+    }
+    // LL of this CTA's rows (rank 0 of each cluster only): fixed-order block sum
+    ll = warp_sum(ll);
+    double* red = reinterpret_cast<double*>(sR);  // r^ is no longer read by any MMA
+    __syncwarp();
+    if (lane == 0) red[warp] = ok ? ll : 0.0;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (t == 0 && rank == 0) slot[ll_index] = ok ? red[0] + red[1] + red[2] + red[3] : 0.0;
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, 512);
+  }
+  cluster_sync();
+}
+
+// ---------------------------------------------------------------------------
+// Prep for the tensor-core pass, one thread per dimension:
+//   m_d = sum_k pi_k mu_kd / sum_k pi_k                  (centring, fp64)
+//   v_d = sum_k pi_k (var_kd + mu_kd^2) / sum_k pi_k - m_d^2   (mixture variance)
+//   s_d = 2^(round(log2 sqrt(v_d)) + 1)                  (exact power-of-two scale)
+// ---------------------------------------------------------------------------
+__global__ void tc_center_kernel(int D, int K, const float* __restrict__ w,
+                                 const float* __restrict__ mu, const float* __restrict__ var,
+                                 float* __restrict__ m_out, float* __restrict__ isc_out,
+                                 float* __restrict__ sc_out) {
+  const int d = blockIdx.x * blockDim.x + threadIdx.x;
+  if (d >= D) return;
+  double s = 0.0, s2 = 0.0, sw = 0.0;
+  for (int k = 0; k < K; k++) {
+    const double wk = (double)w[k];
+    if (wk > 0.0) {
+      const double mk = (double)mu[(size_t)k * D + d];
+      s += wk * mk;
+      s2 += wk * ((double)var[(size_t)k * D + d] + mk * mk);
+      sw += wk;
+    }
+  }
+  const double m = sw > 0.0 ? s / sw : 0.0;
+  const double v = sw > 0.0 ? s2 / sw - m * m : 0.0;
+  int e = 0;
+  if (v > 0.0 && isfinite(v)) {
+    e = (int)lrint(0.5 * log2(v)) + 1;
+    e = max(-60, min(60, e));
+  }
+  m_out[d] = (float)m;
+  isc_out[d] = ldexpf(1.0f, -e);
+  sc_out[d] = ldexpf(1.0f, e);
+}
+
+// One block per (padded) component.  W = [mu^/var^, -1/(2 var^)] scaled by a
+// power of two 2^-g_k so its largest entry lies in [2^13, 2^14), split into
+// fp16 hi/lo rows of Fpad features (padding rows and features zero); the
+// constants of both forms; kappa_k and the direct-form tables mu^, 1/var^.
+__global__ void __launch_bounds__(128) tc_prep_w_kernel(
+    int64_t N, int D, int K, int Fpad, const float* __restrict__ w, const float* __restrict__ mu,
+    const float* __restrict__ var, const float* __restrict__ m, const float* __restrict__ sc,
+    __half* __restrict__ whi, __half* __restrict__ wlo, float* __restrict__ c_out,
+    float* __restrict__ cd_out, float* __restrict__ wsc_out, int* __restrict__ sharp_out,
+    float* __restrict__ muh, float* __restrict__ ph, unsigned int* status) {
+  __shared__ double wv[kTcChunk * kTcMaxChunks];  // Fpad <= 256
+  __shared__ double red[4][4];
+  const int k = blockIdx.x;
+  double s_log = 0.0, s_q = 0.0, kap = 0.0, amax = 0.0;
+  bool bad = false;
+  for (int f = threadIdx.x; f < Fpad; f += blockDim.x) {
+    double v = 0.0;
+    if (k < K && f < 2 * D) {
+      const int d = f < D ? f : f - D;
+      const double sd = (double)sc[d];
+      const double vr = (double)var[(size_t)k * D + d];
+      const double vh = vr / (sd * sd);
+      const double mh = ((double)mu[(size_t)k * D + d] - (double)m[d]) / sd;
+      if (f < D) {
+        v = mh / vh;
+        s_log += log(2.0 * M_PI * vr);
+        s_q += mh * mh / vh;
+        kap += (mh * mh + 1.0) / vh;
+        muh[(size_t)k * D + d] = (float)mh;
+        ph[(size_t)k * D + d] = (float)(1.0 / vh);
+        if (!isfinite(mu[(size_t)k * D + d]) || !(vr > 0.0) || !isfinite(vr)) bad = true;
+      } else {
+        v = -0.5 / vh;
+      }
+    }
+    wv[f] = v;
+    amax = fmax(amax, fabs(v));
+  }
+  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+  double t0 = warp_sum(s_log), t1 = warp_sum(s_q), t2 = warp_sum(kap);
+  double t3 = amax;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t3 = fmax(t3, __shfl_xor_sync(0xffffffffu, t3, o));
+  if (lane == 0) {
+    red[0][wp] = t0;
+    red[1][wp] = t1;
+    red[2][wp] = t2;
+    red[3][wp] = t3;
+  }
+  __syncthreads();
+  const double S_log = red[0][0] + red[0][1] + red[0][2] + red[0][3];
+  const double S_q = red[1][0] + red[1][1] + red[1][2] + red[1][3];
+  const double Kap = red[2][0] + red[2][1] + red[2][2] + red[2][3];
+  const double Amax = fmax(fmax(red[3][0], red[3][1]), fmax(red[3][2], red[3][3]));
+  int ex = 0;
+  if (Amax > 0.0 && isfinite(Amax)) frexp(Amax, &ex);
+  const int g = Amax > 0.0 ? ex - 14 : 0;
+  for (int f = threadIdx.x; f < Fpad; f += blockDim.x) {
+    const float sv = (float)ldexp(wv[f], -g);
+    const __half h = __float2half_rn(sv);
+    whi[(size_t)k * Fpad + f] = h;
+    wlo[(size_t)k * Fpad + f] = __float2half_rn(sv - __half2float(h));
+  }
+  if (threadIdx.x == 0) {
+    const float wk = k < K ? w[k] : 0.f;
+    if (k < K && (!isfinite(wk) || !(wk >= 0.f))) bad = true;
+    const bool live = k < K && wk > 0.f;
+    const bool small = (double)wk * (double)N < kTcSmallPoints;
+    const bool sharp = live && (Kap > kTcSharpKappa || (small && Kap > kTcSmallKappa));
+    const double lw = live ? log((double)wk) : 0.0;
+    cd_out[k] = live ? (float)(lw - 0.5 * S_log) : -INFINITY;
+    c_out[k] = !live ? -INFINITY : (sharp ? 0.f : (float)(lw - 0.5 * (S_log + S_q)));
+    wsc_out[k] = sharp ? 1.f : ldexpf(1.0f, g);
+    sharp_out[k] = sharp ? 1 : 0;
+  }
+  if (bad) atomicOr(status, GMM_DEVFLAG_BAD_PARAMS);
+}
+
+// Fixed-order fp64 sum of the per-cluster slots and the M-step (statistics
+// are in scaled units: r * 2^15 and x^ = (x - m)/s):
+//   pi = N_k/N; if N_k > 1e-12 N: mu = m + s S1/N_k', var = max(s^2 (S2/N_k' - (S1/N_k')^2), floor)
+// with N_k' the scaled count.
+__global__ void __launch_bounds__(256) tc_reduce_mstep_kernel(
+    int64_t N, int D, int K, float var_floor, const float* __restrict__ m,
+    const float* __restrict__ sc, const double* __restrict__ slots, size_t slot_stride,
+    int nslots, float* __restrict__ w, float* __restrict__ mu, float* __restrict__ var,
+    double* __restrict__ loglik) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t ll_index = (size_t)(2 * D + 1) * K;
+  if (i == 0 && loglik) {
+    double ll = 0.0;
+    for (int p = 0; p < nslots; p++) ll += slots[(size_t)p * slot_stride + ll_index];
+    *loglik = ll;
+  }
+  if (i >= (size_t)K * D) return;
+  const int d = (int)(i / K), k = (int)(i - (size_t)d * K);
+  double nks = 0.0, s1 = 0.0, s2 = 0.0;
+  for (int p = 0; p < nslots; p++) {
+    const double* s = slots + (size_t)p * slot_stride;
+    nks += s[(size_t)(2 * D) * K + k];
+    s1 += s[(size_t)d * K + k];
+    s2 += s[(size_t)(D + d) * K + k];
+  }
+  const double nk = nks / (double)kTcRScale;
+  if (d == 0) w[k] = (float)(nk / (double)N);
+  if (nk > 1e-12 * (double)N) {
+    const double sd = (double)sc[d];
+    const double mt = s1 / nks;
+    double v = (s2 / nks - mt * mt) * sd * sd;
+    if (!(v > (double)var_floor)) v = (double)var_floor;
+    mu[(size_t)k * D + d] = (float)((double)m[d] + sd * mt);
+    var[(size_t)k * D + d] = (float)v;
+  }
+}
+
+__global__ void tc_reduce_loglik_kernel(int D, int K, const double* __restrict__ slots,
+                                        size_t slot_stride, int nslots,
+                                        double* __restrict__ loglik) {
+  const size_t ll_index = (size_t)(2 * D + 1) * K;
+  double ll = 0.0;
+  for (int p = 0; p < nslots; p++) ll += slots[(size_t)p * slot_stride + ll_index];
+  *loglik = ll;
+}
+
+}  // namespace scem

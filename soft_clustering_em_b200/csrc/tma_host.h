@@ -30,11 +30,13 @@ inline EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-// Tensor map of a row-major bf16 matrix [rows x cols] (row pitch in bytes, a
-// multiple of 16) read in boxes of [box_rows x 64] columns into the
-// 128-byte-swizzled shared-memory layout.  Returns false on failure.
-inline bool make_tmap_bf16_sw128(CUtensorMap* map, const void* base, uint64_t cols,
-                                 uint64_t rows, uint64_t pitch_bytes, uint32_t box_rows) {
+// Tensor map of a row-major matrix of 16-bit elements [rows x cols] (row
+// pitch in bytes, a multiple of 16) read in boxes of [box_rows x 64] columns
+// into the 128-byte-swizzled shared-memory layout.  The element type only
+// fixes the size (2 bytes), so one map serves fp16 and bf16 data alike.
+// Returns false on failure.
+inline bool make_tmap_16b_sw128(CUtensorMap* map, const void* base, uint64_t cols,
+                                uint64_t rows, uint64_t pitch_bytes, uint32_t box_rows) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   if (((uintptr_t)base) % 16 != 0 || pitch_bytes % 16 != 0) return false;

@@ -18,7 +18,7 @@ using namespace scem::sm100;
 
 namespace {
 
-constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint64_t kWaitLimit = 1000000000ull;  // 1 s
 
 struct ProbeArgs {
   int mode, N;
@@ -136,7 +136,7 @@ extern "C" int tc_probe_run(int mode, int N, const void* A, const void* B, float
   if (mode == 0 && !(N == 16 || N == 64 || N == 128 || N == 256)) return 1;
   CUtensorMap tm;
   memset(&tm, 0, sizeof(tm));
-  if (mode == 0 && !scem::make_tmap_bf16_sw128(&tm, B, 64, (uint64_t)N, 128, (uint32_t)N))
+  if (mode == 0 && !scem::make_tmap_16b_sw128(&tm, B, 64, (uint64_t)N, 128, (uint32_t)N))
     return 2;
   const size_t smem = 69632 + 128 + 1024;
   if (cudaFuncSetAttribute(tc_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -241,3 +241,66 @@ def test_fit_matches_repeated_steps(G):
     # LL of the GPU trajectory is monotone up to fp32 rounding
     h = hist.cpu().numpy()
     assert np.all(np.diff(h) >= -1e-6 * np.abs(h[1:]))
+
+
+@pytest.mark.parametrize("name,N,K,fit_iters", [("uint8img", 20_011, 256, 8),
+                                                 ("bf16stream", 60_001, 1024, 6),
+                                                 ("gauss8", 10_000, 8, 6)])
+def test_late_iteration_step_matches_oracle(G, name, N, K, fit_iters):
+    """Teacher-forced step from parameters the oracle has already fitted for a
+    few iterations: the variances have shrunk, so the expanded form's
+    cancellation (mu~^2 / var up to ~650 on uint8img) is at its worst here."""
+    import torch
+
+    wl = synth.WORKLOADS[name]
+    X, _ = synth.make_data(wl, N)
+    X64 = synth.x_as_f64(wl, X)
+    Xd = to_device(wl, X)
+    rows = synth.init_rows(N, K, wl.init_seed)
+    mode = 0 if wl.var_init == "one" else 1
+    th = oracle.init(X64, rows, K, mode, wl.var_floor)
+    th = oracle.fit(X64, *th, fit_iters, wl.var_floor)[:3]
+    w = torch.tensor(th[0], dtype=torch.float32, device="cuda")
+    mu = torch.tensor(th[1], dtype=torch.float32, device="cuda")
+    var = torch.tensor(th[2], dtype=torch.float32, device="cuda")
+    th32 = params_np(w, mu, var)
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    ws = G.workspace(G.problem_for(Xd, K, wl.var_floor))
+    G.gmm_em_step(Xd, w, mu, var, ll, wl.var_floor, ws=ws)
+    rc, flags = G.gmm_device_status(ws)
+    assert rc == 0, flags
+    w2, mu2, var2, ll_ref, Nk = oracle.em_step(X64, *th32, var_floor=wl.var_floor)
+    rep = compare.compare_step((w2, mu2, var2, ll_ref), (*params_np(w, mu, var), ll.item()), Nk)
+    assert rep["ok"], rep
+
+
+@pytest.mark.parametrize("name,N,K", [("uint8img", 50_000, 256), ("bf16stream", 100_000, 1024),
+                                      ("gauss8", 10_000, 8)])
+def test_tensor_core_and_cuda_core_paths_agree(G, name, N, K, monkeypatch):
+    """The same step through the tensor-core kernel and through the CUDA-core
+    kernel (direct form) from identical parameters, at a size the oracle is
+    not needed for; both must agree within the parity tolerances."""
+    import torch
+
+    wl = synth.WORKLOADS[name]
+    X, _ = synth.make_data(wl, N)
+    Xd = to_device(wl, X)
+    ws = G.workspace(G.problem_for(Xd, K, wl.var_floor))
+    mode = G.GMM_INIT_VAR_ONE if wl.var_init == "one" else G.GMM_INIT_VAR_DATA
+    w, mu, var = G.gmm_init(Xd, synth.init_rows(N, K, wl.init_seed), K, mode, wl.var_floor, ws=ws)
+    for _ in range(3):
+        G.gmm_em_step(Xd, w, mu, var, None, wl.var_floor, ws=ws)
+    outs = []
+    for path in ("tc", "simt"):
+        if path == "simt":
+            monkeypatch.setenv("SCEM_GMM_PATH", "simt")
+        t = [w.clone(), mu.clone(), var.clone()]
+        ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+        G.gmm_em_step(Xd, *t, ll, wl.var_floor, ws=ws)
+        rc, flags = G.gmm_device_status(ws)
+        assert rc == 0, flags
+        outs.append((*params_np(*t), ll.item()))
+    monkeypatch.delenv("SCEM_GMM_PATH")
+    nk = outs[1][0] * N
+    rep = compare.compare_step(outs[1], outs[0], nk)
+    assert rep["ok"], rep
