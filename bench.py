@@ -14,6 +14,11 @@ L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+With N > 1 (one process per GPU under torchrun) the run is row-sharded weak
+scaling: every rank holds its own block of N rows of the same data stream, and
+one step is gmm_estep_stats on each rank, an NCCL all-gather of the fp64
+statistics and gmm_mstep (which sums the shards in rank order) on every rank.
+
 --impl reference times the CPU oracle (plain fp64 EM) on the host cores, on a
 bounded row sample of the same workload per step, scaled to the same unit.
 """
@@ -36,7 +41,8 @@ from soft_clustering_em_b200 import synth  # noqa: E402
 METRIC = "EM iterations/s and fused E+M N·K·D/s on 1 B200, % of roofline"
 UNIT = "EM iterations/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-FUSED_SOURCES = ["soft_clustering_em_b200/csrc/simt_em.cuh",
+FUSED_SOURCES = ["soft_clustering_em_b200/csrc/tc_em.cuh",
+                 "soft_clustering_em_b200/csrc/sm100_prims.cuh",
                  "soft_clustering_em_b200/csrc/common.cuh"]
 
 
@@ -212,16 +218,17 @@ def workload_config(wl, N):
 
 def ours(args):
     import torch
+    import torch.distributed as dist
 
     from soft_clustering_em_b200 import gmm as G
+    from soft_clustering_em_b200 import sharded
 
     world, rank, local = dist_setup(args)
-    if world > 1:
-        raise SystemExit("multi-GPU row-sharded EM is not built yet")
     dev = torch.device("cuda", local)
     wl = synth.WORKLOADS[args.workload]
-    N = args.rows or wl.N
-    X_np, _ = synth.make_data(wl, N)
+    N = args.rows or wl.N  # rows per rank
+    N_total = N * world
+    X_np, _ = synth.make_data(wl, N, start=rank * N)
     Xh = torch.from_numpy(X_np.view(np.int16) if wl.dtype == "bf16" else X_np)
     if wl.dtype == "bf16":
         Xh = Xh.view(torch.bfloat16)
@@ -232,20 +239,40 @@ def ours(args):
     rows = synth.init_rows(N, wl.K, wl.init_seed)
     mode = G.GMM_INIT_VAR_ONE if wl.var_init == "one" else G.GMM_INIT_VAR_DATA
     w, mu, var = G.gmm_init(Xd, rows, wl.K, mode, wl.var_floor, ws=ws)
+    if world > 1:
+        sharded.broadcast_params(w, mu, var)  # every rank starts from rank 0's parameters
     ll = torch.zeros(1, dtype=torch.float64, device=dev)
     stream = torch.cuda.current_stream(dev)
     theta0 = (w.clone(), mu.clone(), var.clone())
     flush = None if Xd.numel() * Xd.element_size() > 126e6 else torch.empty(
         256 << 20, dtype=torch.uint8, device=dev)
+    stats = torch.empty(G.stats_size(wl.K, wl.D), dtype=torch.float64, device=dev)
+    xdt = G.xdtype_of(Xd)
 
-    def step():
-        G.gmm_em_step(Xd, w, mu, var, ll, wl.var_floor, ws=ws)
+    def step(X):
+        if world == 1:
+            G.gmm_em_step(X, w, mu, var, ll, wl.var_floor, ws=ws)
+        else:
+            G.gmm_estep_stats(X, w, mu, var, stats, wl.var_floor, ws=ws)
+            gathered = sharded.gather_stats(stats)
+            G.gmm_mstep(gathered, N_total, w, mu, var, ll, wl.var_floor, xdt)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
 
     props = torch.cuda.get_device_properties(dev)
     sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else None)
     time.sleep(0.5)
     for _ in range(max(3, args.warmup)):
-        step()
+        step(Xd)
     torch.cuda.synchronize(dev)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -255,18 +282,21 @@ def ours(args):
     launches0 = G.gmm_launch_count()
     t_begin = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
     t_begin.record(stream)
     for i in range(args.steps):
         G.gmm_trace_fused(starts[i], stops[i])
-        step()
+        step(Xd)
         if flush is not None:
             flush.zero_()
     t_end.record(stream)
     torch.cuda.synchronize(dev)
+    barrier()
     launches = G.gmm_launch_count() - launches0
     G.gmm_trace_fused(None, None)
     clocks = sampler.stop()
-    total_ms = t_begin.elapsed_time(t_end)
+    total_ms = max_over_ranks(t_begin.elapsed_time(t_end))
     fused_ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
     rc, flags = G.gmm_device_status(ws)
     if rc != 0:
@@ -280,28 +310,30 @@ def ours(args):
     Xd2 = torch.empty_like(Xd)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e2e_steps = args.steps
+    barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
-    for _ in range(e2e_steps):
+    for _ in range(args.steps):
         Xd2.copy_(Xh, non_blocking=True)
         w.copy_(w_h, non_blocking=True)
         mu.copy_(mu_h, non_blocking=True)
         var.copy_(var_h, non_blocking=True)
-        G.gmm_em_step(Xd2, w, mu, var, ll, wl.var_floor, ws=ws)
+        step(Xd2)
         w_h.copy_(w, non_blocking=True)
         mu_h.copy_(mu, non_blocking=True)
         var_h.copy_(var, non_blocking=True)
         ll_h.copy_(ll, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
     pbytes = (w.numel() + mu.numel() + var.numel()) * 4
-    h2d = Xd.numel() * Xd.element_size() + pbytes
-    d2h = pbytes + 8
+    h2d = (Xd.numel() * Xd.element_size() + pbytes) * world
+    d2h = (pbytes + 8) * world
 
     ms = total_ms / args.steps
-    value = 1e3 / ms
+    # whole-job throughput in workload iterations: rows of all ranks per second / workload N
+    value = (N_total / wl.N) * 1e3 / ms
     nkd = float(N) * wl.K * wl.D
     pk, pk_kind = peaks()
     sustained = total_ms >= 1000.0
@@ -309,20 +341,27 @@ def ours(args):
     fused_avg = statistics.mean(fused_ms)
     achieved = 8.0 * nkd / (fused_avg * 1e-3) / 1e12
     traffic = ncu_traffic(wl.name)
+    cfg = workload_config(wl, N)
+    if world > 1:
+        cfg.update({"ranks": world, "rows_per_rank": N, "exchange": "NCCL all-gather of fp64 "
+                    "statistics, M-step sums shards in rank order"})
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": workload_config(wl, N),
-        "nkd_per_s": nkd * value,
+        "vs_baseline": None, "dtype": "f16",
+        "precision": "fp16 hi/lo split operands on the tensor cores, fp32 accumulation, "
+                     "fp64 reductions and M-step",
+        "data": "synthetic", "config": cfg,
+        "nkd_per_s": nkd * world * 1e3 / ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "fused E-step + statistics pass",
+                     "kernel": "fused E-step + statistics pass (tc_fused_kernel)",
                      "algorithmic": "8*N*K*D flop per launch",
                      "fused_ms_per_launch": fused_avg,
                      "peak_source": f"{pk_kind} bf16 dense "
-                                    f"{'sustained' if sustained else 'burst'}"},
-        "e2e": {"value": 1e3 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                                    f"{'sustained' if sustained else 'burst'} "
+                                    "(fp16 runs at the bf16 rate)"},
+        "e2e": {"value": (N_total / wl.N) * 1e3 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
         "clocks": clocks,
@@ -351,6 +390,9 @@ def ours(args):
         line["parity"] = {"rows": n, **{k: rep[k] for k in ("ok", "w", "mu", "var", "ll")}}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
 
 
 def main():

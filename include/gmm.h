@@ -116,6 +116,31 @@ gmm_status gmm_em_step(const gmm_problem* p, const void* X, float* w, float* mu,
                        double* loglik, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The two halves of gmm_em_step, for row-sharded EM (each device holds a row
+ * shard of X; the statistics of all shards are summed between the halves).
+ *
+ * gmm_estep_stats: E-step over the rows of X and their sufficient statistics,
+ * reduced in a fixed order to fp64, into stats (device, K*(2D+1)+1 doubles):
+ *   stats = [ N_k (K) | A (K x D) | B (K x D) | LL ]
+ *   N_k = sum_n r_nk, A_kd = sum_n r_nk (x_nd - mu_kd), B_kd = sum_n r_nk (x_nd - mu_kd)^2
+ * (moments about the input means, data units), LL = sum_n log p(x_n).
+ * Statistics of disjoint row sets add elementwise.  Parameters unchanged.
+ *
+ * gmm_mstep: M-step, in place (see the model at the top), from the
+ * statistics of nshards >= 1 disjoint row shards holding p->N points in
+ * total, stored as nshards consecutive buffers (device, nshards x
+ * (K*(2D+1)+1) doubles, e.g. the output of an all-gather); they are summed in
+ * shard order, so the result does not depend on how the shards were
+ * computed.  loglik (device, may be NULL) receives the summed LL.  p->D, p->K
+ * and p->var_floor as for the shards; no X and no workspace are used.
+ */
+gmm_status gmm_estep_stats(const gmm_problem* p, const void* X, const float* w, const float* mu,
+                           const float* var, double* stats, void* ws, size_t ws_bytes,
+                           void* stream);
+gmm_status gmm_mstep(const gmm_problem* p, const double* stats, int32_t nshards, float* w,
+                     float* mu, float* var, double* loglik, void* stream);
+
+/*
  * gmm_em_step without a caller-provided workspace, for callers that are not
  * allowed to obtain device memory themselves: for example a plug-in running
  * inside a host application that owns the whole device-memory budget and

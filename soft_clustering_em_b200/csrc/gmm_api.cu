@@ -59,8 +59,11 @@ struct Plan {
   WsLayout simt;
   TcLayout tc;
   bool use_tc;
+  size_t stats;  // canonical statistics buffer: K(2D+1)+1 doubles
   size_t total;
 };
+
+size_t stats_doubles(const gmm_problem* p) { return (size_t)p->K * (2 * (size_t)p->D + 1) + 1; }
 
 bool force_cuda_core_path() {
   const char* e = getenv("SCEM_GMM_PATH");
@@ -69,14 +72,18 @@ bool force_cuda_core_path() {
 
 Plan make_plan(const gmm_problem* p, int sms, size_t cap) {
   Plan P;
-  P.simt = cap ? ws_layout_capped(p->D, p->K, sms, cap) : ws_layout(p->D, p->K, sms);
+  const size_t sbytes = align_up(stats_doubles(p) * 8, 256);
+  const size_t c = cap ? (cap > sbytes ? cap - sbytes : 1) : 0;
+  P.simt = c ? ws_layout_capped(p->D, p->K, sms, c) : ws_layout(p->D, p->K, sms);
   P.use_tc = tc_shape_ok(p->D, p->K) && !force_cuda_core_path();
   if (P.use_tc) {
-    P.tc = tc_layout(p->D, p->K, sms, cap);
+    P.tc = tc_layout(p->D, p->K, sms, c);
     if (P.tc.P < 1) P.use_tc = false;
   }
-  P.total = P.simt.P >= 1 ? P.simt.total : 0;
-  if (P.use_tc) P.total = std::max(P.total, P.tc.total);
+  size_t body = P.simt.P >= 1 ? P.simt.total : 0;
+  if (P.use_tc) body = std::max(body, P.tc.total);
+  P.stats = align_up(body, 256);
+  P.total = P.stats + sbytes;
   return P;
 }
 
@@ -167,7 +174,8 @@ gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const 
   tc_prep_w_kernel<<<T.Kpad, 128, 0, st>>>(
       p->N, p->D, p->K, T.Fpad, w, mu, var, m, (const float*)(ws + T.sc), (__half*)(ws + T.whi),
       (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.cd), (float*)(ws + T.wsc),
-      (int*)(ws + T.sharp), (float*)(ws + T.muh), (float*)(ws + T.ph), (unsigned int*)ws);
+      (int*)(ws + T.sharp), (float*)(ws + T.muh), (float*)(ws + T.ph),
+      (int*)(ws + T.precise), (unsigned int*)ws);
   return launched(2);
 }
 
@@ -236,6 +244,7 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, char* ws, const TcLayo
   args.slot_stride = T.slot_stride;
   args.status = (unsigned int*)ws;
   args.drain_tiles = tc_drain_tiles();
+  args.precise = (const int*)(ws + T.precise);
   args.wait_ns = kWaitBudgetNs;
   trace_begin(st);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args, mhi, mlo);
@@ -256,28 +265,46 @@ gmm_status tc_pass(const gmm_problem* p, const void* X, char* ws, const TcLayout
   return tc_launch<float, MODE>(p, X, ws, T, st, nslots);
 }
 
-gmm_status em_step_impl(const gmm_problem* p, const void* X, float* w, float* mu, float* var,
-                        double* loglik, void* ws_base, const Plan& P, cudaStream_t st) {
+// E-step and statistics of the rows of X into the canonical buffer `stats`.
+gmm_status estep_stats_impl(const gmm_problem* p, const void* X, const float* w,
+                            const float* mu, const float* var, double* stats, void* ws_base,
+                            const Plan& P, cudaStream_t st) {
   char* ws = (char*)ws_base;
   gmm_status s;
+  const size_t KD = (size_t)p->K * p->D;
+  const unsigned blocks = (unsigned)((KD + 255) / 256);
   if (P.use_tc) {
     const TcLayout& T = P.tc;
     if ((s = tc_prep(p, w, mu, var, ws, T, st)) != GMM_OK) return s;
     int nslots = 0;
     if ((s = tc_pass<kTcStats>(p, X, ws, T, st, &nslots)) != GMM_OK) return s;
-    const size_t KD = (size_t)p->K * p->D;
-    tc_reduce_mstep_kernel<<<(unsigned)((KD + 255) / 256), 256, 0, st>>>(
-        p->N, p->D, p->K, p->var_floor, (const float*)(ws + T.m), (const float*)(ws + T.sc),
-        (const double*)(ws + T.slots), T.slot_stride, nslots, w, mu, var, loglik);
+    tc_reduce_stats_kernel<<<blocks, 256, 0, st>>>(p->D, p->K, (const float*)(ws + T.m),
+                                                   (const float*)(ws + T.sc), mu,
+                                                   (const double*)(ws + T.slots), T.slot_stride,
+                                                   nslots, stats);
     return launched(1);
   }
   const WsPtrs wp = ws_ptrs(ws_base, P.simt);
   if ((s = prep(p, w, mu, var, wp, st)) != GMM_OK) return s;
   if ((s = fused_pass<kModeStats>(p, X, wp, 0, nullptr, nullptr, st)) != GMM_OK) return s;
-  const size_t KD = (size_t)p->K * p->D;
-  reduce_mstep_kernel<<<(unsigned)((KD + 255) / 256), 256, 0, st>>>(p->N, p->D, p->K, p->var_floor,
-                                                                    wp, w, mu, var, loglik);
+  simt_reduce_stats_kernel<<<blocks, 256, 0, st>>>(p->D, p->K, wp, stats);
   return launched(1);
+}
+
+gmm_status mstep_impl(const gmm_problem* p, const double* stats, int nshards, float* w,
+                      float* mu, float* var, double* loglik, cudaStream_t st) {
+  const size_t KD = (size_t)p->K * p->D;
+  mstep_kernel<<<(unsigned)((KD + 255) / 256), 256, 0, st>>>(p->N, p->D, p->K, p->var_floor,
+                                                             stats, nshards, w, mu, var, loglik);
+  return launched(1);
+}
+
+gmm_status em_step_impl(const gmm_problem* p, const void* X, float* w, float* mu, float* var,
+                        double* loglik, void* ws_base, const Plan& P, cudaStream_t st) {
+  double* stats = (double*)((char*)ws_base + P.stats);
+  gmm_status s = estep_stats_impl(p, X, w, mu, var, stats, ws_base, P, st);
+  if (s != GMM_OK) return s;
+  return mstep_impl(p, stats, 1, w, mu, var, loglik, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -397,6 +424,26 @@ gmm_status gmm_em_step(const gmm_problem* p, const void* X, float* w, float* mu,
   Plan P;
   if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
   return em_step_impl(p, X, w, mu, var, loglik, ws, P, (cudaStream_t)stream);
+}
+
+gmm_status gmm_estep_stats(const gmm_problem* p, const void* X, const float* w, const float* mu,
+                           const float* var, double* stats, void* ws, size_t ws_bytes,
+                           void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if ((s = check_x(p, X)) != GMM_OK) return s;
+  if (!w || !mu || !var || !stats) return GMM_ERR_INVALID_ARG;
+  Plan P;
+  if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  return estep_stats_impl(p, X, w, mu, var, stats, ws, P, (cudaStream_t)stream);
+}
+
+gmm_status gmm_mstep(const gmm_problem* p, const double* stats, int32_t nshards, float* w,
+                     float* mu, float* var, double* loglik, void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if (!stats || !w || !mu || !var || nshards < 1) return GMM_ERR_INVALID_ARG;
+  return mstep_impl(p, stats, nshards, w, mu, var, loglik, (cudaStream_t)stream);
 }
 
 gmm_status gmm_em_step_noalloc(const gmm_problem* p, const void* X, float* w, float* mu,

@@ -303,43 +303,65 @@ __global__ void __launch_bounds__(kSimtThreads) simt_fused_kernel(
   if (tid == 0 && MODE != kModeTopm) *sLL = ll;
 }
 
-// ---------------------------------------------------------------------------
-// Deterministic reduction of the P slots (fixed slot order, fp64) and M-step.
-// One thread per (d, k); thread 0 also writes LL.
-//   pi_k = N_k / N; if N_k > 1e-12 N: delta = A/N_k, mu += delta,
-//   var = max(B/N_k - delta^2, floor); else mu and var are kept.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) reduce_mstep_kernel(int64_t N, int D, int K,
-                                                           float var_floor, WsPtrs ws,
-                                                           float* __restrict__ w,
-                                                           float* __restrict__ mu,
-                                                           float* __restrict__ var,
-                                                           double* __restrict__ loglik) {
+// Fixed-order fp64 sum of the P slots into the canonical statistics buffer
+// (component-major, moments about the means the step started from):
+//   stats = [ N_k (K) | A (K x D) | B (K x D) | LL ].
+__global__ void __launch_bounds__(256) simt_reduce_stats_kernel(int D, int K, WsPtrs ws,
+                                                                double* __restrict__ stats) {
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i == 0 && loglik) {
+  const size_t KD = (size_t)K * D;
+  if (i == 0) {
     double ll = 0.0;
-    for (int p = 0; p < ws.P; p++)
-      ll += ws.slots[(size_t)p * ws.slot_stride + (size_t)K * (2 * (size_t)D + 1)];
-    *loglik = ll;
+    for (int p = 0; p < ws.P; p++) ll += ws.slots[(size_t)p * ws.slot_stride + K + 2 * KD];
+    stats[K + 2 * KD] = ll;
   }
-  if (i >= (size_t)K * D) return;
+  if (i >= KD) return;
   const int d = (int)(i / K), k = (int)(i - (size_t)d * K);
   double nk = 0.0, a = 0.0, b = 0.0;
   for (int p = 0; p < ws.P; p++) {
     const double* s = ws.slots + (size_t)p * ws.slot_stride;
     nk += s[k];
     a += s[K + i];
-    b += s[K + (size_t)K * D + i];
+    b += s[K + KD + i];
   }
-  if (d == 0) w[k] = (float)(nk / (double)N);
-  const size_t o = (size_t)k * D + d;
+  if (d == 0) stats[k] = nk;
+  stats[K + (size_t)k * D + d] = a;
+  stats[K + KD + (size_t)k * D + d] = b;
+}
+
+// M-step from canonical statistics of `nshards` disjoint row shards
+// (consecutive buffers of K(2D+1)+1 doubles, summed here in shard order) of N
+// points in total: pi_k = N_k / N; if N_k > 1e-12 N: delta = A/N_k,
+// mu += delta, var = max(B/N_k - delta^2, floor); else mu and var are kept.
+__global__ void __launch_bounds__(256) mstep_kernel(int64_t N, int D, int K, float var_floor,
+                                                    const double* __restrict__ stats, int nshards,
+                                                    float* __restrict__ w, float* __restrict__ mu,
+                                                    float* __restrict__ var,
+                                                    double* __restrict__ loglik) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t KD = (size_t)K * D;
+  const size_t S = (size_t)K + 2 * KD + 1;
+  if (i == 0 && loglik) {
+    double ll = 0.0;
+    for (int s = 0; s < nshards; s++) ll += stats[(size_t)s * S + K + 2 * KD];
+    *loglik = ll;
+  }
+  if (i >= KD) return;
+  const int k = (int)(i / D);
+  double nk = 0.0, a = 0.0, b = 0.0;
+  for (int s = 0; s < nshards; s++) {
+    const double* st = stats + (size_t)s * S;
+    nk += st[k];
+    a += st[K + i];
+    b += st[K + KD + i];
+  }
+  if (i - (size_t)k * D == 0) w[k] = (float)(nk / (double)N);
   if (nk > 1e-12 * (double)N) {
     const double delta = a / nk;
-    const double mu_old = (double)mu[o];
     double v = b / nk - delta * delta;
     if (!(v > (double)var_floor)) v = (double)var_floor;
-    mu[o] = (float)(mu_old + delta);
-    var[o] = (float)v;
+    mu[i] = (float)((double)mu[i] + delta);
+    var[i] = (float)v;
   }
 }
 

@@ -31,7 +31,14 @@
 //   N_k = sum_n r^_nk,  S1_kd = sum_n r^_nk x^_nd,  S2_kd = sum_n r^_nk x^_nd^2
 // as r_hi^T (F_hi + F_lo) + r_lo^T F_hi and r^T 1 on the tensor cores,
 // accumulated in fp32 in tensor memory over a few tiles and then added into
-// fp64 per-cluster slots.  The M-step undoes the scales exactly.  r^ passes
+// fp64 per-cluster slots.  The variance S2/N - (S1/N)^2 magnifies the
+// relative rounding error of those fp32 sums by rho_k = max_d mu^^2 / var^, and
+// a weight is sensitive to it when the component holds few points; so a
+// "precise" component (rho_k > 64, or pi_k N < 20) is drained after every
+// tile in which it has mass, every other component every kTcDrainTiles tiles.
+// Each compute thread drains its own component (tensor-memory lane) and
+// zeroes its accumulators in place with tcgen05.st.  The M-step undoes the
+// scales exactly.  r^ passes
 // through one 32 KB buffer in two 64-row halves: rows 0-63 first, then rows
 // 64-127 once the MMAs of the first half have released it.
 //
@@ -41,8 +48,9 @@
 // components (W streamed by TMA through a 3-stage ring), reduces each row's
 // max / sum-exp over its components, exchanges those with the other CTAs of
 // the cluster through distributed shared memory, forms r^ and runs the
-// statistics MMAs.  Warps 0-3: conversion, epilogue, drains (warp w owns
-// tensor-memory lanes 32w..32w+31); warp 4: MMA issue; warp 5: TMA issue.
+// statistics MMAs.  Warps 0-7: conversion, epilogue, drains (warp w reads
+// tensor-memory lanes 32(w%4)..32(w%4)+31 and component columns 64(w/4)..+63);
+// warp 8: MMA issue; warp 9: TMA issue.
 //
 // Tensor memory (512 columns): L logits [0,128); S statistics
 // [128, 128 + 64*nchunks); N_k [128 + 64*nchunks, +16).
@@ -61,8 +69,11 @@ constexpr int kTcChunk = 64;      // features per operand chunk (one swizzled 12
 constexpr int kTcStages = 3;      // depth of the W ring
 constexpr int kTcMaxChunks = 4;   // 2D <= 256
 constexpr int kTcMaxCluster = 16;
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 320;          // 8 compute warps + MMA warp + TMA warp
+constexpr int kTcComputeThreads = 256;
+constexpr int kTcMmaWarp = 8, kTcTmaWarp = 9;
 constexpr int kTcDrainTiles = 8;  // tiles accumulated in fp32 before an fp64 drain
+constexpr double kTcRhoPrecise = 64.0;  // rho_k above which a component drains every tile
 constexpr uint32_t kTcChunkBytes = 128u * 128u;  // one [128 x 64] 16-bit operand chunk
 constexpr float kTcRScale = 32768.0f;            // r is stored as fp16(r * 2^15)
 constexpr double kTcSharpKappa = 1e7;            // direct form above this kappa_k ...
@@ -77,7 +88,7 @@ inline int tc_cluster(int K) { return (K + kTcComps - 1) / kTcComps; }
 
 // Byte offsets of the kernel's shared-memory regions (from a 1024-aligned base).
 struct TcSmem {
-  uint32_t F, W, R, ONES, msm, iscs, csm, wscs, cds, shl, xchg, bars, tslot, total;
+  uint32_t F, W, R, ONES, msm, iscs, csm, wscs, cds, shl, precs, xchg, bars, tslot, total;
 };
 
 __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
@@ -103,10 +114,12 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
   off += kTcComps * 4;
   L.shl = off;
   off += (kTcComps + 4) * 4;
+  L.precs = off;
+  off += kTcComps * 4;
   L.xchg = off;
-  off += 2u * C * kTcRows * 8;
+  off += 2u * 2u * C * kTcRows * 8;  // [parity][rank][column half][row]
   L.bars = off;
-  off += 8 * (2 * kTcStages + 10);
+  off += 8 * (2 * kTcStages + 12);
   L.tslot = off;
   off += 16;
   L.total = off + 1024;  // slack for aligning the dynamic base to 1024
@@ -125,7 +138,7 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //          [(2D+1) x K] feature-major statistics (S1 rows 0..D-1, S2 rows
 //          D..2D-1, N_k row 2D) followed by the cluster's LL.
 struct TcLayout {
-  size_t m, isc, sc, c, cd, wsc, sharp, muh, ph, whi, wlo, slots, total, slot_stride;
+  size_t m, isc, sc, c, cd, wsc, sharp, precise, muh, ph, whi, wlo, slots, total, slot_stride;
   int C, nchunks, Kpad, Fpad, P;
 };
 
@@ -164,6 +177,8 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   off = align_up(off + (size_t)L.Kpad * L.Fpad * 2, 256);
   L.wlo = off;
   off = align_up(off + (size_t)L.Kpad * L.Fpad * 2, 256);
+  L.precise = off;
+  off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.slot_stride = align_up((size_t)(2 * D + 1) * K + 1, 32);
   L.slots = off;
   L.P = num_sms / L.C;
@@ -192,6 +207,7 @@ struct TcArgs {
   size_t slot_stride;   // doubles per slot: (2D+1)*K statistics + LL
   unsigned int* status;
   int drain_tiles;
+  const int* precise;   // 1: drain the component after every tile with mass, C*128
   uint64_t wait_ns;
 };
 
@@ -244,7 +260,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* wscs = reinterpret_cast<float*>(sm + L.wscs);
   float* cds = reinterpret_cast<float*>(sm + L.cds);
   int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = local indices
-  float2* xchg = reinterpret_cast<float2*>(sm + L.xchg);  // [2][C][128] (row max, row sum-exp)
+  int* precs = reinterpret_cast<int*>(sm + L.precs);
+  float2* xchg = reinterpret_cast<float2*>(sm + L.xchg);  // [2][C][2][128] (max, sum-exp)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* full = bars;
   uint64_t* empty = bars + kTcStages;
@@ -257,6 +274,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* final_bar = f_full + 7;
   uint64_t* r_full1 = f_full + 8;  // second 64-row half of r^ written
   uint64_t* r_free = f_full + 9;   // MMAs of the first half done with the r^ buffer
+  uint64_t* cbar = f_full + 10;    // rendezvous of the 256 compute threads
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tslot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -276,15 +294,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(f_full, 128);
+    mbar_init(f_full, kTcComputeThreads);
     mbar_init(l_full, 1);
-    mbar_init(r_full, 64);
-    mbar_init(r_full1, 64);
+    mbar_init(r_full, kTcComputeThreads / 2);
+    mbar_init(r_full1, kTcComputeThreads / 2);
     mbar_init(r_free, 1);
     mbar_init(s_done, 1);
-    mbar_init(drained, 128);
-    mbar_init(&xbar[0], (uint32_t)C * 128);
-    mbar_init(&xbar[1], (uint32_t)C * 128);
+    mbar_init(drained, kTcComputeThreads);
+    mbar_init(cbar, kTcComputeThreads);
+    mbar_init(&xbar[0], (uint32_t)C * kTcComputeThreads);
+    mbar_init(&xbar[1], (uint32_t)C * kTcComputeThreads);
     mbar_init(final_bar, 1);
     fence_mbar_init();
   }
@@ -300,6 +319,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     csm[i] = a.c[k0 + i];
     wscs[i] = a.wsc[k0 + i];
     cds[i] = a.cd[k0 + i];
+    precs[i] = a.precise[k0 + i];
   }
   if (tid == 0) {
     int n = 0;
@@ -327,7 +347,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tS = tmem + 128;
   const uint32_t tNK = tmem + 128 + 64 * (uint32_t)nch;
 
-  if (warp == 5) {
+  if (warp == kTcTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_whi);
@@ -357,7 +377,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_wait_bounded(&full[s], (uint32_t)((uses - 1) & 1), status, 0u, a.wait_ns);
       }
     }
-  } else if (warp == 4) {
+  } else if (warp == kTcMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idE = idesc_f16_f32(128, 128, false, false);
@@ -398,8 +418,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after_sync();
         bool ok2 = true;
         if (MODE == kTcStats) {
-          const bool first = (li % a.drain_tiles) == 0;
-          if (first && li > 0) {
+          const bool first = li == 0;  // later tiles add onto whatever the drains left
+          if (li > 0) {
             if (!mbar_wait_bounded(drained, ndrain & 1u, status, kAbort, a.wait_ns)) break;
             ndrain++;
             tc_fence_after_sync();
@@ -443,30 +463,64 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ compute warps
-    const int t = tid;  // row of the tile in the epilogue, component lane in drains
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    const int qd = warp & 3, hf = warp >> 2;
+    const int t = tid;                  // 0..255: position in the conversion loop
+    const int row = 32 * qd + lane;     // tile row (epilogue), component lane (drains)
+    const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
+    const int col0 = 64 * hf;           // this thread's 64 component columns
     double ll = 0.0;
     bool ok = true;
+    uint32_t ncbar = 0;                 // completed rendezvous on cbar
     const int G = D / 4;
 
-    auto drain = [&]() {
-      const int k = k0 + t;
-      for (int c = 0; c < nch; c++) {
-        float v0[32], v1[32];
-        tmem_ld32(tS + lane_base + 64u * c, v0);
-        tmem_ld32(tS + lane_base + 64u * c + 32u, v1);
-        if (k < K) {
-#pragma unroll
-          for (int j = 0; j < 32; j++) {
-            const int f0 = 64 * c + j, f1 = 64 * c + 32 + j;
-            if (f0 < 2 * D) slot[(size_t)f0 * K + k] += (double)v0[j];
-            if (f1 < 2 * D) slot[(size_t)f1 * K + k] += (double)v1[j];
-          }
-        }
-      }
+    // bounded rendezvous of the 256 compute threads
+    auto rendezvous = [&]() -> bool {
+      mbar_arrive(cbar);
+      const bool r = __all_sync(0xffffffffu,
+                                mbar_wait_bounded(cbar, ncbar & 1u, status, kAbort, a.wait_ns));
+      ncbar++;
+      return r;
+    };
+
+    // Drain component lane `row` into the fp64 slot and zero its accumulators,
+    // when it has mass since the last drain and `force` or it is precise.
+    // Column half 0 also owns the N_k column; the other half waits until N_k
+    // has been read by everyone before it is zeroed.
+    auto drain = [&](bool force) -> bool {
+      const int k = k0 + row;
       float vn[32];
       tmem_ld32(tNK + lane_base, vn);
-      if (k < K) slot[(size_t)(2 * D) * K + k] += (double)vn[0];
+      const bool due = k < K && vn[0] != 0.f && (force || precs[row] != 0);
+      if (!rendezvous()) return false;
+      if (!__any_sync(0xffffffffu, due)) return true;
+      double* sk = slot + k;
+      if (hf == 0) {
+        if (due) {
+          sk[(size_t)(2 * D) * K] += (double)vn[0];
+#pragma unroll
+          for (int j = 0; j < 32; j++) vn[j] = 0.f;
+        }
+        tmem_st32(tNK + lane_base, vn);
+      }
+      for (int c = 0; c < nch; c++) {
+        float v[32];
+        const uint32_t cc = tS + lane_base + 64u * c + 32u * hf;
+        tmem_ld32(cc, v);
+        if (due) {
+          const int f0 = 64 * c + 32 * hf;
+          const int nf = min(32, 2 * D - f0);  // features of this column block that exist
+          double acc[32];
+#pragma unroll
+          for (int j = 0; j < 32; j++) acc[j] = j < nf ? sk[(size_t)(f0 + j) * K] : 0.0;
+#pragma unroll
+          for (int j = 0; j < 32; j++)
+            if (j < nf) sk[(size_t)(f0 + j) * K] = acc[j] + (double)v[j];
+#pragma unroll
+          for (int j = 0; j < 32; j++) v[j] = 0.f;
+        }
+        tmem_st32(cc, v);
+      }
+      return true;
     };
 
     for (int64_t li = 0; li < my_tiles && ok; li++) {
@@ -477,52 +531,68 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                           a.wait_ns));
         if (!ok) break;
         tc_fence_after_sync();
-        if (MODE == kTcStats && (li % a.drain_tiles) == 0) {
-          drain();
+        if (MODE == kTcStats) {
+          ok = drain((li % a.drain_tiles) == 0);
+          if (!ok) break;
           tc_fence_before_sync();
           mbar_arrive(drained);
         }
       }
-      // ---- X tile -> F = [x^, x^^2] as fp16 hi/lo in the swizzled layout
+      // ---- X tile -> F = [x^, x^^2] as fp16 hi/lo in the swizzled layout;
+      // four 16-byte loads in flight per thread before any is converted
       bool bad = false, wide = false;
-      for (int u = t; u < kTcRows * G; u += 128) {
-        const int n = u / G, g = u - n * G;
-        const int64_t row = row0 + n;
-        float x[4] = {0.f, 0.f, 0.f, 0.f};
-        if (row < a.N) {
-          load4<XT>(reinterpret_cast<const XT*>(a.X), (size_t)row * D + 4 * g, x);
+      constexpr int kBatch = 4;
+      for (int u0 = t; u0 < kTcRows * G; u0 += kTcComputeThreads * kBatch) {
+        float xb[kBatch][4];
+#pragma unroll
+        for (int b = 0; b < kBatch; b++) {
+          const int u = u0 + b * kTcComputeThreads;
+          const int n = u / G, g = u - n * G;
+#pragma unroll
+          for (int j = 0; j < 4; j++) xb[b][j] = 0.f;
+          if (u < kTcRows * G && row0 + n < a.N)
+            load4<XT>(reinterpret_cast<const XT*>(a.X), (size_t)(row0 + n) * D + 4 * g, xb[b]);
+        }
+#pragma unroll
+        for (int b = 0; b < kBatch; b++) {
+          const int u = u0 + b * kTcComputeThreads;
+          if (u >= kTcRows * G) break;
+          const int n = u / G, g = u - n * G;
+          float x[4];
+          const bool live = row0 + n < a.N;
 #pragma unroll
           for (int j = 0; j < 4; j++) {
-            if (!isfinite(x[j])) bad = true;
-            x[j] = (x[j] - msm[4 * g + j]) * iscs[4 * g + j];
-            if (fabsf(x[j]) > kTcXMax) {
-              wide = true;
-              x[j] = copysignf(kTcXMax, x[j]);
+            x[j] = 0.f;
+            if (live) {
+              if (!isfinite(xb[b][j])) bad = true;
+              x[j] = (xb[b][j] - msm[4 * g + j]) * iscs[4 * g + j];
+              if (fabsf(x[j]) > kTcXMax) {
+                wide = true;
+                x[j] = copysignf(kTcXMax, x[j]);
+              }
             }
           }
-        }
-        float sq[4];
-        uint32_t hx[2], lx[2], hs[2], ls[2];
+          uint32_t hx[2], lx[2], hs[2], ls[2];
 #pragma unroll
-        for (int j = 0; j < 4; j++) sq[j] = x[j] * x[j];
-#pragma unroll
-        for (int h = 0; h < 2; h++) {
-          const float x0 = x[2 * h], x1 = x[2 * h + 1], s0 = sq[2 * h], s1 = sq[2 * h + 1];
-          const float x0h = round_half(x0), x1h = round_half(x1);
-          const float s0h = round_half(s0), s1h = round_half(s1);
-          hx[h] = pack_half2(x0h, x1h);
-          lx[h] = pack_half2(x0 - x0h, x1 - x1h);
-          hs[h] = pack_half2(s0h, s1h);
-          ls[h] = pack_half2(s0 - s0h, s1 - s1h);
+          for (int h = 0; h < 2; h++) {
+            const float x0 = x[2 * h], x1 = x[2 * h + 1];
+            const float s0 = x0 * x0, s1 = x1 * x1;
+            const float x0h = round_half(x0), x1h = round_half(x1);
+            const float s0h = round_half(s0), s1h = round_half(s1);
+            hx[h] = pack_half2(x0h, x1h);
+            lx[h] = pack_half2(x0 - x0h, x1 - x1h);
+            hs[h] = pack_half2(s0h, s1h);
+            ls[h] = pack_half2(s0 - s0h, s1 - s1h);
+          }
+          const int f1 = 4 * g, f2 = D + 4 * g;
+          const uint32_t o1 = (uint32_t)(f1 >> 6) * kTcChunkBytes + sw128_offset(n, f1 & 63);
+          const uint32_t o2 = (uint32_t)(f2 >> 6) * kTcChunkBytes + sw128_offset(n, f2 & 63);
+          const uint32_t lo_off = (uint32_t)nch * kTcChunkBytes;
+          *reinterpret_cast<uint2*>(sF + o1) = make_uint2(hx[0], hx[1]);
+          *reinterpret_cast<uint2*>(sF + lo_off + o1) = make_uint2(lx[0], lx[1]);
+          *reinterpret_cast<uint2*>(sF + o2) = make_uint2(hs[0], hs[1]);
+          *reinterpret_cast<uint2*>(sF + lo_off + o2) = make_uint2(ls[0], ls[1]);
         }
-        const int f1 = 4 * g, f2 = D + 4 * g;
-        const uint32_t o1 = (uint32_t)(f1 >> 6) * kTcChunkBytes + sw128_offset(n, f1 & 63);
-        const uint32_t o2 = (uint32_t)(f2 >> 6) * kTcChunkBytes + sw128_offset(n, f2 & 63);
-        const uint32_t lo_off = (uint32_t)nch * kTcChunkBytes;
-        *reinterpret_cast<uint2*>(sF + o1) = make_uint2(hx[0], hx[1]);
-        *reinterpret_cast<uint2*>(sF + lo_off + o1) = make_uint2(lx[0], lx[1]);
-        *reinterpret_cast<uint2*>(sF + o2) = make_uint2(hs[0], hs[1]);
-        *reinterpret_cast<uint2*>(sF + lo_off + o2) = make_uint2(ls[0], ls[1]);
       }
       if (bad) atomicOr(a.status, GMM_DEVFLAG_NONFINITE_X);
       if (wide) atomicOr(a.status, GMM_DEVFLAG_X_RANGE);
@@ -534,16 +604,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       mbar_wait_bounded(l_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns));
       if (!ok) break;
       tc_fence_after_sync();
-      // sharp components: direct-form log-joints of this row, written over the
-      // tensor-core values (their expanded-form constant is 0 and scale 1)
+      // sharp components of this column half: direct-form log-joints of this
+      // row, written over the tensor-core values (expanded constant 0, scale 1)
       const int nsh = shl[0];
       for (int si = 0; si < nsh; si++) {
         const int j = shl[1 + si];
+        if ((j >> 6) != hf) continue;
         const float* mk = a.muh + (size_t)(k0 + j) * D;
         const float* pk = a.ph + (size_t)(k0 + j) * D;
         float q = 0.f;
         for (int d = 0; d < D; d += 4) {
-          const uint32_t off = (uint32_t)(d >> 6) * kTcChunkBytes + sw128_offset(t, d & 63);
+          const uint32_t off = (uint32_t)(d >> 6) * kTcChunkBytes + sw128_offset(row, d & 63);
           const uint2 hv = *reinterpret_cast<const uint2*>(sF + off);
           const uint2 lv = *reinterpret_cast<const uint2*>(sF + (uint32_t)nch * kTcChunkBytes + off);
           const float4 m4 = __ldg(reinterpret_cast<const float4*>(mk + d));
@@ -552,8 +623,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
           const float2 l0 = __half22float2(*reinterpret_cast<const __half2*>(&lv.x));
           const float2 l1 = __half22float2(*reinterpret_cast<const __half2*>(&lv.y));
-          float e0 = (h0.x + l0.x) - m4.x, e1 = (h0.y + l0.y) - m4.y;
-          float e2 = (h1.x + l1.x) - m4.z, e3 = (h1.y + l1.y) - m4.w;
+          const float e0 = (h0.x + l0.x) - m4.x, e1 = (h0.y + l0.y) - m4.y;
+          const float e2 = (h1.x + l1.x) - m4.z, e3 = (h1.y + l1.y) - m4.w;
           q = fmaf(e0 * e0, p4.x, q);
           q = fmaf(e1 * e1, p4.y, q);
           q = fmaf(e2 * e2, p4.z, q);
@@ -561,28 +632,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tmem_st1(tL + lane_base + (uint32_t)j, cds[j] - 0.5f * q);
       }
-      float e[128];
+      float e[64];
       float mx = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < 4; q++) {
+      for (int q = 0; q < 2; q++) {
         float v[32];
-        tmem_ld32(tL + lane_base + 32u * q, v);
+        tmem_ld32(tL + lane_base + (uint32_t)(col0 + 32 * q), v);
 #pragma unroll
         for (int j = 0; j < 32; j++) {
-          e[32 * q + j] = fmaf(v[j], wscs[32 * q + j], csm[32 * q + j]);
+          const int cidx = col0 + 32 * q + j;
+          e[32 * q + j] = fmaf(v[j], wscs[cidx], csm[cidx]);
           mx = fmaxf(mx, e[32 * q + j]);
         }
       }
       float se = 0.f;
       if (mx > -INFINITY) {
 #pragma unroll
-        for (int j = 0; j < 128; j++) {
+        for (int j = 0; j < 64; j++) {
           e[j] = __expf(e[j] - mx);
           se += e[j];
         }
       }
+      // every (CTA, column half) contributes one (max, sum-exp) partial per row
       const uint32_t par = (uint32_t)(li & 1);
-      const uint32_t my_x = smem_u32(&xchg[(par * C + rank) * kTcRows + t]);
+      const uint32_t my_x = smem_u32(&xchg[((par * C + rank) * 2 + hf) * kTcRows + row]);
       for (int r2 = 0; r2 < C; r2++) st_cluster_f32x2(map_to_rank(my_x, r2), mx, se);
       const uint32_t xb = smem_u32(&xbar[par]);
       for (int r2 = 0; r2 < C; r2++) mbar_arrive_cluster(map_to_rank(xb, r2));
@@ -590,26 +663,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                                      status, kAbort, a.wait_ns, true));
       if (!ok) break;
       float M = -INFINITY;
-      for (int j = 0; j < C; j++) M = fmaxf(M, xchg[(par * C + j) * kTcRows + t].x);
+      for (int j = 0; j < 2 * C; j++) M = fmaxf(M, xchg[(par * C * 2 + j) * kTcRows + row].x);
       float S = 0.f;
-      for (int j = 0; j < C; j++) {
-        const float2 p = xchg[(par * C + j) * kTcRows + t];
+      for (int j = 0; j < 2 * C; j++) {
+        const float2 p = xchg[(par * C * 2 + j) * kTcRows + row];
         if (p.x > -INFINITY) S += p.y * __expf(p.x - M);
       }
       const float lse = M + __logf(S);
-      const bool valid = row0 + t < a.N;
-      if (valid && rank == 0) ll += (double)lse;
+      const bool valid = row0 + row < a.N;
+      if (valid && rank == 0 && hf == 0) ll += (double)lse;
       const float scale = (valid && mx > -INFINITY) ? __expf(mx - lse) * kTcRScale : 0.f;
-      const int half = t >> 6, rr = t & 63;
+      const int hr = row >> 6, rr = row & 63;  // which 64-row half of r^, row within it
       if (MODE == kTcStats) {
-        if (half == 1) {
+        if (hr == 1) {
           // the first half's MMAs must be done with the buffer
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(r_free, (uint32_t)(li & 1), status,
                                                          kAbort, a.wait_ns));
           if (!ok) break;
         }
 #pragma unroll
-        for (int q8 = 0; q8 < 16; q8++) {
+        for (int q8 = 0; q8 < 8; q8++) {
           float v[8], h[8];
 #pragma unroll
           for (int i = 0; i < 8; i++) {
@@ -622,29 +695,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                        pack_half2(v[2] - h[2], v[3] - h[3]),
                                        pack_half2(v[4] - h[4], v[5] - h[5]),
                                        pack_half2(v[6] - h[6], v[7] - h[7]));
-          const uint32_t off = (uint32_t)(q8 >> 3) * 8192u + (uint32_t)rr * 128u +
-                               ((((uint32_t)(q8 & 7)) ^ ((uint32_t)rr & 7u)) << 4);
+          const uint32_t off = (uint32_t)hf * 8192u + (uint32_t)rr * 128u +
+                               ((((uint32_t)q8) ^ ((uint32_t)rr & 7u)) << 4);
           *reinterpret_cast<uint4*>(sR + off) = ph4;
           *reinterpret_cast<uint4*>(sR + 16384u + off) = pl4;
         }
         fence_proxy_async_smem();
       }
       tc_fence_before_sync();
-      mbar_arrive(half == 0 ? r_full : r_full1);
+      mbar_arrive(hr == 0 ? r_full : r_full1);
     }
     if (ok && my_tiles > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(s_done, (uint32_t)((my_tiles - 1) & 1),
                                                      status, kAbort, a.wait_ns));
       tc_fence_after_sync();
-      if (ok && MODE == kTcStats) drain();
+      if (ok && MODE == kTcStats) ok = drain(true);
     }
-    // LL of this CTA's rows (rank 0 of each cluster only): fixed-order block sum
+    // LL of this CTA's rows (rank 0 of each cluster, column half 0): fixed-order sum
     ll = warp_sum(ll);
     double* red = reinterpret_cast<double*>(sR);  // r^ is no longer read by any MMA
     __syncwarp();
     if (lane == 0) red[warp] = ok ? ll : 0.0;
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (t == 0 && rank == 0) slot[ll_index] = ok ? red[0] + red[1] + red[2] + red[3] : 0.0;
+    const bool met = rendezvous();
+    if (t == 0 && rank == 0) {
+      double s = 0.0;
+      for (int w = 0; w < 8; w++) s += red[w];
+      slot[ll_index] = (ok && met) ? s : 0.0;
+    }
   }
 
   // ---------------------------------------------------------------- teardown
@@ -700,11 +777,12 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     const float* __restrict__ var, const float* __restrict__ m, const float* __restrict__ sc,
     __half* __restrict__ whi, __half* __restrict__ wlo, float* __restrict__ c_out,
     float* __restrict__ cd_out, float* __restrict__ wsc_out, int* __restrict__ sharp_out,
-    float* __restrict__ muh, float* __restrict__ ph, unsigned int* status) {
+    float* __restrict__ muh, float* __restrict__ ph, int* __restrict__ precise_out,
+    unsigned int* status) {
   __shared__ double wv[kTcChunk * kTcMaxChunks];  // Fpad <= 256
   __shared__ double red[4][4];
   const int k = blockIdx.x;
-  double s_log = 0.0, s_q = 0.0, kap = 0.0, amax = 0.0;
+  double s_log = 0.0, s_q = 0.0, kap = 0.0, amax = 0.0, rho = 0.0;
   bool bad = false;
   for (int f = threadIdx.x; f < Fpad; f += blockDim.x) {
     double v = 0.0;
@@ -719,6 +797,7 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
         s_log += log(2.0 * M_PI * vr);
         s_q += mh * mh / vh;
         kap += (mh * mh + 1.0) / vh;
+        if (k < K && w[k] > 0.f) rho = fmax(rho, mh * mh / vh);
         muh[(size_t)k * D + d] = (float)mh;
         ph[(size_t)k * D + d] = (float)(1.0 / vh);
         if (!isfinite(mu[(size_t)k * D + d]) || !(vr > 0.0) || !isfinite(vr)) bad = true;
@@ -745,6 +824,13 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
   const double S_q = red[1][0] + red[1][1] + red[1][2] + red[1][3];
   const double Kap = red[2][0] + red[2][1] + red[2][2] + red[2][3];
   const double Amax = fmax(fmax(red[3][0], red[3][1]), fmax(red[3][2], red[3][3]));
+  __syncthreads();
+  double t4 = rho;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t4 = fmax(t4, __shfl_xor_sync(0xffffffffu, t4, o));
+  if (lane == 0) red[0][wp] = t4;
+  __syncthreads();
+  const double Rho = fmax(fmax(red[0][0], red[0][1]), fmax(red[0][2], red[0][3]));
   int ex = 0;
   if (Amax > 0.0 && isfinite(Amax)) frexp(Amax, &ex);
   const int g = Amax > 0.0 ? ex - 14 : 0;
@@ -765,27 +851,28 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     c_out[k] = !live ? -INFINITY : (sharp ? 0.f : (float)(lw - 0.5 * (S_log + S_q)));
     wsc_out[k] = sharp ? 1.f : ldexpf(1.0f, g);
     sharp_out[k] = sharp ? 1 : 0;
+    precise_out[k] = live && (Rho > kTcRhoPrecise || small) ? 1 : 0;
   }
   if (bad) atomicOr(status, GMM_DEVFLAG_BAD_PARAMS);
 }
 
-// Fixed-order fp64 sum of the per-cluster slots and the M-step (statistics
-// are in scaled units: r * 2^15 and x^ = (x - m)/s):
-//   pi = N_k/N; if N_k > 1e-12 N: mu = m + s S1/N_k', var = max(s^2 (S2/N_k' - (S1/N_k')^2), floor)
-// with N_k' the scaled count.
-__global__ void __launch_bounds__(256) tc_reduce_mstep_kernel(
-    int64_t N, int D, int K, float var_floor, const float* __restrict__ m,
-    const float* __restrict__ sc, const double* __restrict__ slots, size_t slot_stride,
-    int nslots, float* __restrict__ w, float* __restrict__ mu, float* __restrict__ var,
-    double* __restrict__ loglik) {
+// Fixed-order fp64 sum of the per-cluster slots into the canonical
+// statistics buffer [ N_k | A | B | LL ] (component-major, moments about the
+// input means mu, data units).  The slots hold N' = 2^15 N_k and
+// S1' = 2^15 sum r x^, S2' = 2^15 sum r x^^2 with x^ = (x - m)/s, so with
+// dm = mu - m:  A = s S1 - dm N,  B = s^2 S2 - 2 s dm S1 + dm^2 N.
+__global__ void __launch_bounds__(256) tc_reduce_stats_kernel(
+    int D, int K, const float* __restrict__ m, const float* __restrict__ sc,
+    const float* __restrict__ mu, const double* __restrict__ slots, size_t slot_stride,
+    int nslots, double* __restrict__ stats) {
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const size_t ll_index = (size_t)(2 * D + 1) * K;
-  if (i == 0 && loglik) {
+  const size_t KD = (size_t)K * D;
+  if (i == 0) {
     double ll = 0.0;
-    for (int p = 0; p < nslots; p++) ll += slots[(size_t)p * slot_stride + ll_index];
-    *loglik = ll;
+    for (int p = 0; p < nslots; p++) ll += slots[(size_t)p * slot_stride + (size_t)(2 * D + 1) * K];
+    stats[K + 2 * KD] = ll;
   }
-  if (i >= (size_t)K * D) return;
+  if (i >= KD) return;
   const int d = (int)(i / K), k = (int)(i - (size_t)d * K);
   double nks = 0.0, s1 = 0.0, s2 = 0.0;
   for (int p = 0; p < nslots; p++) {
@@ -794,16 +881,13 @@ __global__ void __launch_bounds__(256) tc_reduce_mstep_kernel(
     s1 += s[(size_t)d * K + k];
     s2 += s[(size_t)(D + d) * K + k];
   }
-  const double nk = nks / (double)kTcRScale;
-  if (d == 0) w[k] = (float)(nk / (double)N);
-  if (nk > 1e-12 * (double)N) {
-    const double sd = (double)sc[d];
-    const double mt = s1 / nks;
-    double v = (s2 / nks - mt * mt) * sd * sd;
-    if (!(v > (double)var_floor)) v = (double)var_floor;
-    mu[(size_t)k * D + d] = (float)((double)m[d] + sd * mt);
-    var[(size_t)k * D + d] = (float)v;
-  }
+  const double inv = 1.0 / (double)kTcRScale;
+  const double n = nks * inv, S1 = s1 * inv, S2 = s2 * inv;
+  const double sd = (double)sc[d];
+  const double dm = (double)mu[(size_t)k * D + d] - (double)m[d];
+  if (d == 0) stats[k] = n;
+  stats[K + (size_t)k * D + d] = sd * S1 - dm * n;
+  stats[K + KD + (size_t)k * D + d] = sd * sd * S2 - 2.0 * sd * dm * S1 + dm * dm * n;
 }
 
 __global__ void tc_reduce_loglik_kernel(int D, int K, const double* __restrict__ slots,

@@ -20,8 +20,8 @@ GMM_F32, GMM_BF16 = 0, 1
 GMM_INIT_VAR_ONE, GMM_INIT_VAR_DATA = 0, 1
 GMM_DEVFLAG_NONFINITE_X, GMM_DEVFLAG_BAD_PARAMS, GMM_DEVFLAG_WAIT_TIMEOUT = 0x1, 0x2, 0x4
 
-EXPORTS = ("gmm_workspace_size", "gmm_init", "gmm_em_step", "gmm_em_step_noalloc", "gmm_fit",
-           "gmm_loglik",
+EXPORTS = ("gmm_workspace_size", "gmm_init", "gmm_em_step", "gmm_em_step_noalloc",
+           "gmm_estep_stats", "gmm_mstep", "gmm_fit", "gmm_loglik",
            "gmm_assign_topm", "gmm_device_status", "gmm_trace_fused", "gmm_launch_count",
            "gmm_status_string")
 
@@ -55,6 +55,8 @@ def load_library(path: str = LIB_PATH):
     lib.gmm_init.argtypes = [PP, P, ctypes.POINTER(I64), I32, P, P, P, P, SZ, P]
     lib.gmm_em_step.argtypes = [PP, P, P, P, P, P, P, SZ, P]
     lib.gmm_em_step_noalloc.argtypes = [PP, P, P, P, P, P, P, P]
+    lib.gmm_estep_stats.argtypes = [PP, P, P, P, P, P, P, SZ, P]
+    lib.gmm_mstep.argtypes = [PP, P, I32, P, P, P, P, P]
     lib.gmm_fit.argtypes = [PP, P, I32, P, P, P, P, P, SZ, P]
     lib.gmm_loglik.argtypes = [PP, P, P, P, P, P, P, SZ, P]
     lib.gmm_assign_topm.argtypes = [PP, P, P, P, P, I32, P, P, P, SZ, P]
@@ -141,6 +143,38 @@ def gmm_em_step(X, w, mu, var, loglik=None, var_floor=1e-6, ws=None, stream=None
     _check(load_library().gmm_em_step(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu), _ptr(var),
                                       _ptr(loglik), _ptr(ws), ws.numel(), _stream(stream)),
            "gmm_em_step")
+
+
+def stats_size(K, D) -> int:
+    """Doubles in a statistics buffer: [N_k (K) | A (K x D) | B (K x D) | LL]."""
+    return int(K) * (2 * int(D) + 1) + 1
+
+
+def gmm_estep_stats(X, w, mu, var, stats=None, var_floor=1e-6, ws=None, stream=None):
+    """E-step statistics of the rows of X (fp64 device tensor [N_k | A | B | LL])."""
+    p = problem_for(X, w.numel(), var_floor)
+    ws = _ws(p, ws, X.device)
+    if stats is None:
+        stats = torch.empty(stats_size(w.numel(), X.shape[1]), dtype=torch.float64,
+                            device=X.device)
+    _check(load_library().gmm_estep_stats(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu), _ptr(var),
+                                          _ptr(stats), _ptr(ws), ws.numel(), _stream(stream)),
+           "gmm_estep_stats")
+    return stats
+
+
+def gmm_mstep(stats, N_total, w, mu, var, loglik=None, var_floor=1e-6, xdtype=GMM_F32,
+              stream=None):
+    """M-step in place from the statistics of row shards holding N_total points.
+
+    stats: fp64 device tensor of shape (S,) or (nshards, S), S = stats_size(K, D);
+    the shards are summed in order inside the library."""
+    K, D = mu.shape
+    nshards = 1 if stats.dim() == 1 else stats.shape[0]
+    p = problem(N_total, D, K, xdtype, var_floor)
+    _check(load_library().gmm_mstep(ctypes.byref(p), _ptr(stats.contiguous()), int(nshards),
+                                    _ptr(w), _ptr(mu), _ptr(var), _ptr(loglik), _stream(stream)),
+           "gmm_mstep")
 
 
 def gmm_em_step_noalloc(X, w, mu, var, loglik=None, dev_flags=None, var_floor=1e-6,

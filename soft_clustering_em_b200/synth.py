@@ -109,13 +109,15 @@ def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
-def make_data(wl: Workload, N: int = None, chunk: int = 1 << 16):
-    """Sample X (N x D) of workload ``wl``.
+def make_data(wl: Workload, N: int = None, chunk: int = 1 << 16, start: int = 0):
+    """Sample rows [start, start + N) of workload ``wl``'s data stream.
 
     Returns (X, labels).  X is float32, or uint16 bf16 bit patterns when
-    wl.dtype == "bf16".  Rows are generated in chunks so the result does not
-    depend on N except through truncation of the same stream: the first n rows
-    of make_data(wl, N) equal make_data(wl, n) for n <= N.
+    wl.dtype == "bf16".  The stream is cut into chunks of ``chunk`` rows, each
+    drawn from its own seeded generator, so any block of rows is the same
+    whatever else is generated: make_data(wl, n) is a prefix of
+    make_data(wl, N) for n <= N, and make_data(wl, n, start=s) equals rows
+    s .. s+n-1 of a longer draw (one block of rows per rank).
     """
     N = wl.N if N is None else int(N)
     pi, mu, sd, rng = true_params(wl)
@@ -124,16 +126,19 @@ def make_data(wl: Workload, N: int = None, chunk: int = 1 << 16):
     labels = np.empty(N, dtype=np.int32)
     cdf = np.cumsum(pi)
     cdf[-1] = 1.0
-    for c0 in range(0, N, chunk):
-        # every chunk draws from its own seeded stream, so prefixes are stable
-        crng = np.random.Generator(np.random.PCG64([wl.data_seed, c0 // chunk]))
-        n = min(chunk, N - c0)
-        z = np.searchsorted(cdf, crng.random(n), side="right").astype(np.int32)
+    stop = start + N
+    for ci in range(start // chunk, (stop + chunk - 1) // chunk):
+        c0 = ci * chunk
+        crng = np.random.Generator(np.random.PCG64([wl.data_seed, ci]))
+        z = np.searchsorted(cdf, crng.random(chunk), side="right").astype(np.int32)
         z = np.minimum(z, wl.K - 1)
-        eps = crng.standard_normal(size=(n, wl.D))
-        x = _finish(wl, mu[z] + sd[z] * eps).astype(np.float32)
-        X[c0:c0 + n] = bf16_round(x) if wl.dtype == "bf16" else x
-        labels[c0:c0 + n] = z
+        lo, hi = max(start, c0), min(stop, c0 + chunk)
+        # draw the whole chunk so its rows do not depend on the block requested
+        eps = crng.standard_normal(size=(hi - c0, wl.D))[lo - c0:]
+        zz = z[lo - c0:hi - c0]
+        x = _finish(wl, mu[zz] + sd[zz] * eps).astype(np.float32)
+        X[lo - start:hi - start] = bf16_round(x) if wl.dtype == "bf16" else x
+        labels[lo - start:hi - start] = zz
     return X, labels
 
 

@@ -27,7 +27,8 @@ def declared_functions():
 
 def test_header_declares_the_calls():
     names = declared_functions()
-    for n in ("gmm_init", "gmm_em_step", "gmm_em_step_noalloc", "gmm_fit", "gmm_loglik",
+    for n in ("gmm_init", "gmm_em_step", "gmm_em_step_noalloc", "gmm_estep_stats", "gmm_mstep",
+              "gmm_fit", "gmm_loglik",
               "gmm_assign_topm", "gmm_workspace_size", "gmm_device_status", "gmm_trace_fused",
               "gmm_launch_count", "gmm_status_string"):
         assert n in names
@@ -108,3 +109,17 @@ def test_trace_hook_arguments(lib):
     P = ctypes.c_void_p
     assert lib.gmm_trace_fused(P(16), None) == G.GMM_ERR_INVALID_ARG
     assert lib.gmm_trace_fused(None, None) == G.GMM_OK
+
+
+def test_split_step_argument_checks(lib):
+    P = ctypes.c_void_p
+    p = G.problem(10, 4, 3)
+    assert lib.gmm_estep_stats(ctypes.byref(p), P(16), P(16), P(16), P(16), P(0), P(256), 1 << 30,
+                               P(0)) == G.GMM_ERR_INVALID_ARG
+    assert lib.gmm_mstep(ctypes.byref(p), P(0), 1, P(16), P(16), P(16), P(0), P(0)) == \
+        G.GMM_ERR_INVALID_ARG
+    assert lib.gmm_mstep(ctypes.byref(p), P(16), 0, P(16), P(16), P(16), P(0), P(0)) == \
+        G.GMM_ERR_INVALID_ARG
+    bad = G.problem(0, 4, 3)
+    assert lib.gmm_mstep(ctypes.byref(bad), P(16), 1, P(16), P(16), P(16), P(0), P(0)) == \
+        G.GMM_ERR_INVALID_ARG

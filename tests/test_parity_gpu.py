@@ -304,3 +304,64 @@ def test_tensor_core_and_cuda_core_paths_agree(G, name, N, K, monkeypatch):
     nk = outs[1][0] * N
     rep = compare.compare_step(outs[1], outs[0], nk)
     assert rep["ok"], rep
+
+
+@pytest.mark.parametrize("name,N,K", [("uint8img", 20_011, 256), ("bf16stream", 30_001, 1024),
+                                      ("sphere768", 2_003, 1024)])
+def test_estep_statistics_match_oracle(G, name, N, K):
+    """gmm_estep_stats returns [N_k | A | B | LL] about the input means, the
+    same quantities (and layout) as the oracle's E-step statistics."""
+    import torch
+
+    wl = synth.WORKLOADS[name]
+    X, _ = synth.make_data(wl, N)
+    X64 = synth.x_as_f64(wl, X)
+    Xd = to_device(wl, X)
+    ws = G.workspace(G.problem_for(Xd, K, wl.var_floor))
+    w, mu, var = G.gmm_init(Xd, synth.init_rows(N, K, wl.init_seed), K, 1, wl.var_floor, ws=ws)
+    G.gmm_em_step(Xd, w, mu, var, None, wl.var_floor, ws=ws)
+    th = params_np(w, mu, var)
+    st = G.gmm_estep_stats(Xd, w, mu, var, None, wl.var_floor, ws=ws).cpu().numpy()
+    Nk, A, B, ll = oracle.estep_stats(X64, *th)
+    D = X.shape[1]
+    gN, gA = st[:K], st[K:K + K * D].reshape(K, D)
+    gB, gll = st[K + K * D:K + 2 * K * D].reshape(K, D), st[-1]
+    np.testing.assert_allclose(gN, Nk, rtol=1e-3, atol=1e-9 * N)
+    gate = Nk >= 10
+    # a sum of deviations is judged against its natural scale sqrt(N_k * B)
+    scale = np.sqrt(np.maximum(Nk[:, None] * B, 1e-300))
+    assert np.all(np.abs(gA - A)[gate] <= 1e-3 * scale[gate] + 1e-9)
+    assert np.all(np.abs(gB - B)[gate] <= 1e-3 * B[gate] + 1e-12)
+    assert abs(gll - ll) <= compare.LL_REL * abs(ll)
+
+
+@pytest.mark.parametrize("name,N,K,shards", [("uint8img", 40_000, 256, 3),
+                                             ("bf16stream", 50_000, 1024, 2)])
+def test_row_shards_sum_to_the_full_step(G, name, N, K, shards):
+    """Statistics of disjoint row blocks, summed by gmm_mstep in shard order,
+    give the same M-step as one gmm_em_step over all rows."""
+    import torch
+
+    from soft_clustering_em_b200 import sharded
+
+    wl = synth.WORKLOADS[name]
+    X, _ = synth.make_data(wl, N)
+    Xd = to_device(wl, X)
+    ws = G.workspace(G.problem_for(Xd, K, wl.var_floor))
+    w, mu, var = G.gmm_init(Xd, synth.init_rows(N, K, wl.init_seed), K, 1, wl.var_floor, ws=ws)
+    full = [w.clone(), mu.clone(), var.clone()]
+    ll_full = torch.zeros(1, dtype=torch.float64, device="cuda")
+    G.gmm_em_step(Xd, *full, ll_full, wl.var_floor, ws=ws)
+    parts = []
+    for r in range(shards):
+        lo, hi = sharded.shard_rows(N, shards, r)
+        Xs = Xd[lo:hi]
+        wss = G.workspace(G.problem_for(Xs, K, wl.var_floor))
+        parts.append(G.gmm_estep_stats(Xs, w, mu, var, None, wl.var_floor, ws=wss))
+    ll_sh = torch.zeros(1, dtype=torch.float64, device="cuda")
+    sh = [w.clone(), mu.clone(), var.clone()]
+    G.gmm_mstep(torch.stack(parts), N, *sh, ll_sh, wl.var_floor, G.xdtype_of(Xd))
+    nk = full[0].double().cpu().numpy() * N
+    rep = compare.compare_step((*params_np(*full), ll_full.item()), (*params_np(*sh), ll_sh.item()),
+                               nk)
+    assert rep["ok"], rep
