@@ -175,7 +175,7 @@ gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const 
       p->N, p->D, p->K, T.Fpad, w, mu, var, m, (const float*)(ws + T.sc), (__half*)(ws + T.whi),
       (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.cd), (float*)(ws + T.wsc),
       (int*)(ws + T.sharp), (float*)(ws + T.muh), (float*)(ws + T.ph),
-      (int*)(ws + T.precise), (unsigned int*)ws);
+      (int*)(ws + T.precise), (float*)(ws + T.ci), (unsigned int*)ws);
   return launched(2);
 }
 
@@ -235,6 +235,7 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, char* ws, const TcLayo
   args.m = (const float*)(ws + T.m);
   args.isc = (const float*)(ws + T.isc);
   args.c = (const float*)(ws + T.c);
+  args.ci = (const float*)(ws + T.ci);
   args.cd = (const float*)(ws + T.cd);
   args.wsc = (const float*)(ws + T.wsc);
   args.sharp = (const int*)(ws + T.sharp);
@@ -570,3 +571,15 @@ gmm_status gmm_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* 
 }
 
 }  // extern "C"
+
+#ifdef SCEM_PHASE_TRACE
+// Performance-work builds only: copy the phase timestamps of the last
+// tensor-core pass to the host.
+extern "C" int scem_phase_trace_read(unsigned long long* host, int n) {
+  if (n > 64 * 16) n = 64 * 16;
+  return cudaMemcpyFromSymbol(host, scem::g_phase_trace, sizeof(unsigned long long) * n) ==
+                 cudaSuccess
+             ? 0
+             : 1;
+}
+#endif

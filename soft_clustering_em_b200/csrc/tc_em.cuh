@@ -15,15 +15,19 @@
 // F and W = [a, b] are split into fp16 pairs (hi + lo, 22 significant bits;
 // each W row carries its own power-of-two scale so it sits in fp16 range) and
 // the contraction takes F_hi W_hi + F_lo W_hi + F_hi W_lo (the lo*lo term is
-// below fp32 rounding), accumulated in fp32 in tensor memory.
+// below fp32 rounding), accumulated in fp32 in tensor memory, starting from
+// -5/8 sum_d mu^^2/var^ rather than zero (kTcStartFrac); c_k absorbs the split's
+// systematic error on the component's own points (tc_prep_w_kernel).
 //
 // Sharp components.  The expanded form cancels: its fp32 error grows with
 // kappa_k = sum_d (mu^_kd^2 + 1) / var^_kd, up to ~1e-3 nat at kappa ~ 1e5.
 // A component with kappa_k > 1e7 (in practice one collapsed onto a few points,
-// at the variance floor), or with kappa_k > 3e3 while it expects fewer than 20
-// points (pi_k N < 20, where such an error moves its weight by ~1e-3), gets its
-// log-joints recomputed in direct form, sum_d (x^ - mu^)^2 / var^, on the CUDA
-// cores and written over the tensor-core value in tensor memory.
+// at the variance floor), or with kappa_k > 500 while it expects fewer than 50
+// points (pi_k N < 50, where such an error moves its weight by ~1e-3), gets its
+// log-joints recomputed in direct form, sum_d (x - mu)^2 / var in data units
+// from X itself (the fp16 split of x^ is too coarse next to a narrow
+// component's width), on the CUDA cores, written over the tensor-core value
+// in tensor memory.
 //
 // Statistics.  r is scaled by 2^15 and split into an fp16 pair r^ = r_hi +
 // r_lo (about 22 significant bits; fp16 alone leaves components that hold a
@@ -77,18 +81,44 @@ constexpr double kTcRhoPrecise = 64.0;  // rho_k above which a component drains 
 constexpr uint32_t kTcChunkBytes = 128u * 128u;  // one [128 x 64] 16-bit operand chunk
 constexpr float kTcRScale = 32768.0f;            // r is stored as fp16(r * 2^15)
 constexpr double kTcSharpKappa = 1e7;            // direct form above this kappa_k ...
-constexpr double kTcSmallKappa = 3e3;            // ... or above this one for a component
-constexpr double kTcSmallPoints = 20.0;          //     expecting fewer points than this
+constexpr double kTcSmallKappa = 500.0;          // ... or above this one for a component
+constexpr double kTcSmallPoints = 50.0;          //     expecting fewer points than this
 constexpr float kTcXMax = 240.0f;                // |x^| beyond this cannot be split into fp16
+// Start value of the E-step accumulator, as a multiple of Q_k = sum_d mu^^2/var^.
+// For a point the component explains, the linear K-steps add about +Q_k and
+// the quadratic ones about -Q_k/2 (over as many accumulations), so from
+// -5/8 Q_k the partial sums run -5/8 -> +3/8 -> -1/8 (in Q_k): they stay below
+// Q_k in size and spend as long above zero as below it.  The tensor core's
+// fp32 accumulation rounds toward zero (measured on sm_100a: its N_k errors
+// follow that model, not round-to-nearest), so its errors then cancel instead
+// of adding up; from zero they would grow with Q_k, which reaches 10^4 for
+// tight components far from the centring point.
+constexpr double kTcStartFrac = -0.625;
 
 enum TcMode { kTcStats = 0, kTcLoglik = 1 };
+
+// Optional phase timestamps for performance work (off unless the library is
+// built with -DSCEM_PHASE_TRACE): slot `idx` of the first 64 tiles of cluster
+// 0, rank 0, taken by compute thread 0 or the MMA thread.
+#ifdef SCEM_PHASE_TRACE
+__device__ unsigned long long g_phase_trace[64 * 16];
+#define SCEM_TRACE(li, idx)                                                  \
+  do {                                                                       \
+    if (cid == 0 && rank == 0 && (li) < 64)                                  \
+      g_phase_trace[(li) * 16 + (idx)] = sm100::globaltimer_ns();            \
+  } while (0)
+#else
+#define SCEM_TRACE(li, idx) \
+  do {                      \
+  } while (0)
+#endif
 
 inline int tc_nchunks(int D) { return (2 * D + kTcChunk - 1) / kTcChunk; }
 inline int tc_cluster(int K) { return (K + kTcComps - 1) / kTcComps; }
 
 // Byte offsets of the kernel's shared-memory regions (from a 1024-aligned base).
 struct TcSmem {
-  uint32_t F, W, R, ONES, msm, iscs, csm, wscs, cds, shl, precs, xchg, bars, tslot, total;
+  uint32_t F, W, R, ONES, msm, iscs, csm, cis, wscs, cds, shl, precs, xchg, bars, tslot, total;
 };
 
 __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
@@ -108,12 +138,14 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
   off += ((uint32_t)D * 4 + 15) & ~15u;
   L.csm = off;
   off += kTcComps * 4;
+  L.cis = off;
+  off += kTcComps * 4;
   L.wscs = off;
   off += kTcComps * 4;
   L.cds = off;
   off += kTcComps * 4;
   L.shl = off;
-  off += (kTcComps + 4) * 4;
+  off += (kTcComps + 8) * 4;
   L.precs = off;
   off += kTcComps * 4;
   L.xchg = off;
@@ -128,17 +160,20 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 
 // Workspace layout of the tensor-core path (after the 256-byte status block).
 //   m, isc, sc : D f32 centring vector, 1/s and s (powers of two)
-//   c    : C*128 f32 per-component constants of the expanded form (0 if sharp)
+//   c    : C*128 f32 per-component constants of the expanded form: the part
+//          added in the epilogue (0 if sharp)
+//   ci   : C*128 f32 the part of that constant the accumulator starts from, in
+//          units of the W row scale (0 if sharp)
 //   cd   : C*128 f32 per-component constants of the direct form
 //   wsc  : C*128 f32 power-of-two scale of each W row (1 if sharp)
 //   sharp: C*128 int32 1 if the component's log-joints are computed in direct form
-//   muh, ph : [C*128 x D] f32 mu^ and 1/var^ for the direct form
+//   muh, ph : [C*128 x D] f32 mu and 1/var (data units) for the direct form
 //   whi, wlo : [C*128 x 64*nchunks] fp16 operand W (hi and lo parts)
 //   slots: P per-cluster slots of slot_stride doubles:
 //          [(2D+1) x K] feature-major statistics (S1 rows 0..D-1, S2 rows
 //          D..2D-1, N_k row 2D) followed by the cluster's LL.
 struct TcLayout {
-  size_t m, isc, sc, c, cd, wsc, sharp, precise, muh, ph, whi, wlo, slots, total, slot_stride;
+  size_t m, isc, sc, c, ci, cd, wsc, sharp, precise, muh, ph, whi, wlo, slots, total, slot_stride;
   int C, nchunks, Kpad, Fpad, P;
 };
 
@@ -162,6 +197,8 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   L.sc = off;
   off = align_up(off + (size_t)D * 4, 256);
   L.c = off;
+  off = align_up(off + (size_t)L.Kpad * 4, 256);
+  L.ci = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.cd = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
@@ -197,7 +234,9 @@ struct TcArgs {
   int D, K, C, nchunks;
   const float* m;       // centring vector, D
   const float* isc;     // 1/s, D
-  const float* c;       // expanded-form constants, C*128 (-inf for padding / pi = 0)
+  const float* c;       // expanded-form constants added in the epilogue, C*128
+                        // (-inf for padding / pi = 0)
+  const float* ci;      // accumulator start values (W-row-scale units), C*128
   const float* cd;      // direct-form constants, C*128
   const float* wsc;     // W row scales, C*128
   const int* sharp;     // direct-form flags, C*128
@@ -211,12 +250,26 @@ struct TcArgs {
   uint64_t wait_ns;
 };
 
+// A shared-memory descriptor advanced by `bytes` (start-address field only;
+// every operand lies within the first 256 KB of shared memory, so no carry).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 __device__ __forceinline__ float round_half(float a) { return __half2float(__float2half_rn(a)); }
+
+// (a, b) -> fp16 pairs hi = fp16(a, b) and lo = fp16(a - hi_a, b - hi_b), packed:
+// three conversion instructions for two values.
+__device__ __forceinline__ void split_half2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(a, b);
+  const float2 f = __half22float2(h);
+  const __half2 l = __floats2half2_rn(a - f.x, b - f.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
 
 template <typename XT>
 __device__ __forceinline__ void load4(const XT* X, size_t i, float (&x)[4]);
@@ -257,6 +310,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* msm = reinterpret_cast<float*>(sm + L.msm);
   float* iscs = reinterpret_cast<float*>(sm + L.iscs);
   float* csm = reinterpret_cast<float*>(sm + L.csm);
+  float* cis = reinterpret_cast<float*>(sm + L.cis);
   float* wscs = reinterpret_cast<float*>(sm + L.wscs);
   float* cds = reinterpret_cast<float*>(sm + L.cds);
   int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = local indices
@@ -302,8 +356,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init(s_done, 1);
     mbar_init(drained, kTcComputeThreads);
     mbar_init(cbar, kTcComputeThreads);
-    mbar_init(&xbar[0], (uint32_t)C * kTcComputeThreads);
-    mbar_init(&xbar[1], (uint32_t)C * kTcComputeThreads);
+    mbar_init(&xbar[0], (uint32_t)C * (kTcComputeThreads / 32));  // one arrive per warp
+    mbar_init(&xbar[1], (uint32_t)C * (kTcComputeThreads / 32));
     mbar_init(final_bar, 1);
     fence_mbar_init();
   }
@@ -317,15 +371,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   for (int i = tid; i < kTcComps; i += kTcThreads) {
     csm[i] = a.c[k0 + i];
+    cis[i] = a.ci[k0 + i];
     wscs[i] = a.wsc[k0 + i];
     cds[i] = a.cd[k0 + i];
     precs[i] = a.precise[k0 + i];
   }
   if (tid == 0) {
     int n = 0;
+    uint32_t mw[4] = {0u, 0u, 0u, 0u};
     for (int j = 0; j < kTcComps; j++)
-      if (a.sharp[k0 + j]) shl[1 + n++] = j;
+      if (a.sharp[k0 + j]) {
+        shl[1 + n++] = j;
+        mw[j >> 5] |= 1u << (j & 31);
+      }
     shl[0] = n;
+    for (int q = 0; q < 4; q++) shl[kTcComps + q] = (int)mw[q];  // bit j: local component j
   }
   for (int i = tid; i < 2048; i += kTcThreads)
     reinterpret_cast<__half*>(sOnes)[i] = __float2half_rn(1.0f);
@@ -381,13 +441,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idE = idesc_f16_f32(128, 128, false, false);
-      const uint32_t idS = idesc_f16_f32(128, 64, true, true);
+      // one statistics MMA covers all 64*nch features: the chunks are MN atoms 16 KB apart
+      const uint32_t idS = idesc_f16_f32(128, 64 * nch, true, true);
       const uint32_t idN = idesc_f16_f32(128, 16, true, false);
       const uint32_t fb = smem_u32(sF), wb = smem_u32(sW), rb = smem_u32(sR);
       const uint32_t ob = smem_u32(sOnes);
+      const uint64_t dF = sw128_desc(fb, 16, 1024);        // F as the K-major E-step A operand
+      const uint64_t dW = sw128_desc(wb, 16, 1024);        // W stage as the E-step B operand
+      const uint64_t dFs = sw128_desc(fb, 16384, 1024);    // F as the MN-major statistics B
+      const uint64_t dR = sw128_desc(rb, 8192, 1024);      // r^ as the MN-major statistics A
+      const uint64_t dOnes = sw128_desc(ob, 16, 1024);
       uint32_t stage = 0, phase = 0, ndrain = 0;
       for (int64_t li = 0; li < my_tiles; li++) {
         if (!mbar_wait_bounded(f_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) break;
+        SCEM_TRACE(li, 8);
         tc_fence_after_sync();
         bool ok = true;
         for (int c = 0; c < nch && ok; c++) {
@@ -397,13 +464,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ok = mbar_wait_bounded(&full[stage], phase, status, kAbort, a.wait_ns);
             if (!ok) break;
             tc_fence_after_sync();
-            const uint32_t w = wb + stage * kTcChunkBytes;
+            const uint64_t wd = desc_add(dW, stage * kTcChunkBytes);
+            const uint64_t fhd = desc_add(dF, fhi - fb), fld = desc_add(dF, flo - fb);
 #pragma unroll
             for (int ks = 0; ks < 4; ks++) {
-              const uint64_t bd = sw128_desc(w + 32u * ks, 16, 1024);
-              mma_bf16(tL, sw128_desc(fhi + 32u * ks, 16, 1024), bd, idE,
-                       !(part == 0 && c == 0 && ks == 0));
-              if (part == 0) mma_bf16(tL, sw128_desc(flo + 32u * ks, 16, 1024), bd, idE, true);
+              const uint64_t bd = desc_add(wd, 32u * ks);
+              mma_bf16(tL, desc_add(fhd, 32u * ks), bd, idE, true);  // onto the start values
+              if (part == 0) mma_bf16(tL, desc_add(fld, 32u * ks), bd, idE, true);
             }
             mma_commit(&empty[stage]);
             if (++stage == kTcStages) {
@@ -414,7 +481,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (!ok) break;
         mma_commit(l_full);
+        SCEM_TRACE(li, 9);
         if (!mbar_wait_bounded(r_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) break;
+        SCEM_TRACE(li, 10);
         tc_fence_after_sync();
         bool ok2 = true;
         if (MODE == kTcStats) {
@@ -431,23 +500,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               if (!ok2) break;
               tc_fence_after_sync();
             }
-#pragma unroll 1
+#pragma unroll
             for (int ks = 0; ks < 4; ks++) {
-              const uint64_t ahi = sw128_desc(rb + 2048u * ks, 8192, 1024);
-              const uint64_t alo = sw128_desc(rb + 16384u + 2048u * ks, 8192, 1024);
+              const uint64_t ahi = desc_add(dR, 2048u * ks);
+              const uint64_t alo = desc_add(dR, 16384u + 2048u * ks);
               const bool acc = !(first && half == 0 && ks == 0);
               const uint32_t kr = 2048u * (uint32_t)(4 * half + ks);  // F rows of this K-step
-              for (int c = 0; c < nch; c++) {
-                const uint64_t fhi = sw128_desc(fb + (uint32_t)c * kTcChunkBytes + kr, 16384, 1024);
-                const uint64_t flo =
-                    sw128_desc(fb + (uint32_t)(nch + c) * kTcChunkBytes + kr, 16384, 1024);
-                mma_bf16(tS + 64u * c, ahi, fhi, idS, acc);
-                mma_bf16(tS + 64u * c, ahi, flo, idS, true);
-                mma_bf16(tS + 64u * c, alo, fhi, idS, true);
-              }
-              const uint64_t od = sw128_desc(ob, 16, 1024);
-              mma_bf16(tNK, ahi, od, idN, acc);
-              mma_bf16(tNK, alo, od, idN, true);
+              const uint64_t fhi = desc_add(dFs, kr);
+              const uint64_t flo = desc_add(dFs, (uint32_t)nch * kTcChunkBytes + kr);
+              mma_bf16(tS, ahi, fhi, idS, acc);
+              mma_bf16(tS, ahi, flo, idS, true);
+              mma_bf16(tS, alo, fhi, idS, true);
+              mma_bf16(tNK, ahi, dOnes, idN, acc);
+              mma_bf16(tNK, alo, dOnes, idN, true);
             }
           }
         } else {
@@ -456,6 +521,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (!ok2) break;
         mma_commit(s_done);
+        SCEM_TRACE(li, 11);
       }
       // every MMA issued must be complete before tensor memory is released
       mma_commit(final_bar);
@@ -523,25 +589,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       return true;
     };
 
+    // The E-step accumulator of each tile starts from -5/8 Q_k (kTcStartFrac,
+    // in W-row-scale units; the rest of the constant is added in the
+    // epilogue) rather than from zero, so that its rounding errors cancel.
+    // Each thread writes its own row and column half; the stores are waited
+    // on before the F-full arrive.
+    auto store_start = [&]() {
+#pragma unroll
+      for (int q = 0; q < 2; q++) {
+        float v[32];
+#pragma unroll
+        for (int j4 = 0; j4 < 8; j4++) {
+          const float4 c4 = reinterpret_cast<const float4*>(cis + col0 + 32 * q)[j4];
+          v[4 * j4 + 0] = c4.x;
+          v[4 * j4 + 1] = c4.y;
+          v[4 * j4 + 2] = c4.z;
+          v[4 * j4 + 3] = c4.w;
+        }
+        tmem_st32_nowait(tL + lane_base + (uint32_t)(col0 + 32 * q), v);
+      }
+    };
+    if (my_tiles > 0) store_start();
+
     for (int64_t li = 0; li < my_tiles && ok; li++) {
       const int64_t row0 = ((int64_t)cid + li * ncl) * kTcRows;
+      if (t == 0) SCEM_TRACE(li, 0);
       if (li > 0) {
         ok = __all_sync(0xffffffffu,
                         mbar_wait_bounded(s_done, (uint32_t)((li - 1) & 1), status, kAbort,
                                           a.wait_ns));
         if (!ok) break;
+        if (t == 0) SCEM_TRACE(li, 1);
         tc_fence_after_sync();
         if (MODE == kTcStats) {
           ok = drain((li % a.drain_tiles) == 0);
+          if (t == 0) SCEM_TRACE(li, 2);
           if (!ok) break;
           tc_fence_before_sync();
           mbar_arrive(drained);
         }
       }
-      // ---- X tile -> F = [x^, x^^2] as fp16 hi/lo in the swizzled layout;
-      // four 16-byte loads in flight per thread before any is converted
+      // ---- X tile -> F = [x^, x^^2] as fp16 hi/lo in the swizzled layout.
+      // The next tile's rows (contiguous in X) are pulled into L2 now, so that
+      // its loads meet L2 rather than DRAM latency; up to 16 16-byte loads per
+      // thread are in flight before any is converted.
+      if (t == 0 && li + 1 < my_tiles) {
+        const int64_t nrow0 = row0 + (int64_t)ncl * kTcRows;
+        const int64_t nrows = min((int64_t)kTcRows, a.N - nrow0);
+        if (nrows > 0)
+          prefetch_l2_bulk(reinterpret_cast<const XT*>(a.X) + (size_t)nrow0 * D,
+                           (uint32_t)((size_t)nrows * D * sizeof(XT)));
+      }
       bool bad = false, wide = false;
-      constexpr int kBatch = 4;
+      constexpr int kBatch = 16;
+      int nbatch = 0;
       for (int u0 = t; u0 < kTcRows * G; u0 += kTcComputeThreads * kBatch) {
         float xb[kBatch][4];
 #pragma unroll
@@ -553,6 +654,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (u < kTcRows * G && row0 + n < a.N)
             load4<XT>(reinterpret_cast<const XT*>(a.X), (size_t)(row0 + n) * D + 4 * g, xb[b]);
         }
+        if (t == 0 && nbatch == 0) SCEM_TRACE(li, 12);
 #pragma unroll
         for (int b = 0; b < kBatch; b++) {
           const int u = u0 + b * kTcComputeThreads;
@@ -560,12 +662,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int n = u / G, g = u - n * G;
           float x[4];
           const bool live = row0 + n < a.N;
+          const float4 m4 = reinterpret_cast<const float4*>(msm)[g];
+          const float4 i4 = reinterpret_cast<const float4*>(iscs)[g];
+          const float mv[4] = {m4.x, m4.y, m4.z, m4.w}, iv[4] = {i4.x, i4.y, i4.z, i4.w};
 #pragma unroll
           for (int j = 0; j < 4; j++) {
             x[j] = 0.f;
             if (live) {
               if (!isfinite(xb[b][j])) bad = true;
-              x[j] = (xb[b][j] - msm[4 * g + j]) * iscs[4 * g + j];
+              x[j] = (xb[b][j] - mv[j]) * iv[j];
               if (fabsf(x[j]) > kTcXMax) {
                 wide = true;
                 x[j] = copysignf(kTcXMax, x[j]);
@@ -576,13 +681,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int h = 0; h < 2; h++) {
             const float x0 = x[2 * h], x1 = x[2 * h + 1];
-            const float s0 = x0 * x0, s1 = x1 * x1;
-            const float x0h = round_half(x0), x1h = round_half(x1);
-            const float s0h = round_half(s0), s1h = round_half(s1);
-            hx[h] = pack_half2(x0h, x1h);
-            lx[h] = pack_half2(x0 - x0h, x1 - x1h);
-            hs[h] = pack_half2(s0h, s1h);
-            ls[h] = pack_half2(s0 - s0h, s1 - s1h);
+            split_half2(x0, x1, hx[h], lx[h]);
+            split_half2(x0 * x0, x1 * x1, hs[h], ls[h]);
           }
           const int f1 = 4 * g, f2 = D + 4 * g;
           const uint32_t o1 = (uint32_t)(f1 >> 6) * kTcChunkBytes + sw128_offset(n, f1 & 63);
@@ -593,58 +693,76 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           *reinterpret_cast<uint2*>(sF + o2) = make_uint2(hs[0], hs[1]);
           *reinterpret_cast<uint2*>(sF + lo_off + o2) = make_uint2(ls[0], ls[1]);
         }
+        if (t == 0) SCEM_TRACE(li, 13 + min(nbatch, 2));
+        nbatch++;
       }
       if (bad) atomicOr(a.status, GMM_DEVFLAG_NONFINITE_X);
       if (wide) atomicOr(a.status, GMM_DEVFLAG_X_RANGE);
       fence_proxy_async_smem();
+      tmem_wait_st();  // the accumulator's start values are in place
+      tc_fence_before_sync();
       mbar_arrive(f_full);
+      if (t == 0) SCEM_TRACE(li, 3);
 
       // ---- epilogue: logits -> row max / sum-exp -> cluster exchange -> r^
       ok = __all_sync(0xffffffffu,
                       mbar_wait_bounded(l_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns));
       if (!ok) break;
+      if (t == 0) SCEM_TRACE(li, 4);
       tc_fence_after_sync();
-      // sharp components of this column half: direct-form log-joints of this
-      // row, written over the tensor-core values (expanded constant 0, scale 1)
-      const int nsh = shl[0];
-      for (int si = 0; si < nsh; si++) {
-        const int j = shl[1 + si];
-        if ((j >> 6) != hf) continue;
-        const float* mk = a.muh + (size_t)(k0 + j) * D;
-        const float* pk = a.ph + (size_t)(k0 + j) * D;
-        float q = 0.f;
-        for (int d = 0; d < D; d += 4) {
-          const uint32_t off = (uint32_t)(d >> 6) * kTcChunkBytes + sw128_offset(row, d & 63);
-          const uint2 hv = *reinterpret_cast<const uint2*>(sF + off);
-          const uint2 lv = *reinterpret_cast<const uint2*>(sF + (uint32_t)nch * kTcChunkBytes + off);
-          const float4 m4 = __ldg(reinterpret_cast<const float4*>(mk + d));
-          const float4 p4 = __ldg(reinterpret_cast<const float4*>(pk + d));
-          const float2 h0 = __half22float2(*reinterpret_cast<const __half2*>(&hv.x));
-          const float2 h1 = __half22float2(*reinterpret_cast<const __half2*>(&hv.y));
-          const float2 l0 = __half22float2(*reinterpret_cast<const __half2*>(&lv.x));
-          const float2 l1 = __half22float2(*reinterpret_cast<const __half2*>(&lv.y));
-          const float e0 = (h0.x + l0.x) - m4.x, e1 = (h0.y + l0.y) - m4.y;
-          const float e2 = (h1.x + l1.x) - m4.z, e3 = (h1.y + l1.y) - m4.w;
-          q = fmaf(e0 * e0, p4.x, q);
-          q = fmaf(e1 * e1, p4.y, q);
-          q = fmaf(e2 * e2, p4.z, q);
-          q = fmaf(e3 * e3, p4.w, q);
-        }
-        tmem_st1(tL + lane_base + (uint32_t)j, cds[j] - 0.5f * q);
-      }
       float e[64];
       float mx = -INFINITY;
+      auto load_logits = [&](bool skip_sharp, uint32_t m0, uint32_t m1) {
+        mx = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < 2; q++) {
-        float v[32];
-        tmem_ld32(tL + lane_base + (uint32_t)(col0 + 32 * q), v);
+        for (int q = 0; q < 2; q++) {
+          float v[32];
+          tmem_ld32(tL + lane_base + (uint32_t)(col0 + 32 * q), v);
+          const uint32_t mq = q ? m1 : m0;
 #pragma unroll
-        for (int j = 0; j < 32; j++) {
-          const int cidx = col0 + 32 * q + j;
-          e[32 * q + j] = fmaf(v[j], wscs[cidx], csm[cidx]);
-          mx = fmaxf(mx, e[32 * q + j]);
+          for (int j = 0; j < 32; j++) {
+            const int cidx = col0 + 32 * q + j;
+            e[32 * q + j] = fmaf(v[j], wscs[cidx], csm[cidx]);
+            if (!(skip_sharp && ((mq >> j) & 1u))) mx = fmaxf(mx, e[32 * q + j]);
+          }
         }
+      };
+      const uint32_t sm0 = (uint32_t)shl[kTcComps + 2 * hf], sm1 = (uint32_t)shl[kTcComps + 2 * hf + 1];
+      load_logits(true, sm0, sm1);
+      if (sm0 | sm1) {
+        // sharp components of this column half: direct-form log-joints of this
+        // row written over the tensor-core values (expanded constant 0, scale 1);
+        // a row stops summing once the component is 80 nats below the best
+        // non-sharp component of this half (its responsibility is then 0)
+        const float floor_l = mx - 80.f;
+        const int nsh = shl[0];
+        const bool rvalid = row0 + row < a.N;
+        const XT* xrow = reinterpret_cast<const XT*>(a.X) + (size_t)(rvalid ? row0 + row : 0) * D;
+        for (int si = 0; si < nsh; si++) {
+          const int j = shl[1 + si];
+          if ((j >> 6) != hf) continue;
+          const float* mk = a.muh + (size_t)(k0 + j) * D;
+          const float* pk = a.ph + (size_t)(k0 + j) * D;
+          const float qmax = 2.f * (cds[j] - floor_l);  // q beyond this: below the floor
+          float q = 0.f;
+          for (int d = 0; d < D && q <= qmax; d += 4) {
+            float x4[4];
+            load4<XT>(xrow, (size_t)d, x4);
+            const float4 m4 = __ldg(reinterpret_cast<const float4*>(mk + d));
+            const float4 p4 = __ldg(reinterpret_cast<const float4*>(pk + d));
+            const float e0 = x4[0] - m4.x, e1 = x4[1] - m4.y;
+            const float e2 = x4[2] - m4.z, e3 = x4[3] - m4.w;
+            q = fmaf(e0 * e0, p4.x, q);
+            q = fmaf(e1 * e1, p4.y, q);
+            q = fmaf(e2 * e2, p4.z, q);
+            q = fmaf(e3 * e3, p4.w, q);
+          }
+          tmem_st1(tL + lane_base + (uint32_t)j, q <= qmax ? cds[j] - 0.5f * q : -INFINITY);
+        }
+        load_logits(false, 0u, 0u);
       }
+      if (li + 1 < my_tiles) store_start();  // L is no longer read in this tile
+      if (t == 0) SCEM_TRACE(li, 5);
       float se = 0.f;
       if (mx > -INFINITY) {
 #pragma unroll
@@ -657,11 +775,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t par = (uint32_t)(li & 1);
       const uint32_t my_x = smem_u32(&xchg[((par * C + rank) * 2 + hf) * kTcRows + row]);
       for (int r2 = 0; r2 < C; r2++) st_cluster_f32x2(map_to_rank(my_x, r2), mx, se);
-      const uint32_t xb = smem_u32(&xbar[par]);
-      for (int r2 = 0; r2 < C; r2++) mbar_arrive_cluster(map_to_rank(xb, r2));
+      __syncwarp();  // the warp's stores happen before lane 0's release-arrive
+      if (lane == 0) {
+        const uint32_t xb = smem_u32(&xbar[par]);
+        for (int r2 = 0; r2 < C; r2++) mbar_arrive_cluster(map_to_rank(xb, r2));
+      }
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&xbar[par], (uint32_t)((li >> 1) & 1),
                                                      status, kAbort, a.wait_ns, true));
       if (!ok) break;
+      if (t == 0) SCEM_TRACE(li, 6);
       float M = -INFINITY;
       for (int j = 0; j < 2 * C; j++) M = fmaxf(M, xchg[(par * C * 2 + j) * kTcRows + row].x);
       float S = 0.f;
@@ -683,18 +805,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
 #pragma unroll
         for (int q8 = 0; q8 < 8; q8++) {
-          float v[8], h[8];
-#pragma unroll
-          for (int i = 0; i < 8; i++) {
-            v[i] = e[8 * q8 + i] * scale;
-            h[i] = round_half(v[i]);
-          }
-          const uint4 ph4 = make_uint4(pack_half2(h[0], h[1]), pack_half2(h[2], h[3]),
-                                       pack_half2(h[4], h[5]), pack_half2(h[6], h[7]));
-          const uint4 pl4 = make_uint4(pack_half2(v[0] - h[0], v[1] - h[1]),
-                                       pack_half2(v[2] - h[2], v[3] - h[3]),
-                                       pack_half2(v[4] - h[4], v[5] - h[5]),
-                                       pack_half2(v[6] - h[6], v[7] - h[7]));
+          uint4 ph4, pl4;
+          split_half2(e[8 * q8 + 0] * scale, e[8 * q8 + 1] * scale, ph4.x, pl4.x);
+          split_half2(e[8 * q8 + 2] * scale, e[8 * q8 + 3] * scale, ph4.y, pl4.y);
+          split_half2(e[8 * q8 + 4] * scale, e[8 * q8 + 5] * scale, ph4.z, pl4.z);
+          split_half2(e[8 * q8 + 6] * scale, e[8 * q8 + 7] * scale, ph4.w, pl4.w);
           const uint32_t off = (uint32_t)hf * 8192u + (uint32_t)rr * 128u +
                                ((((uint32_t)q8) ^ ((uint32_t)rr & 7u)) << 4);
           *reinterpret_cast<uint4*>(sR + off) = ph4;
@@ -704,6 +819,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tc_fence_before_sync();
       mbar_arrive(hr == 0 ? r_full : r_full1);
+      if (t == 0) SCEM_TRACE(li, 7);
     }
     if (ok && my_tiles > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(s_done, (uint32_t)((my_tiles - 1) & 1),
@@ -725,6 +841,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 
   // ---------------------------------------------------------------- teardown
+  if (warp < kTcMmaWarp) tmem_wait_st();
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 0) {
@@ -772,20 +889,32 @@ __global__ void tc_center_kernel(int D, int K, const float* __restrict__ w,
 // power of two 2^-g_k so its largest entry lies in [2^13, 2^14), split into
 // fp16 hi/lo rows of Fpad features (padding rows and features zero); the
 // constants of both forms; kappa_k and the direct-form tables mu^, 1/var^.
+//
+// The expanded-form constant c_k = log pi_k - (1/2) sum_d [log(2 pi var_kd) +
+// mu^_kd^2 / var^_kd] is corrected for the part of W that the fp16 hi/lo split
+// drops: the MMA sums F (W_hi + W_lo) 2^g, short of F W 2^g by F dW 2^g with
+// dW = W 2^-g - W_hi - W_lo, known exactly here.  For the points the component
+// explains F is near its expectation E[F] = [mu^, mu^^2 + var^], so
+// 2^g E[F] . dW is added to c_k: that removes the split's systematic error on
+// those points (what remains is (F - E[F]) . dW, of either sign from point to
+// point).  The accumulator starts from ci_k = kTcStartFrac sum_d mu^^2/var^
+// (fp32, in 2^g units); the fp32 remainder c_k - 2^g ci_k is added after the
+// MMAs.
 __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     int64_t N, int D, int K, int Fpad, const float* __restrict__ w, const float* __restrict__ mu,
     const float* __restrict__ var, const float* __restrict__ m, const float* __restrict__ sc,
     __half* __restrict__ whi, __half* __restrict__ wlo, float* __restrict__ c_out,
     float* __restrict__ cd_out, float* __restrict__ wsc_out, int* __restrict__ sharp_out,
     float* __restrict__ muh, float* __restrict__ ph, int* __restrict__ precise_out,
-    unsigned int* status) {
+    float* __restrict__ ci_out, unsigned int* status) {
   __shared__ double wv[kTcChunk * kTcMaxChunks];  // Fpad <= 256
+  __shared__ double ef[kTcChunk * kTcMaxChunks];  // E[F] under the component
   __shared__ double red[4][4];
   const int k = blockIdx.x;
   double s_log = 0.0, s_q = 0.0, kap = 0.0, amax = 0.0, rho = 0.0;
   bool bad = false;
   for (int f = threadIdx.x; f < Fpad; f += blockDim.x) {
-    double v = 0.0;
+    double v = 0.0, e = 0.0;
     if (k < K && f < 2 * D) {
       const int d = f < D ? f : f - D;
       const double sd = (double)sc[d];
@@ -794,18 +923,21 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
       const double mh = ((double)mu[(size_t)k * D + d] - (double)m[d]) / sd;
       if (f < D) {
         v = mh / vh;
+        e = mh;
         s_log += log(2.0 * M_PI * vr);
         s_q += mh * mh / vh;
         kap += (mh * mh + 1.0) / vh;
         if (k < K && w[k] > 0.f) rho = fmax(rho, mh * mh / vh);
-        muh[(size_t)k * D + d] = (float)mh;
-        ph[(size_t)k * D + d] = (float)(1.0 / vh);
+        muh[(size_t)k * D + d] = mu[(size_t)k * D + d];
+        ph[(size_t)k * D + d] = (float)(1.0 / vr);
         if (!isfinite(mu[(size_t)k * D + d]) || !(vr > 0.0) || !isfinite(vr)) bad = true;
       } else {
         v = -0.5 / vh;
+        e = mh * mh + vh;
       }
     }
     wv[f] = v;
+    ef[f] = e;
     amax = fmax(amax, fabs(v));
   }
   const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
@@ -834,12 +966,21 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
   int ex = 0;
   if (Amax > 0.0 && isfinite(Amax)) frexp(Amax, &ex);
   const int g = Amax > 0.0 ? ex - 14 : 0;
+  double dsplit = 0.0;  // E[F] . dW in 2^g units
   for (int f = threadIdx.x; f < Fpad; f += blockDim.x) {
-    const float sv = (float)ldexp(wv[f], -g);
+    const double svd = ldexp(wv[f], -g);
+    const float sv = (float)svd;
     const __half h = __float2half_rn(sv);
+    const __half l = __float2half_rn(sv - __half2float(h));
     whi[(size_t)k * Fpad + f] = h;
-    wlo[(size_t)k * Fpad + f] = __float2half_rn(sv - __half2float(h));
+    wlo[(size_t)k * Fpad + f] = l;
+    dsplit += ef[f] * (svd - (double)__half2float(h) - (double)__half2float(l));
   }
+  dsplit = warp_sum(dsplit);
+  __syncthreads();  // every thread is done reading red[0][*] (Rho)
+  if (lane == 0) red[1][wp] = dsplit;
+  __syncthreads();
+  const double Dsplit = red[1][0] + red[1][1] + red[1][2] + red[1][3];
   if (threadIdx.x == 0) {
     const float wk = k < K ? w[k] : 0.f;
     if (k < K && (!isfinite(wk) || !(wk >= 0.f))) bad = true;
@@ -848,7 +989,10 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     const bool sharp = live && (Kap > kTcSharpKappa || (small && Kap > kTcSmallKappa));
     const double lw = live ? log((double)wk) : 0.0;
     cd_out[k] = live ? (float)(lw - 0.5 * S_log) : -INFINITY;
-    c_out[k] = !live ? -INFINITY : (sharp ? 0.f : (float)(lw - 0.5 * (S_log + S_q)));
+    const double cfull = lw - 0.5 * (S_log + S_q) + ldexp(Dsplit, g);
+    const float cstart = (live && !sharp) ? (float)ldexp(kTcStartFrac * S_q, -g) : 0.f;
+    ci_out[k] = cstart;
+    c_out[k] = !live ? -INFINITY : (sharp ? 0.f : (float)(cfull - ldexp((double)cstart, g)));
     wsc_out[k] = sharp ? 1.f : ldexpf(1.0f, g);
     sharp_out[k] = sharp ? 1 : 0;
     precise_out[k] = live && (Rho > kTcRhoPrecise || small) ? 1 : 0;
