@@ -173,9 +173,10 @@ gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const 
                                                        (float*)(ws + T.isc), (float*)(ws + T.sc));
   tc_prep_w_kernel<<<T.Kpad, 128, 0, st>>>(
       p->N, p->D, p->K, T.Fpad, w, mu, var, m, (const float*)(ws + T.sc), (__half*)(ws + T.whi),
-      (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.cd), (float*)(ws + T.wsc),
-      (int*)(ws + T.sharp), (float*)(ws + T.muh), (float*)(ws + T.ph),
-      (int*)(ws + T.precise), (float*)(ws + T.ci), (unsigned int*)ws);
+      (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.wsc), (int*)(ws + T.sharp),
+      (int*)(ws + T.nsplit), (float*)(ws + T.muh), (float*)(ws + T.ph), (int*)(ws + T.precise),
+      (float*)(ws + T.ci), (uint8_t*)(ws + T.perm), (float*)(ws + T.mhp), (float*)(ws + T.php),
+      (unsigned int*)ws);
   return launched(2);
 }
 
@@ -236,11 +237,14 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, char* ws, const TcLayo
   args.isc = (const float*)(ws + T.isc);
   args.c = (const float*)(ws + T.c);
   args.ci = (const float*)(ws + T.ci);
-  args.cd = (const float*)(ws + T.cd);
   args.wsc = (const float*)(ws + T.wsc);
   args.sharp = (const int*)(ws + T.sharp);
+  args.nsplit = (const int*)(ws + T.nsplit);
   args.muh = (const float*)(ws + T.muh);
   args.ph = (const float*)(ws + T.ph);
+  args.perm = (const uint8_t*)(ws + T.perm);
+  args.mhp = (const float*)(ws + T.mhp);
+  args.php = (const float*)(ws + T.php);
   args.slots = (double*)(ws + T.slots);
   args.slot_stride = T.slot_stride;
   args.status = (unsigned int*)ws;

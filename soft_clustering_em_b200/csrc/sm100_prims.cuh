@@ -104,6 +104,11 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
+// Hint: bring the line holding `p` into L1 (no register, no wait).
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -217,6 +222,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 
 // Each thread of the warp writes one 32-bit value to column `taddr`'s column
 // of its own lane (32 lanes x 1 column), and waits for the store to land.
+// 32 lanes x 1 column: thread i reads its own lane (base lane + i) at `taddr`'s
+// column, and waits for the value.
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r)
+      : "r"(taddr)
+      : "memory");
+  return __uint_as_float(r);
+}
+
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};\n\t"

@@ -19,15 +19,17 @@
 // -5/8 sum_d mu^^2/var^ rather than zero (kTcStartFrac); c_k absorbs the split's
 // systematic error on the component's own points (tc_prep_w_kernel).
 //
-// Sharp components.  The expanded form cancels: its fp32 error grows with
-// kappa_k = sum_d (mu^_kd^2 + 1) / var^_kd, up to ~1e-3 nat at kappa ~ 1e5.
-// A component with kappa_k > 1e7 (in practice one collapsed onto a few points,
-// at the variance floor), or with kappa_k > 500 while it expects fewer than 50
-// points (pi_k N < 50, where such an error moves its weight by ~1e-3), gets its
-// log-joints recomputed in direct form, sum_d (x - mu)^2 / var in data units
-// from X itself (the fp16 split of x^ is too coarse next to a narrow
-// component's width), on the CUDA cores, written over the tensor-core value
-// in tensor memory.
+// Split dimensions.  The expanded form cancels: its fp32 error grows with
+// kappa_k = sum_d (mu^_kd^2 + 1) / var^_kd.  A component with kappa_k > 1e7 (in
+// practice one collapsed onto a few points at the variance floor in some
+// dimensions), or with kappa_k > 2e4 while it expects fewer than 50 points,
+// has its dimensions with the largest shares of kappa_k -- just enough that
+// the rest sum below the threshold -- taken out of the contraction (zero W).
+// For each row the CUDA cores add -1/2 sum (x - mu)^2 / var over those
+// dimensions, in data units from X itself (the fp16 split of x^ is too coarse
+// next to a narrow dimension), onto the tensor-core log-joint of the rest,
+// after a cheap filter on the tile's own features drops the rows that are
+// certainly far below the best component.
 //
 // Statistics.  r is scaled by 2^15 and split into an fp16 pair r^ = r_hi +
 // r_lo (about 22 significant bits; fp16 alone leaves components that hold a
@@ -72,6 +74,7 @@ constexpr int kTcComps = 128;     // components per CTA
 constexpr int kTcChunk = 64;      // features per operand chunk (one swizzled 128-byte row)
 constexpr int kTcStages = 3;      // depth of the W ring
 constexpr int kTcMaxChunks = 4;   // 2D <= 256
+constexpr int kTcMaxD = 128;
 constexpr int kTcMaxCluster = 16;
 constexpr int kTcThreads = 320;          // 8 compute warps + MMA warp + TMA warp
 constexpr int kTcComputeThreads = 256;
@@ -81,7 +84,7 @@ constexpr double kTcRhoPrecise = 64.0;  // rho_k above which a component drains 
 constexpr uint32_t kTcChunkBytes = 128u * 128u;  // one [128 x 64] 16-bit operand chunk
 constexpr float kTcRScale = 32768.0f;            // r is stored as fp16(r * 2^15)
 constexpr double kTcSharpKappa = 1e7;            // direct form above this kappa_k ...
-constexpr double kTcSmallKappa = 500.0;          // ... or above this one for a component
+constexpr double kTcSmallKappa = 2.0e4;          // ... or above this one for a component
 constexpr double kTcSmallPoints = 50.0;          //     expecting fewer points than this
 constexpr float kTcXMax = 240.0f;                // |x^| beyond this cannot be split into fp16
 // Start value of the E-step accumulator, as a multiple of Q_k = sum_d mu^^2/var^.
@@ -118,7 +121,7 @@ inline int tc_cluster(int K) { return (K + kTcComps - 1) / kTcComps; }
 
 // Byte offsets of the kernel's shared-memory regions (from a 1024-aligned base).
 struct TcSmem {
-  uint32_t F, W, R, ONES, msm, iscs, csm, cis, wscs, cds, shl, precs, xchg, bars, tslot, total;
+  uint32_t F, W, R, ONES, msm, iscs, csm, cis, wscs, shl, precs, xchg, bars, tslot, total;
 };
 
 __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
@@ -142,8 +145,6 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
   off += kTcComps * 4;
   L.wscs = off;
   off += kTcComps * 4;
-  L.cds = off;
-  off += kTcComps * 4;
   L.shl = off;
   off += (kTcComps + 8) * 4;
   L.precs = off;
@@ -164,16 +165,20 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //          added in the epilogue (0 if sharp)
 //   ci   : C*128 f32 the part of that constant the accumulator starts from, in
 //          units of the W row scale (0 if sharp)
-//   cd   : C*128 f32 per-component constants of the direct form
 //   wsc  : C*128 f32 power-of-two scale of each W row (1 if sharp)
-//   sharp: C*128 int32 1 if the component's log-joints are computed in direct form
-//   muh, ph : [C*128 x D] f32 mu and 1/var (data units) for the direct form
+//   sharp: C*128 int32 1 if some of the component's dimensions are summed in
+//          direct form (nsplit: C*128 int32, how many: the first nsplit of perm)
+//   perm : [C*128 x D] u8 dimensions of each component by decreasing
+//          (mu^^2 + 1)/var^
+//   muh, ph : [C*128 x D] f32 mu and 1/var (data units) in perm order
+//   mhp, php : [C*128 x D] f32 mu^ and 1/var^ in perm order
 //   whi, wlo : [C*128 x 64*nchunks] fp16 operand W (hi and lo parts)
 //   slots: P per-cluster slots of slot_stride doubles:
 //          [(2D+1) x K] feature-major statistics (S1 rows 0..D-1, S2 rows
 //          D..2D-1, N_k row 2D) followed by the cluster's LL.
 struct TcLayout {
-  size_t m, isc, sc, c, ci, cd, wsc, sharp, precise, muh, ph, whi, wlo, slots, total, slot_stride;
+  size_t m, isc, sc, c, ci, wsc, sharp, nsplit, precise, muh, ph, perm, mhp, php, whi, wlo, slots,
+      total, slot_stride;
   int C, nchunks, Kpad, Fpad, P;
 };
 
@@ -200,15 +205,21 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.ci = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
-  L.cd = off;
-  off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.wsc = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.sharp = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
+  L.nsplit = off;
+  off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.muh = off;
   off = align_up(off + (size_t)L.Kpad * D * 4, 256);
   L.ph = off;
+  off = align_up(off + (size_t)L.Kpad * D * 4, 256);
+  L.perm = off;
+  off = align_up(off + (size_t)L.Kpad * D, 256);
+  L.mhp = off;
+  off = align_up(off + (size_t)L.Kpad * D * 4, 256);
+  L.php = off;
   off = align_up(off + (size_t)L.Kpad * D * 4, 256);
   L.whi = off;
   off = align_up(off + (size_t)L.Kpad * L.Fpad * 2, 256);
@@ -237,11 +248,14 @@ struct TcArgs {
   const float* c;       // expanded-form constants added in the epilogue, C*128
                         // (-inf for padding / pi = 0)
   const float* ci;      // accumulator start values (W-row-scale units), C*128
-  const float* cd;      // direct-form constants, C*128
   const float* wsc;     // W row scales, C*128
-  const int* sharp;     // direct-form flags, C*128
-  const float* muh;     // mu^, C*128 x D
-  const float* ph;      // 1/var^, C*128 x D
+  const int* sharp;     // 1: some dimensions in direct form, C*128
+  const int* nsplit;    // how many (the first of perm), C*128
+  const float* muh;     // mu (data units) in perm order, C*128 x D
+  const float* ph;      // 1/var (data units) in perm order, C*128 x D
+  const uint8_t* perm;  // dimensions by decreasing (mu^^2 + 1)/var^, C*128 x D
+  const float* mhp;     // mu^ in that order, C*128 x D
+  const float* php;     // 1/var^ in that order, C*128 x D
   double* slots;        // per-cluster statistic slots
   size_t slot_stride;   // doubles per slot: (2D+1)*K statistics + LL
   unsigned int* status;
@@ -293,6 +307,19 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* X, siz
   x[3] = __high2float(b);
 }
 
+template <typename XT>
+__device__ __forceinline__ float load1(const XT* X, int i);
+template <>
+__device__ __forceinline__ float load1<float>(const float* X, int i) {
+  return __ldg(X + i);
+}
+template <>
+__device__ __forceinline__ float load1<__nv_bfloat16>(const __nv_bfloat16* X, int i) {
+  return __bfloat162float(X[i]);
+}
+
+// 10 warps put 3 on some of the 4 sub-partitions (16K registers each): 168 registers
+// per thread at most.
 template <typename XT, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fused_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tm_whi,
@@ -312,7 +339,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* csm = reinterpret_cast<float*>(sm + L.csm);
   float* cis = reinterpret_cast<float*>(sm + L.cis);
   float* wscs = reinterpret_cast<float*>(sm + L.wscs);
-  float* cds = reinterpret_cast<float*>(sm + L.cds);
   int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = local indices
   int* precs = reinterpret_cast<int*>(sm + L.precs);
   float2* xchg = reinterpret_cast<float2*>(sm + L.xchg);  // [2][C][2][128] (max, sum-exp)
@@ -373,7 +399,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     csm[i] = a.c[k0 + i];
     cis[i] = a.ci[k0 + i];
     wscs[i] = a.wsc[k0 + i];
-    cds[i] = a.cd[k0 + i];
     precs[i] = a.precise[k0 + i];
   }
   if (tid == 0) {
@@ -559,10 +584,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const bool due = k < K && vn[0] != 0.f && (force || precs[row] != 0);
       if (!rendezvous()) return false;
       if (!__any_sync(0xffffffffu, due)) return true;
+      // Fire-and-forget fp64 reductions into the slot: one thread owns each
+      // address, so the additions land in program order (deterministic) and
+      // the thread does not wait for the old value.
       double* sk = slot + k;
       if (hf == 0) {
         if (due) {
-          sk[(size_t)(2 * D) * K] += (double)vn[0];
+          if (vn[0] != 0.f) atomicAdd(sk + (size_t)(2 * D) * K, (double)vn[0]);
 #pragma unroll
           for (int j = 0; j < 32; j++) vn[j] = 0.f;
         }
@@ -575,12 +603,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (due) {
           const int f0 = 64 * c + 32 * hf;
           const int nf = min(32, 2 * D - f0);  // features of this column block that exist
-          double acc[32];
-#pragma unroll
-          for (int j = 0; j < 32; j++) acc[j] = j < nf ? sk[(size_t)(f0 + j) * K] : 0.0;
 #pragma unroll
           for (int j = 0; j < 32; j++)
-            if (j < nf) sk[(size_t)(f0 + j) * K] = acc[j] + (double)v[j];
+            if (j < nf && v[j] != 0.f) atomicAdd(sk + (size_t)(f0 + j) * K, (double)v[j]);
 #pragma unroll
           for (int j = 0; j < 32; j++) v[j] = 0.f;
         }
@@ -712,7 +737,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after_sync();
       float e[64];
       float mx = -INFINITY;
-      auto load_logits = [&](bool skip_sharp, uint32_t m0, uint32_t m1) {
+      // first pass (final = false): every column is an accumulator value,
+      // scaled to a log-joint; columns in the mask (split components) stay out
+      // of the max.  Second pass (final = true): the masked columns already
+      // hold finished log-joints.
+      auto load_logits = [&](bool final, uint32_t m0, uint32_t m1) {
         mx = -INFINITY;
 #pragma unroll
         for (int q = 0; q < 2; q++) {
@@ -722,44 +751,108 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; j++) {
             const int cidx = col0 + 32 * q + j;
-            e[32 * q + j] = fmaf(v[j], wscs[cidx], csm[cidx]);
-            if (!(skip_sharp && ((mq >> j) & 1u))) mx = fmaxf(mx, e[32 * q + j]);
+            const bool masked = (mq >> j) & 1u;
+            e[32 * q + j] = (final && masked) ? v[j] : fmaf(v[j], wscs[cidx], csm[cidx]);
+            if (final || !masked) mx = fmaxf(mx, e[32 * q + j]);
           }
         }
       };
       const uint32_t sm0 = (uint32_t)shl[kTcComps + 2 * hf], sm1 = (uint32_t)shl[kTcComps + 2 * hf + 1];
-      load_logits(true, sm0, sm1);
+      load_logits(false, sm0, sm1);
       if (sm0 | sm1) {
-        // sharp components of this column half: direct-form log-joints of this
-        // row written over the tensor-core values (expanded constant 0, scale 1);
-        // a row stops summing once the component is 80 nats below the best
-        // non-sharp component of this half (its responsibility is then 0)
+        // Components of this column half with split dimensions: the tensor
+        // cores gave the log-joint over their other dimensions; add
+        // -1/2 sum (x - mu)^2/var over the split ones, in data units.  A row
+        // whose log-joint falls 80 nats below the best component of the half
+        // without split dimensions has responsibility 0 and gets -inf.
         const float floor_l = mx - 80.f;
         const int nsh = shl[0];
         const bool rvalid = row0 + row < a.N;
         const XT* xrow = reinterpret_cast<const XT*>(a.X) + (size_t)(rvalid ? row0 + row : 0) * D;
+        const uint32_t lo_off = (uint32_t)nch * kTcChunkBytes;
         for (int si = 0; si < nsh; si++) {
           const int j = shl[1 + si];
           if ((j >> 6) != hf) continue;
-          const float* mk = a.muh + (size_t)(k0 + j) * D;
-          const float* pk = a.ph + (size_t)(k0 + j) * D;
-          const float qmax = 2.f * (cds[j] - floor_l);  // q beyond this: below the floor
-          float q = 0.f;
-          for (int d = 0; d < D && q <= qmax; d += 4) {
-            float x4[4];
-            load4<XT>(xrow, (size_t)d, x4);
-            const float4 m4 = __ldg(reinterpret_cast<const float4*>(mk + d));
-            const float4 p4 = __ldg(reinterpret_cast<const float4*>(pk + d));
-            const float e0 = x4[0] - m4.x, e1 = x4[1] - m4.y;
-            const float e2 = x4[2] - m4.z, e3 = x4[3] - m4.w;
-            q = fmaf(e0 * e0, p4.x, q);
-            q = fmaf(e1 * e1, p4.y, q);
-            q = fmaf(e2 * e2, p4.z, q);
-            q = fmaf(e3 * e3, p4.w, q);
+          const size_t base = (size_t)(k0 + j) * D;
+          const int ns = __ldg(a.nsplit + k0 + j);
+          const float v0 = tmem_ld1(tL + lane_base + (uint32_t)j);
+          const float lr = fmaf(v0, wscs[j], csm[j]);  // log-joint over the kept dimensions
+          const float qmax = 2.f * (lr - floor_l);      // split sum beyond this: below the floor
+          // Filter: the row's own features x^ = F_hi + F_lo (shared memory).
+          // With a = x^ - mu^ and the feature's error |da_d| <= e_d =
+          // 2^-20 (|x^_d| + |mu^_d|) + 2^-24 (fp32 x^, the fp16 split, fp32
+          // mu^), the weighted norms obey |sqrt(q~) - sqrt(q)| <=
+          // sqrt(sum_d e_d^2 / var^_d); a row whose approximate split sum
+          // exceeds qmax by more than that bound is below the floor, and its
+          // exact sum is not needed.
+          bool far = !rvalid || !(qmax >= 0.f);
+          if (!far) {
+            const float sq_max = sqrtf(qmax);
+            float qa = 0.f, eb = 0.f;
+            for (int i0 = 0; i0 < ns && !far; i0 += 16) {
+              uchar4 pp[4];
+              float4 m4[4], p4[4];
+#pragma unroll
+              for (int g4 = 0; g4 < 4; g4++) {
+                const int i = min(i0 + 4 * g4, D - 4);  // in range; entries past ns are not summed
+                pp[g4] = __ldg(reinterpret_cast<const uchar4*>(a.perm + base + i));
+                m4[g4] = __ldg(reinterpret_cast<const float4*>(a.mhp + base + i));
+                p4[g4] = __ldg(reinterpret_cast<const float4*>(a.php + base + i));
+              }
+#pragma unroll
+              for (int g4 = 0; g4 < 4; g4++) {
+                const int fs[4] = {pp[g4].x, pp[g4].y, pp[g4].z, pp[g4].w};
+                const float ms[4] = {m4[g4].x, m4[g4].y, m4[g4].z, m4[g4].w};
+                const float ps[4] = {p4[g4].x, p4[g4].y, p4[g4].z, p4[g4].w};
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                  if (i0 + 4 * g4 + u >= ns) break;
+                  const int f = min(fs[u], D - 1);
+                  const uint32_t o = (uint32_t)(f >> 6) * kTcChunkBytes + sw128_offset(row, f & 63);
+                  const float xh = __half2float(*reinterpret_cast<const __half*>(sF + o)) +
+                                   __half2float(*reinterpret_cast<const __half*>(sF + lo_off + o));
+                  const float dd = xh - ms[u];
+                  qa = fmaf(dd * dd, ps[u], qa);
+                  const float ed = 9.6e-7f * (fabsf(xh) + fabsf(ms[u])) + 6.0e-8f;
+                  eb = fmaf(ed * ed, ps[u], eb);
+                  if (fabsf(xh) >= kTcXMax) eb = INFINITY;  // clamped feature: no bound
+                }
+              }
+              far = sqrtf(qa) * 0.99999f > sq_max + 1.01f * sqrtf(eb) + 1e-3f;
+            }
           }
-          tmem_st1(tL + lane_base + (uint32_t)j, q <= qmax ? cds[j] - 0.5f * q : -INFINITY);
+          // exact split sum in data units from X, 16 dimensions per step
+          float q = far ? INFINITY : 0.f;
+          for (int i0 = 0; i0 < ns && q <= qmax; i0 += 16) {
+            float x4[4][4];
+            float4 m4[4], p4[4];
+#pragma unroll
+            for (int g4 = 0; g4 < 4; g4++) {
+              const int i = min(i0 + 4 * g4, D - 4);
+              const uchar4 pp = __ldg(reinterpret_cast<const uchar4*>(a.perm + base + i));
+              x4[g4][0] = load1<XT>(xrow, min((int)pp.x, D - 1));
+              x4[g4][1] = load1<XT>(xrow, min((int)pp.y, D - 1));
+              x4[g4][2] = load1<XT>(xrow, min((int)pp.z, D - 1));
+              x4[g4][3] = load1<XT>(xrow, min((int)pp.w, D - 1));
+              m4[g4] = __ldg(reinterpret_cast<const float4*>(a.muh + base + i));
+              p4[g4] = __ldg(reinterpret_cast<const float4*>(a.ph + base + i));
+            }
+#pragma unroll
+            for (int g4 = 0; g4 < 4; g4++) {
+              const float ms[4] = {m4[g4].x, m4[g4].y, m4[g4].z, m4[g4].w};
+              const float ps[4] = {p4[g4].x, p4[g4].y, p4[g4].z, p4[g4].w};
+#pragma unroll
+              for (int u = 0; u < 4; u++) {
+                if (i0 + 4 * g4 + u >= ns) break;
+                const float e0 = x4[g4][u] - ms[u];
+                q = fmaf(e0 * e0, ps[u], q);
+              }
+            }
+          }
+          // the finished log-joint (the second load_logits takes it as is)
+          tmem_st1(tL + lane_base + (uint32_t)j, q <= qmax ? lr - 0.5f * q : -INFINITY);
         }
-        load_logits(false, 0u, 0u);
+        load_logits(true, sm0, sm1);
       }
       if (li + 1 < my_tiles) store_start();  // L is no longer read in this tile
       if (t == 0) SCEM_TRACE(li, 5);
@@ -770,6 +863,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           e[j] = __expf(e[j] - mx);
           se += e[j];
         }
+      } else {
+        // no finite log-joint in this half (dead or padding components, or a
+        // row past N): its responsibilities are exactly 0, not -inf * 0
+#pragma unroll
+        for (int j = 0; j < 64; j++) e[j] = 0.f;
       }
       // every (CTA, column half) contributes one (max, sum-exp) partial per row
       const uint32_t par = (uint32_t)(li & 1);
@@ -885,84 +983,149 @@ __global__ void tc_center_kernel(int D, int K, const float* __restrict__ w,
   sc_out[d] = ldexpf(1.0f, e);
 }
 
-// One block per (padded) component.  W = [mu^/var^, -1/(2 var^)] scaled by a
-// power of two 2^-g_k so its largest entry lies in [2^13, 2^14), split into
-// fp16 hi/lo rows of Fpad features (padding rows and features zero); the
-// constants of both forms; kappa_k and the direct-form tables mu^, 1/var^.
+// One block per (padded) component, one thread per dimension (D <= 128).
 //
-// The expanded-form constant c_k = log pi_k - (1/2) sum_d [log(2 pi var_kd) +
-// mu^_kd^2 / var^_kd] is corrected for the part of W that the fp16 hi/lo split
-// drops: the MMA sums F (W_hi + W_lo) 2^g, short of F W 2^g by F dW 2^g with
-// dW = W 2^-g - W_hi - W_lo, known exactly here.  For the points the component
-// explains F is near its expectation E[F] = [mu^, mu^^2 + var^], so
-// 2^g E[F] . dW is added to c_k: that removes the split's systematic error on
-// those points (what remains is (F - E[F]) . dW, of either sign from point to
-// point).  The accumulator starts from ci_k = kTcStartFrac sum_d mu^^2/var^
-// (fp32, in 2^g units); the fp32 remainder c_k - 2^g ci_k is added after the
-// MMAs.
+// Direct-form split.  The expanded form's fp32 error grows with
+// kappa_k = sum_d (mu^_kd^2 + 1)/var^_kd.  When kappa_k exceeds kTcSharpKappa (a
+// component collapsed onto a few points in some dimensions), or kTcSmallKappa
+// for a component expecting fewer than kTcSmallPoints points, its dimensions
+// are ranked by their share kappa_kd and the leading ones -- just enough that
+// the rest sum below the threshold -- are taken out of the contraction: their
+// W entries are zero, and the kernel adds -1/2 sum (x - mu)^2/var over them in
+// data units on the CUDA cores ("split" dimensions, nsplit_k of them, first in
+// perm).  The tensor cores keep the rest.
+//
+// W = [mu^/var^, -1/(2 var^)] over the remaining dimensions, scaled by a power
+// of two 2^-g_k so its largest entry lies in [2^13, 2^14), split into fp16
+// hi/lo rows of Fpad features (padding rows and features zero).
+//
+// The expanded-form constant c_k = log pi_k - (1/2) sum_d log(2 pi var_kd)
+// - (1/2) sum_{d kept} mu^_kd^2 / var^_kd is corrected for the part of W that
+// the fp16 hi/lo split drops: the MMA sums F (W_hi + W_lo) 2^g, short of F W 2^g
+// by F dW 2^g with dW = W 2^-g - W_hi - W_lo, known exactly here.  For the
+// points the component explains F is near its expectation E[F] = [mu^,
+// mu^^2 + var^], so 2^g E[F] . dW is added to c_k: that removes the split's
+// systematic error on those points (what remains is (F - E[F]) . dW, of either
+// sign from point to point).  The accumulator starts from ci_k = kTcStartFrac
+// sum_{d kept} mu^^2/var^ (fp32, in 2^g units); the fp32 remainder
+// c_k - 2^g ci_k is added after the MMAs.
+//
+// Tables for the split dimensions, in perm order: mu^ and 1/var^ (the filter on
+// the tile's features) and mu and 1/var in data units (the exact sum).
 __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     int64_t N, int D, int K, int Fpad, const float* __restrict__ w, const float* __restrict__ mu,
     const float* __restrict__ var, const float* __restrict__ m, const float* __restrict__ sc,
     __half* __restrict__ whi, __half* __restrict__ wlo, float* __restrict__ c_out,
-    float* __restrict__ cd_out, float* __restrict__ wsc_out, int* __restrict__ sharp_out,
+    float* __restrict__ wsc_out, int* __restrict__ sharp_out, int* __restrict__ nsplit_out,
     float* __restrict__ muh, float* __restrict__ ph, int* __restrict__ precise_out,
-    float* __restrict__ ci_out, unsigned int* status) {
+    float* __restrict__ ci_out, uint8_t* __restrict__ perm_out, float* __restrict__ mhp_out,
+    float* __restrict__ php_out, unsigned int* status) {
+  __shared__ double mh_s[kTcMaxD], vh_s[kTcMaxD], kd_s[kTcMaxD], ksort[kTcMaxD];
+  __shared__ int rank_s[kTcMaxD];
   __shared__ double wv[kTcChunk * kTcMaxChunks];  // Fpad <= 256
   __shared__ double ef[kTcChunk * kTcMaxChunks];  // E[F] under the component
   __shared__ double red[4][4];
+  __shared__ int ns_s;
   const int k = blockIdx.x;
-  double s_log = 0.0, s_q = 0.0, kap = 0.0, amax = 0.0, rho = 0.0;
+  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+  const float wk = k < K ? w[k] : 0.f;
+  const bool live = k < K && wk > 0.f;
+  auto block_sum = [&](double v) -> double {
+    v = warp_sum(v);
+    __syncthreads();
+    if (lane == 0) red[0][wp] = v;
+    __syncthreads();
+    return red[0][0] + red[0][1] + red[0][2] + red[0][3];
+  };
+  auto block_max = [&](double v) -> double {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    __syncthreads();
+    if (lane == 0) red[0][wp] = v;
+    __syncthreads();
+    return fmax(fmax(red[0][0], red[0][1]), fmax(red[0][2], red[0][3]));
+  };
+
+  // ---- pass 1: per dimension
+  double s_log = 0.0, kap = 0.0, rho = 0.0;
   bool bad = false;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    double mh = 0.0, vh = 1.0, kd = 0.0;
+    if (k < K) {
+      const double sd = (double)sc[d];
+      const double vr = (double)var[(size_t)k * D + d];
+      vh = vr / (sd * sd);
+      mh = ((double)mu[(size_t)k * D + d] - (double)m[d]) / sd;
+      kd = (mh * mh + 1.0) / vh;
+      s_log += log(2.0 * M_PI * vr);
+      kap += kd;
+      if (live) rho = fmax(rho, mh * mh / vh);
+      if (!isfinite(mu[(size_t)k * D + d]) || !(vr > 0.0) || !isfinite(vr)) bad = true;
+    }
+    mh_s[d] = mh;
+    vh_s[d] = vh;
+    kd_s[d] = kd >= 0.0 ? fmin(kd, 1e300) : 0.0;  // NaN -> 0: the ranks stay a permutation
+  }
+  const double S_log = block_sum(s_log);
+  const double Kap = block_sum(kap);
+  const double Rho = block_max(rho);
+  const bool small = (double)wk * (double)N < kTcSmallPoints;
+  const double thr = small ? kTcSmallKappa : kTcSharpKappa;
+  const bool sharp = live && Kap > thr;
+
+  // ---- dimensions by decreasing kappa_kd (ties to the lower index)
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    const double key = kd_s[d];
+    int r = 0;
+    for (int e2 = 0; e2 < D; e2++) {
+      const double o = kd_s[e2];
+      r += (o > key || (o == key && e2 < d)) ? 1 : 0;
+    }
+    rank_s[d] = r;
+    ksort[r] = key;
+    const size_t o = (size_t)k * D + r;
+    perm_out[o] = (uint8_t)d;
+    mhp_out[o] = (float)mh_s[d];
+    php_out[o] = (float)(1.0 / vh_s[d]);
+    muh[o] = k < K ? mu[(size_t)k * D + d] : 0.f;
+    ph[o] = k < K ? (float)(1.0 / (double)var[(size_t)k * D + d]) : 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ns = 0;
+    if (sharp) {
+      double rem = Kap;
+      while (ns < D && rem > thr) rem -= ksort[ns++];
+    }
+    ns_s = ns;
+  }
+  __syncthreads();
+  const int ns = ns_s;
+
+  // ---- pass 2: the contraction's features, without the split dimensions
+  double s_q = 0.0, amax = 0.0;
   for (int f = threadIdx.x; f < Fpad; f += blockDim.x) {
     double v = 0.0, e = 0.0;
     if (k < K && f < 2 * D) {
       const int d = f < D ? f : f - D;
-      const double sd = (double)sc[d];
-      const double vr = (double)var[(size_t)k * D + d];
-      const double vh = vr / (sd * sd);
-      const double mh = ((double)mu[(size_t)k * D + d] - (double)m[d]) / sd;
-      if (f < D) {
-        v = mh / vh;
-        e = mh;
-        s_log += log(2.0 * M_PI * vr);
-        s_q += mh * mh / vh;
-        kap += (mh * mh + 1.0) / vh;
-        if (k < K && w[k] > 0.f) rho = fmax(rho, mh * mh / vh);
-        muh[(size_t)k * D + d] = mu[(size_t)k * D + d];
-        ph[(size_t)k * D + d] = (float)(1.0 / vr);
-        if (!isfinite(mu[(size_t)k * D + d]) || !(vr > 0.0) || !isfinite(vr)) bad = true;
-      } else {
-        v = -0.5 / vh;
-        e = mh * mh + vh;
+      if (rank_s[d] >= ns) {
+        const double mh = mh_s[d], vh = vh_s[d];
+        if (f < D) {
+          v = mh / vh;
+          e = mh;
+          s_q += mh * mh / vh;
+        } else {
+          v = -0.5 / vh;
+          e = mh * mh + vh;
+        }
       }
     }
     wv[f] = v;
     ef[f] = e;
     amax = fmax(amax, fabs(v));
   }
-  const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-  double t0 = warp_sum(s_log), t1 = warp_sum(s_q), t2 = warp_sum(kap);
-  double t3 = amax;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) t3 = fmax(t3, __shfl_xor_sync(0xffffffffu, t3, o));
-  if (lane == 0) {
-    red[0][wp] = t0;
-    red[1][wp] = t1;
-    red[2][wp] = t2;
-    red[3][wp] = t3;
-  }
-  __syncthreads();
-  const double S_log = red[0][0] + red[0][1] + red[0][2] + red[0][3];
-  const double S_q = red[1][0] + red[1][1] + red[1][2] + red[1][3];
-  const double Kap = red[2][0] + red[2][1] + red[2][2] + red[2][3];
-  const double Amax = fmax(fmax(red[3][0], red[3][1]), fmax(red[3][2], red[3][3]));
-  __syncthreads();
-  double t4 = rho;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) t4 = fmax(t4, __shfl_xor_sync(0xffffffffu, t4, o));
-  if (lane == 0) red[0][wp] = t4;
-  __syncthreads();
-  const double Rho = fmax(fmax(red[0][0], red[0][1]), fmax(red[0][2], red[0][3]));
+  const double S_q = block_sum(s_q);
+  const double Amax = block_max(amax);
   int ex = 0;
   if (Amax > 0.0 && isfinite(Amax)) frexp(Amax, &ex);
   const int g = Amax > 0.0 ? ex - 14 : 0;
@@ -976,25 +1139,17 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     wlo[(size_t)k * Fpad + f] = l;
     dsplit += ef[f] * (svd - (double)__half2float(h) - (double)__half2float(l));
   }
-  dsplit = warp_sum(dsplit);
-  __syncthreads();  // every thread is done reading red[0][*] (Rho)
-  if (lane == 0) red[1][wp] = dsplit;
-  __syncthreads();
-  const double Dsplit = red[1][0] + red[1][1] + red[1][2] + red[1][3];
+  const double Dsplit = block_sum(dsplit);
   if (threadIdx.x == 0) {
-    const float wk = k < K ? w[k] : 0.f;
     if (k < K && (!isfinite(wk) || !(wk >= 0.f))) bad = true;
-    const bool live = k < K && wk > 0.f;
-    const bool small = (double)wk * (double)N < kTcSmallPoints;
-    const bool sharp = live && (Kap > kTcSharpKappa || (small && Kap > kTcSmallKappa));
     const double lw = live ? log((double)wk) : 0.0;
-    cd_out[k] = live ? (float)(lw - 0.5 * S_log) : -INFINITY;
     const double cfull = lw - 0.5 * (S_log + S_q) + ldexp(Dsplit, g);
-    const float cstart = (live && !sharp) ? (float)ldexp(kTcStartFrac * S_q, -g) : 0.f;
+    const float cstart = live ? (float)ldexp(kTcStartFrac * S_q, -g) : 0.f;
     ci_out[k] = cstart;
-    c_out[k] = !live ? -INFINITY : (sharp ? 0.f : (float)(cfull - ldexp((double)cstart, g)));
-    wsc_out[k] = sharp ? 1.f : ldexpf(1.0f, g);
-    sharp_out[k] = sharp ? 1 : 0;
+    c_out[k] = live ? (float)(cfull - ldexp((double)cstart, g)) : -INFINITY;
+    wsc_out[k] = ldexpf(1.0f, g);
+    sharp_out[k] = ns > 0 ? 1 : 0;
+    nsplit_out[k] = ns;
     precise_out[k] = live && (Rho > kTcRhoPrecise || small) ? 1 : 0;
   }
   if (bad) atomicOr(status, GMM_DEVFLAG_BAD_PARAMS);
