@@ -176,7 +176,7 @@ gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const 
       (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.wsc), (int*)(ws + T.sharp),
       (int*)(ws + T.nsplit), (float*)(ws + T.muh), (float*)(ws + T.ph), (int*)(ws + T.precise),
       (float*)(ws + T.ci), (uint8_t*)(ws + T.perm), (float*)(ws + T.mhp), (float*)(ws + T.php),
-      (unsigned int*)ws);
+      (uint32_t*)(ws + T.pmask), (unsigned int*)ws);
   return launched(2);
 }
 
@@ -250,6 +250,7 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, char* ws, const TcLayo
   args.status = (unsigned int*)ws;
   args.drain_tiles = tc_drain_tiles();
   args.precise = (const int*)(ws + T.precise);
+  args.pmask = (const uint32_t*)(ws + T.pmask);
   args.wait_ns = kWaitBudgetNs;
   trace_begin(st);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args, mhi, mlo);

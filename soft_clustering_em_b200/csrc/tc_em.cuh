@@ -38,15 +38,17 @@
 // as r_hi^T (F_hi + F_lo) + r_lo^T F_hi and r^T 1 on the tensor cores,
 // accumulated in fp32 in tensor memory over a few tiles and then added into
 // fp64 per-cluster slots.  The variance S2/N - (S1/N)^2 magnifies the
-// relative rounding error of those fp32 sums by rho_k = max_d mu^^2 / var^, and
-// a weight is sensitive to it when the component holds few points; so a
-// "precise" component (rho_k > 64, or pi_k N < 20) is drained after every
-// tile in which it has mass, every other component every kTcDrainTiles tiles.
-// Each compute thread drains its own component (tensor-memory lane) and
-// zeroes its accumulators in place with tcgen05.st.  The M-step undoes the
-// scales exactly.  r^ passes
-// through one 32 KB buffer in two 64-row halves: rows 0-63 first, then rows
-// 64-127 once the MMAs of the first half have released it.
+// relative rounding error of dimension d's fp32 sums by mu^_kd^2 / var^_kd, and
+// a weight is sensitive to it when the component holds few points; so the
+// "precise" features (both of a dimension with mu^^2/var^ > 64, every feature
+// of a component expecting fewer than 50 points) and N_k are drained after
+// every tile in which the component has mass, everything every kTcDrainTiles
+// tiles.  Each compute thread drains its own component (tensor-memory lane)
+// with fire-and-forget fp64 reductions and zeroes what it drained in place
+// with tcgen05.st, while the next tile's E-step MMAs run.  The M-step undoes
+// the scales exactly.  r^ passes through one 32 KB buffer in two 64-row
+// halves: rows 0-63 first, then rows 64-127 once the MMAs of the first half
+// have released it.
 //
 // Work split.  A cluster of C = ceil(K/128) CTAs takes one 128-row tile at a
 // time; CTA `rank` owns components [128 rank, 128 rank + 128).  Per tile each
@@ -168,6 +170,8 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //   wsc  : C*128 f32 power-of-two scale of each W row (1 if sharp)
 //   sharp: C*128 int32 1 if some of the component's dimensions are summed in
 //          direct form (nsplit: C*128 int32, how many: the first nsplit of perm)
+//   pmask: [C*128 x Fpad/32] u32 per feature of each component, 1 if it is
+//          drained after every tile with mass (see tc_prep_w_kernel)
 //   perm : [C*128 x D] u8 dimensions of each component by decreasing
 //          (mu^^2 + 1)/var^
 //   muh, ph : [C*128 x D] f32 mu and 1/var (data units) in perm order
@@ -177,8 +181,8 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //          [(2D+1) x K] feature-major statistics (S1 rows 0..D-1, S2 rows
 //          D..2D-1, N_k row 2D) followed by the cluster's LL.
 struct TcLayout {
-  size_t m, isc, sc, c, ci, wsc, sharp, nsplit, precise, muh, ph, perm, mhp, php, whi, wlo, slots,
-      total, slot_stride;
+  size_t m, isc, sc, c, ci, wsc, sharp, nsplit, precise, pmask, muh, ph, perm, mhp, php, whi, wlo,
+      slots, total, slot_stride;
   int C, nchunks, Kpad, Fpad, P;
 };
 
@@ -227,6 +231,8 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   off = align_up(off + (size_t)L.Kpad * L.Fpad * 2, 256);
   L.precise = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
+  L.pmask = off;
+  off = align_up(off + (size_t)L.Kpad * (L.Fpad / 32) * 4, 256);
   L.slot_stride = align_up((size_t)(2 * D + 1) * K + 1, 32);
   L.slots = off;
   L.P = num_sms / L.C;
@@ -260,7 +266,8 @@ struct TcArgs {
   size_t slot_stride;   // doubles per slot: (2D+1)*K statistics + LL
   unsigned int* status;
   int drain_tiles;
-  const int* precise;   // 1: drain the component after every tile with mass, C*128
+  const int* precise;   // 1: some feature of the component is drained every tile, C*128
+  const uint32_t* pmask;  // which features, C*128 x (Fpad/32) words
   uint64_t wait_ns;
 };
 
@@ -573,16 +580,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       return r;
     };
 
-    // Drain component lane `row` into the fp64 slot and zero its accumulators,
-    // when it has mass since the last drain and `force` or it is precise.
-    // Column half 0 also owns the N_k column; the other half waits until N_k
-    // has been read by everyone before it is zeroed.
-    auto drain = [&](bool force) -> bool {
+    // Drain component lane `row` into the fp64 slot and zero what was drained.
+    // `force`: every accumulator of every component (features not drained
+    // since the last forced drain may hold mass even when N_k, drained more
+    // often, does not).  Otherwise, for a component with mass in this tile,
+    // its precise features only (pmask) and its N_k: those whose fp32 sums
+    // would lose too much over several tiles.  Column half 0 also owns the N_k
+    // column.
+    auto drain = [&](bool force, int64_t li) -> bool {
       const int k = k0 + row;
       float vn[32];
       tmem_ld32(tNK + lane_base, vn);
-      const bool due = k < K && vn[0] != 0.f && (force || precs[row] != 0);
+      const bool due = k < K && (force || (precs[row] != 0 && vn[0] != 0.f));
       if (!rendezvous()) return false;
+      if (t == 0) SCEM_TRACE(li, 14);
       if (!__any_sync(0xffffffffu, due)) return true;
       // Fire-and-forget fp64 reductions into the slot: one thread owns each
       // address, so the additions land in program order (deterministic) and
@@ -596,18 +607,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tmem_st32(tNK + lane_base, vn);
       }
+      if (t == 0) SCEM_TRACE(li, 15);
+      const uint32_t* pm = a.pmask + (size_t)(due ? k : 0) * (2 * nch);
+      uint32_t mw[kTcMaxChunks];
+#pragma unroll
+      for (int c = 0; c < kTcMaxChunks; c++)
+        mw[c] = (!due || c >= nch) ? 0u : (force ? 0xffffffffu : __ldg(pm + 2 * c + hf));
       for (int c = 0; c < nch; c++) {
+        uint32_t mask = mw[0];
+#pragma unroll
+        for (int c2 = 1; c2 < kTcMaxChunks; c2++)
+          if (c == c2) mask = mw[c2];
+        if (!__any_sync(0xffffffffu, mask != 0u)) continue;  // nothing of this block is due
         float v[32];
         const uint32_t cc = tS + lane_base + 64u * c + 32u * hf;
         tmem_ld32(cc, v);
-        if (due) {
+        if (mask) {
           const int f0 = 64 * c + 32 * hf;
           const int nf = min(32, 2 * D - f0);  // features of this column block that exist
 #pragma unroll
           for (int j = 0; j < 32; j++)
-            if (j < nf && v[j] != 0.f) atomicAdd(sk + (size_t)(f0 + j) * K, (double)v[j]);
-#pragma unroll
-          for (int j = 0; j < 32; j++) v[j] = 0.f;
+            if ((mask >> j) & 1u) {
+              if (j < nf && v[j] != 0.f) atomicAdd(sk + (size_t)(f0 + j) * K, (double)v[j]);
+              v[j] = 0.f;
+            }
         }
         tmem_st32(cc, v);
       }
@@ -646,13 +669,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!ok) break;
         if (t == 0) SCEM_TRACE(li, 1);
         tc_fence_after_sync();
-        if (MODE == kTcStats) {
-          ok = drain((li % a.drain_tiles) == 0);
-          if (t == 0) SCEM_TRACE(li, 2);
-          if (!ok) break;
-          tc_fence_before_sync();
-          mbar_arrive(drained);
-        }
       }
       // ---- X tile -> F = [x^, x^^2] as fp16 hi/lo in the swizzled layout.
       // The next tile's rows (contiguous in X) are pulled into L2 now, so that
@@ -718,7 +734,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           *reinterpret_cast<uint2*>(sF + o2) = make_uint2(hs[0], hs[1]);
           *reinterpret_cast<uint2*>(sF + lo_off + o2) = make_uint2(ls[0], ls[1]);
         }
-        if (t == 0) SCEM_TRACE(li, 13 + min(nbatch, 2));
+        if (t == 0) SCEM_TRACE(li, 13);
         nbatch++;
       }
       if (bad) atomicOr(a.status, GMM_DEVFLAG_NONFINITE_X);
@@ -728,6 +744,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before_sync();
       mbar_arrive(f_full);
       if (t == 0) SCEM_TRACE(li, 3);
+      // Drain the previous tiles' statistics while the E-step MMAs run (they
+      // write other tensor-memory columns); this tile's statistics MMAs wait
+      // for it.
+      if (MODE == kTcStats && li > 0) {
+        ok = drain((li % a.drain_tiles) == 0, li);
+        if (t == 0) SCEM_TRACE(li, 2);
+        if (!ok) break;
+        tc_fence_before_sync();
+        mbar_arrive(drained);
+      }
 
       // ---- epilogue: logits -> row max / sum-exp -> cluster exchange -> r^
       ok = __all_sync(0xffffffffu,
@@ -770,6 +796,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool rvalid = row0 + row < a.N;
         const XT* xrow = reinterpret_cast<const XT*>(a.X) + (size_t)(rvalid ? row0 + row : 0) * D;
         const uint32_t lo_off = (uint32_t)nch * kTcChunkBytes;
+        // the filter tables of every split component head for L1 now (one lane
+        // per component), so the per-component loop below meets L1, not L2
+        for (int sj = lane; sj < nsh; sj += 32) {
+          const size_t base = (size_t)(k0 + shl[1 + sj]) * D;
+          prefetch_l1(a.perm + base);
+          prefetch_l1(a.mhp + base);
+          prefetch_l1(a.php + base);
+        }
         for (int si = 0; si < nsh; si++) {
           const int j = shl[1 + si];
           if ((j >> 6) != hf) continue;
@@ -923,7 +957,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(s_done, (uint32_t)((my_tiles - 1) & 1),
                                                      status, kAbort, a.wait_ns));
       tc_fence_after_sync();
-      if (ok && MODE == kTcStats) ok = drain(true);
+      if (ok && MODE == kTcStats) ok = drain(true, my_tiles);
     }
     // LL of this CTA's rows (rank 0 of each cluster, column half 0): fixed-order sum
     ll = warp_sum(ll);
@@ -1019,7 +1053,7 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     float* __restrict__ wsc_out, int* __restrict__ sharp_out, int* __restrict__ nsplit_out,
     float* __restrict__ muh, float* __restrict__ ph, int* __restrict__ precise_out,
     float* __restrict__ ci_out, uint8_t* __restrict__ perm_out, float* __restrict__ mhp_out,
-    float* __restrict__ php_out, unsigned int* status) {
+    float* __restrict__ php_out, uint32_t* __restrict__ pmask_out, unsigned int* status) {
   __shared__ double mh_s[kTcMaxD], vh_s[kTcMaxD], kd_s[kTcMaxD], ksort[kTcMaxD];
   __shared__ int rank_s[kTcMaxD];
   __shared__ double wv[kTcChunk * kTcMaxChunks];  // Fpad <= 256
@@ -1126,6 +1160,18 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
   }
   const double S_q = block_sum(s_q);
   const double Amax = block_max(amax);
+  // Precise features: both features of a dimension with mu^^2/var^ > kTcRhoPrecise
+  // (the variance S2/N - (S1/N)^2 magnifies their fp32 rounding by that ratio),
+  // every feature of a component expecting fewer than kTcSmallPoints points.
+  for (int f = threadIdx.x; f < Fpad; f += blockDim.x) {  // warp w: features 32w.. of each 128
+    bool pf = false;
+    if (live && f < 2 * D) {
+      const int d = f < D ? f : f - D;
+      pf = small || mh_s[d] * mh_s[d] / vh_s[d] > kTcRhoPrecise;
+    }
+    const uint32_t word = __ballot_sync(0xffffffffu, pf);
+    if (lane == 0) pmask_out[(size_t)k * (Fpad / 32) + f / 32] = word;
+  }
   int ex = 0;
   if (Amax > 0.0 && isfinite(Amax)) frexp(Amax, &ex);
   const int g = Amax > 0.0 ? ex - 14 : 0;
@@ -1150,7 +1196,7 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     wsc_out[k] = ldexpf(1.0f, g);
     sharp_out[k] = ns > 0 ? 1 : 0;
     nsplit_out[k] = ns;
-    precise_out[k] = live && (Rho > kTcRhoPrecise || small) ? 1 : 0;
+    precise_out[k] = live && (Rho > kTcRhoPrecise || small) ? 1 : 0;  // some pmask bit set
   }
   if (bad) atomicOr(status, GMM_DEVFLAG_BAD_PARAMS);
 }
