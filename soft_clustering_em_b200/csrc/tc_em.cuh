@@ -346,7 +346,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* csm = reinterpret_cast<float*>(sm + L.csm);
   float* cis = reinterpret_cast<float*>(sm + L.cis);
   float* wscs = reinterpret_cast<float*>(sm + L.wscs);
-  int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = local indices
+  int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = j | nsplit << 8
   int* precs = reinterpret_cast<int*>(sm + L.precs);
   float2* xchg = reinterpret_cast<float2*>(sm + L.xchg);  // [2][C][2][128] (max, sum-exp)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
@@ -413,7 +413,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t mw[4] = {0u, 0u, 0u, 0u};
     for (int j = 0; j < kTcComps; j++)
       if (a.sharp[k0 + j]) {
-        shl[1 + n++] = j;
+        shl[1 + n++] = j | (a.nsplit[k0 + j] << 8);  // local index | split count
         mw[j >> 5] |= 1u << (j & 31);
       }
     shl[0] = n;
@@ -799,16 +799,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // the filter tables of every split component head for L1 now (one lane
         // per component), so the per-component loop below meets L1, not L2
         for (int sj = lane; sj < nsh; sj += 32) {
-          const size_t base = (size_t)(k0 + shl[1 + sj]) * D;
+          const size_t base = (size_t)(k0 + (shl[1 + sj] & 255)) * D;
           prefetch_l1(a.perm + base);
           prefetch_l1(a.mhp + base);
           prefetch_l1(a.php + base);
         }
         for (int si = 0; si < nsh; si++) {
-          const int j = shl[1 + si];
+          const int j = shl[1 + si] & 255, ns = shl[1 + si] >> 8;
           if ((j >> 6) != hf) continue;
           const size_t base = (size_t)(k0 + j) * D;
-          const int ns = __ldg(a.nsplit + k0 + j);
           const float v0 = tmem_ld1(tL + lane_base + (uint32_t)j);
           const float lr = fmaf(v0, wscs[j], csm[j]);  // log-joint over the kept dimensions
           const float qmax = 2.f * (lr - floor_l);      // split sum beyond this: below the floor
