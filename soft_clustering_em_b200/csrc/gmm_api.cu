@@ -176,7 +176,7 @@ gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const 
       (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.wsc), (int*)(ws + T.sharp),
       (int*)(ws + T.nsplit), (float*)(ws + T.muh), (float*)(ws + T.ph), (int*)(ws + T.precise),
       (float*)(ws + T.ci), (uint8_t*)(ws + T.perm), (float*)(ws + T.mhp), (float*)(ws + T.php),
-      (uint32_t*)(ws + T.pmask), (unsigned int*)ws);
+      (uint32_t*)(ws + T.pmask), (uint8_t*)(ws + T.rank), (unsigned int*)ws);
   return launched(2);
 }
 
@@ -284,10 +284,10 @@ gmm_status estep_stats_impl(const gmm_problem* p, const void* X, const float* w,
     if ((s = tc_prep(p, w, mu, var, ws, T, st)) != GMM_OK) return s;
     int nslots = 0;
     if ((s = tc_pass<kTcStats>(p, X, ws, T, st, &nslots)) != GMM_OK) return s;
-    tc_reduce_stats_kernel<<<blocks, 256, 0, st>>>(p->D, p->K, (const float*)(ws + T.m),
-                                                   (const float*)(ws + T.sc), mu,
-                                                   (const double*)(ws + T.slots), T.slot_stride,
-                                                   nslots, stats);
+    tc_reduce_stats_kernel<<<blocks, 256, 0, st>>>(
+        p->D, p->K, (const float*)(ws + T.m), (const float*)(ws + T.sc), mu,
+        (const uint8_t*)(ws + T.rank), (const int*)(ws + T.nsplit),
+        (const double*)(ws + T.slots), T.slot_stride, nslots, stats);
     return launched(1);
   }
   const WsPtrs wp = ws_ptrs(ws_base, P.simt);

@@ -177,12 +177,15 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //   muh, ph : [C*128 x D] f32 mu and 1/var (data units) in perm order
 //   mhp, php : [C*128 x D] f32 mu^ and 1/var^ in perm order
 //   whi, wlo : [C*128 x 64*nchunks] fp16 operand W (hi and lo parts)
+//   rank : [C*128 x D] u8 position of each dimension in perm
 //   slots: P per-cluster slots of slot_stride doubles:
 //          [(2D+1) x K] feature-major statistics (S1 rows 0..D-1, S2 rows
-//          D..2D-1, N_k row 2D) followed by the cluster's LL.
+//          D..2D-1, N_k row 2D), the cluster's LL, then [2D x K] direct-form
+//          moments of split dimensions about the input means, by perm position
+//          i: sum r (x - mu) in row i, sum r (x - mu)^2 in row D + i.
 struct TcLayout {
-  size_t m, isc, sc, c, ci, wsc, sharp, nsplit, precise, pmask, muh, ph, perm, mhp, php, whi, wlo,
-      slots, total, slot_stride;
+  size_t m, isc, sc, c, ci, wsc, sharp, nsplit, precise, pmask, muh, ph, perm, rank, mhp, php, whi,
+      wlo, slots, total, slot_stride;
   int C, nchunks, Kpad, Fpad, P;
 };
 
@@ -221,6 +224,8 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   off = align_up(off + (size_t)L.Kpad * D * 4, 256);
   L.perm = off;
   off = align_up(off + (size_t)L.Kpad * D, 256);
+  L.rank = off;
+  off = align_up(off + (size_t)L.Kpad * D, 256);
   L.mhp = off;
   off = align_up(off + (size_t)L.Kpad * D * 4, 256);
   L.php = off;
@@ -233,7 +238,7 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.pmask = off;
   off = align_up(off + (size_t)L.Kpad * (L.Fpad / 32) * 4, 256);
-  L.slot_stride = align_up((size_t)(2 * D + 1) * K + 1, 32);
+  L.slot_stride = align_up((size_t)(4 * D + 1) * K + 1, 32);
   L.slots = off;
   L.P = num_sms / L.C;
   if (cap) {
@@ -428,6 +433,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int f = 0; f <= 2 * D; f++)
       for (int kk = tid; kk < kTcComps; kk += kTcThreads)
         if (k0 + kk < K) slot[(size_t)f * K + k0 + kk] = 0.0;
+    // the direct-form moments of split dimensions (the rows the reduction reads)
+    double* dir = slot + ll_index + 1;
+    for (int kk = tid; kk < kTcComps; kk += kTcThreads)
+      if (k0 + kk < K) {
+        const int ns = a.nsplit[k0 + kk];
+        for (int i = 0; i < ns; i++) {
+          dir[(size_t)i * K + k0 + kk] = 0.0;
+          dir[(size_t)(D + i) * K + k0 + kk] = 0.0;
+        }
+      }
   }
   fence_proxy_async_smem();
   tc_fence_before_sync();
@@ -887,7 +902,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         load_logits(true, sm0, sm1);
       }
-      if (li + 1 < my_tiles) store_start();  // L is no longer read in this tile
       if (t == 0) SCEM_TRACE(li, 5);
       float se = 0.f;
       if (mx > -INFINITY) {
@@ -951,6 +965,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before_sync();
       mbar_arrive(hr == 0 ? r_full : r_full1);
       if (t == 0) SCEM_TRACE(li, 7);
+      // Moments of split dimensions in direct form, about the input means, in
+      // data units from X (no cancellation however narrow the dimension),
+      // while the statistics MMAs run.  Only rows with a finite log-joint for
+      // the component contribute: the few near it.  (X, not F: F may already
+      // hold the next tile once the statistics MMAs are done.)
+      if (MODE == kTcStats && (sm0 | sm1)) {
+        const int nsh = shl[0];
+        const XT* xrow = reinterpret_cast<const XT*>(a.X) + (size_t)(valid ? row0 + row : 0) * D;
+        double* dir = slot + ll_index + 1;  // [2D x K] after the LL
+        for (int si = 0; si < nsh; si++) {
+          const int j = shl[1 + si] & 255, ns = shl[1 + si] >> 8;
+          if ((j >> 6) != hf) continue;
+          const float l = tmem_ld1(tL + lane_base + (uint32_t)j);  // the finished log-joint
+          const double r = (valid && l > -INFINITY) ? (double)__expf(l - lse) : 0.0;
+          if (r > 0.0) {
+            const size_t base = (size_t)(k0 + j) * D;
+            for (int i = 0; i < ns; i++) {
+              const int d = min((int)a.perm[base + i], D - 1);
+              const double dx = (double)load1<XT>(xrow, d) - (double)a.muh[base + i];
+              atomicAdd(dir + (size_t)i * K + (k0 + j), r * dx);
+              atomicAdd(dir + (size_t)(D + i) * K + (k0 + j), r * dx * dx);
+            }
+          }
+        }
+      }
+      if (li + 1 < my_tiles) store_start();  // L is no longer read in this tile
     }
     if (ok && my_tiles > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(s_done, (uint32_t)((my_tiles - 1) & 1),
@@ -1052,7 +1092,8 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     float* __restrict__ wsc_out, int* __restrict__ sharp_out, int* __restrict__ nsplit_out,
     float* __restrict__ muh, float* __restrict__ ph, int* __restrict__ precise_out,
     float* __restrict__ ci_out, uint8_t* __restrict__ perm_out, float* __restrict__ mhp_out,
-    float* __restrict__ php_out, uint32_t* __restrict__ pmask_out, unsigned int* status) {
+    float* __restrict__ php_out, uint32_t* __restrict__ pmask_out, uint8_t* __restrict__ rank_out,
+    unsigned int* status) {
   __shared__ double mh_s[kTcMaxD], vh_s[kTcMaxD], kd_s[kTcMaxD], ksort[kTcMaxD];
   __shared__ int rank_s[kTcMaxD];
   __shared__ double wv[kTcChunk * kTcMaxChunks];  // Fpad <= 256
@@ -1116,6 +1157,7 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     }
     rank_s[d] = r;
     ksort[r] = key;
+    rank_out[(size_t)k * D + d] = (uint8_t)r;
     const size_t o = (size_t)k * D + r;
     perm_out[o] = (uint8_t)d;
     mhp_out[o] = (float)mh_s[d];
@@ -1204,10 +1246,13 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
 // statistics buffer [ N_k | A | B | LL ] (component-major, moments about the
 // input means mu, data units).  The slots hold N' = 2^15 N_k and
 // S1' = 2^15 sum r x^, S2' = 2^15 sum r x^^2 with x^ = (x - m)/s, so with
-// dm = mu - m:  A = s S1 - dm N,  B = s^2 S2 - 2 s dm S1 + dm^2 N.
+// dm = mu - m:  A = s S1 - dm N,  B = s^2 S2 - 2 s dm S1 + dm^2 N.  A split
+// dimension (perm position below nsplit_k) takes A and B from the direct-form
+// moments instead.
 __global__ void __launch_bounds__(256) tc_reduce_stats_kernel(
     int D, int K, const float* __restrict__ m, const float* __restrict__ sc,
-    const float* __restrict__ mu, const double* __restrict__ slots, size_t slot_stride,
+    const float* __restrict__ mu, const uint8_t* __restrict__ rank,
+    const int* __restrict__ nsplit, const double* __restrict__ slots, size_t slot_stride,
     int nslots, double* __restrict__ stats) {
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t KD = (size_t)K * D;
@@ -1230,6 +1275,19 @@ __global__ void __launch_bounds__(256) tc_reduce_stats_kernel(
   const double sd = (double)sc[d];
   const double dm = (double)mu[(size_t)k * D + d] - (double)m[d];
   if (d == 0) stats[k] = n;
+  const int r = rank[(size_t)k * D + d];
+  if (r < nsplit[k]) {
+    const size_t dir = (size_t)(2 * D + 1) * K + 1;
+    double A = 0.0, B = 0.0;
+    for (int p = 0; p < nslots; p++) {
+      const double* s = slots + (size_t)p * slot_stride + dir;
+      A += s[(size_t)r * K + k];
+      B += s[(size_t)(D + r) * K + k];
+    }
+    stats[K + (size_t)k * D + d] = A;
+    stats[K + KD + (size_t)k * D + d] = B;
+    return;
+  }
   stats[K + (size_t)k * D + d] = sd * S1 - dm * n;
   stats[K + KD + (size_t)k * D + d] = sd * sd * S2 - 2.0 * sd * dm * S1 + dm * dm * n;
 }

@@ -370,3 +370,56 @@ def test_row_shards_sum_to_the_full_step(G, name, N, K, shards):
     rep = compare.compare_step((*params_np(*full), ll_full.item()), (*params_np(*sh), ll_sh.item()),
                                nk)
     assert rep["ok"], rep
+
+
+def _kappa(w, mu, var):
+    """kappa_k = sum_d (mu^^2 + 1)/var^ in the whitened units of the tensor-core path
+    (centring at the mixture mean, s = 2^(round(log2 std) + 1)); recomputed here only
+    to show that a case reaches the split thresholds."""
+    w, mu, var = (np.asarray(a, dtype=np.float64) for a in (w, mu, var))
+    m = (w[:, None] * mu).sum(0) / w.sum()
+    v = (w[:, None] * (var + mu ** 2)).sum(0) / w.sum() - m ** 2
+    s = 2.0 ** (np.rint(0.5 * np.log2(v)) + 1)
+    return ((((mu - m) / s) ** 2 + 1) / (var / s ** 2)).sum(1)
+
+
+def test_split_dimensions_match_oracle(G):
+    """A component collapsed onto rows that share exact values in some dimensions
+    (variance at the floor there: kappa far above 1e7), and a tight component
+    expecting 20 points (kappa between 2e4 and 1e7): both have dimensions summed in
+    direct form on the CUDA cores next to the tensor-core contraction of the rest,
+    and the split dimensions' moments summed in direct form too.  (The tight
+    component sits 0.1 from the centring point in x^ units: far from it, mu^^2/var^ of
+    its kept dimensions would bound its variance's precision at about that ratio times
+    2^-22; right at it, x^^2 of its points would fall below fp16's normal range -- the
+    tensor-core statistics' two limits.)"""
+    rng = np.random.default_rng(11)
+    N, D, K = 6_001, 16, 12
+    centers = rng.uniform(-20, 20, size=(K, D))
+    z = rng.integers(2, K, size=N)
+    X = (centers[z] + rng.normal(size=(N, D))).astype(np.float32)
+    X[:40, :4] = 7.0  # 40 rows identical in dimensions 0-3
+    X[:40, 4:] = (centers[0, 4:] + rng.normal(size=(40, D - 4))).astype(np.float32)
+    # 3.2 from the mixture mean (0.1 in x^ units), spread 0.2: mu^^2/var^ stays ~200,
+    # and x^^2 of its points stays in fp16's normal range
+    centers[1] = centers[2:].mean(0) + 3.2
+    X[40:60] = (centers[1] + 0.2 * rng.normal(size=(20, D))).astype(np.float32)
+    w = np.full(K, 1.0 / K)
+    w[0], w[1] = 40.0 / N, 20.0 / N
+    w = w / w.sum()
+    mu = centers.copy()
+    mu[0, :4] = 7.0
+    mu[0, 4:] = X[:40, 4:].mean(0)
+    mu[1] = X[40:60].mean(0)
+    var = np.ones((K, D))
+    var[0, :4] = 1e-6
+    var[1] = 0.05
+    kap = _kappa(np.float32(w), np.float32(mu), np.float32(var))
+    # component 0 by kappa alone, component 1 only because it expects few points
+    assert kap[0] > 1e7 and w[1] * N < 50 and 2e4 < kap[1] < 1e7, kap[:2]
+    ref, got = _tiny(G, X, w, mu, var)
+    rep = compare.compare_step(ref[:4], got, ref[4])
+    assert rep["ok"], rep
+    # the collapsed component keeps its 40 points and its zero spread in dimensions 0-3
+    assert abs(got[0][0] * N - 40.0) < 0.05
+    np.testing.assert_allclose(got[2][0][:4], 1e-6, rtol=1e-6)
