@@ -82,10 +82,11 @@ constexpr int kTcThreads = 320;          // 8 compute warps + MMA warp + TMA war
 constexpr int kTcComputeThreads = 256;
 constexpr int kTcMmaWarp = 8, kTcTmaWarp = 9;
 constexpr int kTcDrainTiles = 8;  // tiles accumulated in fp32 before an fp64 drain
-constexpr double kTcRhoPrecise = 64.0;  // rho_k above which a component drains every tile
+constexpr double kTcRhoPrecise = 64.0;  // mu^^2/var^ of a dimension above which its features
+                                        // drain after every tile with mass
 constexpr uint32_t kTcChunkBytes = 128u * 128u;  // one [128 x 64] 16-bit operand chunk
 constexpr float kTcRScale = 32768.0f;            // r is stored as fp16(r * 2^15)
-constexpr double kTcSharpKappa = 1e7;            // direct form above this kappa_k ...
+constexpr double kTcSharpKappa = 1e7;            // split dimensions above this kappa_k ...
 constexpr double kTcSmallKappa = 2.0e4;          // ... or above this one for a component
 constexpr double kTcSmallPoints = 50.0;          //     expecting fewer points than this
 constexpr float kTcXMax = 240.0f;                // |x^| beyond this cannot be split into fp16
@@ -163,11 +164,12 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 
 // Workspace layout of the tensor-core path (after the 256-byte status block).
 //   m, isc, sc : D f32 centring vector, 1/s and s (powers of two)
-//   c    : C*128 f32 per-component constants of the expanded form: the part
-//          added in the epilogue (0 if sharp)
+//   c    : C*128 f32 per-component constants of the expanded form (over the
+//          dimensions the contraction keeps): the part added in the epilogue
+//          (-inf for padding / pi = 0)
 //   ci   : C*128 f32 the part of that constant the accumulator starts from, in
-//          units of the W row scale (0 if sharp)
-//   wsc  : C*128 f32 power-of-two scale of each W row (1 if sharp)
+//          units of the W row scale
+//   wsc  : C*128 f32 power-of-two scale of each W row
 //   sharp: C*128 int32 1 if some of the component's dimensions are summed in
 //          direct form (nsplit: C*128 int32, how many: the first nsplit of perm)
 //   pmask: [C*128 x Fpad/32] u32 per feature of each component, 1 if it is
