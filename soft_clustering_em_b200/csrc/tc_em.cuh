@@ -29,7 +29,10 @@
 // dimensions, in data units from X itself (the fp16 split of x^ is too coarse
 // next to a narrow dimension), onto the tensor-core log-joint of the rest,
 // after a cheap filter on the tile's own features drops the rows that are
-// certainly far below the best component.
+// certainly far below the best component.  Their moments, sum r (x - mu) and
+// sum r (x - mu)^2 about the input means, are summed the same way (fp64
+// reductions from the few rows near the component) and replace the
+// tensor-core statistics of those dimensions.
 //
 // Statistics.  r is scaled by 2^15 and split into an fp16 pair r^ = r_hi +
 // r_lo (about 22 significant bits; fp16 alone leaves components that hold a
