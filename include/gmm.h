@@ -153,11 +153,12 @@ gmm_status gmm_mstep(const gmm_problem* p, const double* stats, int32_t nshards,
  * device that loads the library until the process exits.  The first call on a
  * device looks up that array's device address (cudaGetSymbolAddress) and
  * caches it; make that first call before any stream capture.  When the
- * statistics slots of the regular workspace do not all fit, fewer CTAs run the
- * fused pass (one slot each), which is slower but gives the same result up to
- * summation order; a problem for which not even one slot fits
- * (K*(2D+1)+1 doubles plus the parameter tables, above 32 MiB) is rejected with
- * GMM_ERR_UNSUPPORTED and a message on stderr.
+ * statistics slots of the regular workspace do not all fit, fewer CTAs (or
+ * clusters) run the fused pass, one slot each, which is slower but gives the
+ * same result up to summation order.  A tensor-core slot holds K*(4D+1)+1
+ * doubles; when not even one fits next to the parameter tables, the call runs
+ * the CUDA-core kernel, whose slot holds K*(2D+1)+1.  A problem for which not
+ * even that fits is rejected with GMM_ERR_UNSUPPORTED and a message on stderr.
  *
  * Every call on a device uses the same array and it keeps the previous call's
  * contents; each call resets the status word and rewrites everything else it
