@@ -126,15 +126,23 @@ inline int tc_nchunks(int D) { return (2 * D + kTcChunk - 1) / kTcChunk; }
 inline int tc_cluster(int K) { return (K + kTcComps - 1) / kTcComps; }
 
 // Byte offsets of the kernel's shared-memory regions (from a 1024-aligned base).
+// nfb F buffers of fbytes each: two when they fit (small D), so that a tile's
+// features can be written while the previous tile's statistics MMAs still
+// read the other buffer.
 struct TcSmem {
   uint32_t F, W, R, ONES, msm, iscs, csm, cis, wscs, shl, precs, xchg, bars, tslot, total;
+  uint32_t nfb, fbytes;
 };
 
-__host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
+constexpr uint32_t kTcMaxSmem = 232448;  // 227 KB per CTA
+
+__host__ __device__ inline TcSmem tc_smem_layout_n(int D, int C, int nchunks, uint32_t nfb) {
   TcSmem L;
   uint32_t off = 0;
+  L.nfb = nfb;
+  L.fbytes = 2u * nchunks * kTcChunkBytes;
   L.F = off;
-  off += 2u * nchunks * kTcChunkBytes;
+  off += nfb * L.fbytes;
   L.W = off;
   off += kTcStages * kTcChunkBytes;
   L.R = off;
@@ -163,6 +171,11 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
   off += 16;
   L.total = off + 1024;  // slack for aligning the dynamic base to 1024
   return L;
+}
+
+__host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
+  const TcSmem two = tc_smem_layout_n(D, C, nchunks, 2);
+  return two.total <= kTcMaxSmem ? two : tc_smem_layout_n(D, C, nchunks, 1);
 }
 
 // Workspace layout of the tensor-core path (after the 256-byte status block).
@@ -197,7 +210,7 @@ struct TcLayout {
 inline bool tc_shape_ok(int D, int K) {
   if (!(D >= 4 && D <= 128 && D % 4 == 0 && K >= 1 && K <= kTcComps * kTcMaxCluster))
     return false;
-  return tc_smem_layout(D, tc_cluster(K), tc_nchunks(D)).total <= 232448;  // 227 KB per CTA
+  return tc_smem_layout(D, tc_cluster(K), tc_nchunks(D)).total <= kTcMaxSmem;
 }
 
 inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
@@ -432,7 +445,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   for (int i = tid; i < 2048; i += kTcThreads)
     reinterpret_cast<__half*>(sOnes)[i] = __float2half_rn(1.0f);
   // padding features of F must read as zero in every MMA
-  for (uint32_t i = tid; i < 2u * nch * kTcChunkBytes / 16; i += kTcThreads)
+  for (uint32_t i = tid; i < L.nfb * L.fbytes / 16; i += kTcThreads)
     reinterpret_cast<uint4*>(sF)[i] = make_uint4(0, 0, 0, 0);
   if (MODE == kTcStats) {
     for (int f = 0; f <= 2 * D; f++)
@@ -509,9 +522,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         SCEM_TRACE(li, 8);
         tc_fence_after_sync();
         bool ok = true;
+        const uint32_t fofs = (uint32_t)(li % L.nfb) * L.fbytes;  // this tile's F buffer
         for (int c = 0; c < nch && ok; c++) {
-          const uint32_t fhi = fb + (uint32_t)c * kTcChunkBytes;
-          const uint32_t flo = fb + (uint32_t)(nch + c) * kTcChunkBytes;
+          const uint32_t fhi = fb + fofs + (uint32_t)c * kTcChunkBytes;
+          const uint32_t flo = fb + fofs + (uint32_t)(nch + c) * kTcChunkBytes;
           for (int part = 0; part < 2; part++) {
             ok = mbar_wait_bounded(&full[stage], phase, status, kAbort, a.wait_ns);
             if (!ok) break;
@@ -558,8 +572,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const uint64_t alo = desc_add(dR, 16384u + 2048u * ks);
               const bool acc = !(first && half == 0 && ks == 0);
               const uint32_t kr = 2048u * (uint32_t)(4 * half + ks);  // F rows of this K-step
-              const uint64_t fhi = desc_add(dFs, kr);
-              const uint64_t flo = desc_add(dFs, (uint32_t)nch * kTcChunkBytes + kr);
+              const uint64_t fhi = desc_add(dFs, fofs + kr);
+              const uint64_t flo = desc_add(dFs, fofs + (uint32_t)nch * kTcChunkBytes + kr);
               mma_bf16(tS, ahi, fhi, idS, acc);
               mma_bf16(tS, ahi, flo, idS, true);
               mma_bf16(tS, alo, fhi, idS, true);
@@ -682,14 +696,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int64_t li = 0; li < my_tiles && ok; li++) {
       const int64_t row0 = ((int64_t)cid + li * ncl) * kTcRows;
       if (t == 0) SCEM_TRACE(li, 0);
-      if (li > 0) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait_bounded(s_done, (uint32_t)((li - 1) & 1), status, kAbort,
-                                          a.wait_ns));
-        if (!ok) break;
+      // The previous tile's statistics MMAs must be done before its drain and
+      // before this tile's r^ reuses their buffer -- and, with one F buffer,
+      // before this tile's features overwrite theirs.  With two F buffers the
+      // wait moves past the conversion, which then overlaps those MMAs.
+      auto wait_prev_stats = [&]() -> bool {
+        const bool r = __all_sync(0xffffffffu,
+                                  mbar_wait_bounded(s_done, (uint32_t)((li - 1) & 1), status,
+                                                    kAbort, a.wait_ns));
         if (t == 0) SCEM_TRACE(li, 1);
         tc_fence_after_sync();
+        return r;
+      };
+      if (li > 0 && L.nfb == 1) {
+        ok = wait_prev_stats();
+        if (!ok) break;
       }
+      uint8_t* sFc = sF + (uint32_t)(li % L.nfb) * L.fbytes;  // this tile's F buffer
       // ---- X tile -> F = [x^, x^^2] as fp16 hi/lo in the swizzled layout.
       // The next tile's rows (contiguous in X) are pulled into L2 now, so that
       // its loads meet L2 rather than DRAM latency; up to 16 16-byte loads per
@@ -749,10 +772,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t o1 = (uint32_t)(f1 >> 6) * kTcChunkBytes + sw128_offset(n, f1 & 63);
           const uint32_t o2 = (uint32_t)(f2 >> 6) * kTcChunkBytes + sw128_offset(n, f2 & 63);
           const uint32_t lo_off = (uint32_t)nch * kTcChunkBytes;
-          *reinterpret_cast<uint2*>(sF + o1) = make_uint2(hx[0], hx[1]);
-          *reinterpret_cast<uint2*>(sF + lo_off + o1) = make_uint2(lx[0], lx[1]);
-          *reinterpret_cast<uint2*>(sF + o2) = make_uint2(hs[0], hs[1]);
-          *reinterpret_cast<uint2*>(sF + lo_off + o2) = make_uint2(ls[0], ls[1]);
+          *reinterpret_cast<uint2*>(sFc + o1) = make_uint2(hx[0], hx[1]);
+          *reinterpret_cast<uint2*>(sFc + lo_off + o1) = make_uint2(lx[0], lx[1]);
+          *reinterpret_cast<uint2*>(sFc + o2) = make_uint2(hs[0], hs[1]);
+          *reinterpret_cast<uint2*>(sFc + lo_off + o2) = make_uint2(ls[0], ls[1]);
         }
         if (t == 0) SCEM_TRACE(li, 13);
         nbatch++;
@@ -764,6 +787,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before_sync();
       mbar_arrive(f_full);
       if (t == 0) SCEM_TRACE(li, 3);
+      if (li > 0 && L.nfb == 2) {
+        ok = wait_prev_stats();
+        if (!ok) break;
+      }
       // Drain the previous tiles' statistics while the E-step MMAs run (they
       // write other tensor-memory columns); this tile's statistics MMAs wait
       // for it.
@@ -862,8 +889,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                   if (i0 + 4 * g4 + u >= ns) break;
                   const int f = min(fs[u], D - 1);
                   const uint32_t o = (uint32_t)(f >> 6) * kTcChunkBytes + sw128_offset(row, f & 63);
-                  const float xh = __half2float(*reinterpret_cast<const __half*>(sF + o)) +
-                                   __half2float(*reinterpret_cast<const __half*>(sF + lo_off + o));
+                  const float xh = __half2float(*reinterpret_cast<const __half*>(sFc + o)) +
+                                   __half2float(*reinterpret_cast<const __half*>(sFc + lo_off + o));
                   const float dd = xh - ms[u];
                   qa = fmaf(dd * dd, ps[u], qa);
                   const float ed = 9.6e-7f * (fabsf(xh) + fabsf(ms[u])) + 6.0e-8f;
