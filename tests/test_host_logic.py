@@ -1,0 +1,141 @@
+"""Host-side logic on the CPU: the input generator's guarantees, the parity rules
+the GPU tests judge by, and the bench's gating of stored ncu traffic."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import compare
+from soft_clustering_em_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+# ---------------------------------------------------------------- generator
+
+@pytest.mark.parametrize("name", ["uint8img", "bf16stream"])
+def test_row_blocks_are_the_same_whatever_else_is_drawn(name):
+    wl = synth.WORKLOADS[name]
+    start, n = 65_000, 1_200  # crosses the 65,536-row chunk boundary
+    full, zf = synth.make_data(wl, start + n)
+    block, zb = synth.make_data(wl, n, start=start)
+    np.testing.assert_array_equal(block, full[start:])
+    np.testing.assert_array_equal(zb, zf[start:])
+    small, _ = synth.make_data(wl, 500)
+    np.testing.assert_array_equal(small, full[:500])
+
+
+def test_workload_value_structure():
+    X, _ = synth.make_data(synth.WORKLOADS["uint8img"], 3_000)
+    assert X.dtype == np.float32 and X.min() >= 0 and X.max() <= 255
+    np.testing.assert_array_equal(X, np.rint(X))  # integers, exact in fp32
+    S, _ = synth.make_data(synth.WORKLOADS["sphere768"], 200)
+    np.testing.assert_allclose(np.linalg.norm(S.astype(np.float64), axis=1), 1.0, atol=1e-6)
+    B, _ = synth.make_data(synth.WORKLOADS["bf16stream"], 2_000)
+    assert B.dtype == np.uint16
+    f = synth.x_as_f64(synth.WORKLOADS["bf16stream"], B)
+    assert np.all(np.abs(f) < 4.0)  # means in [-1, 1], std <= 0.2
+
+
+def test_bf16_rounding_is_to_nearest_even():
+    one, next_up = 1.0, 1.0 + 2.0 ** -7  # adjacent bf16 values
+    x = np.array([one + 2.0 ** -8,            # halfway: ties to the even (1.0)
+                  next_up + 2.0 ** -8,        # halfway above an odd mantissa: up
+                  one + 2.0 ** -8 + 2.0 ** -20,  # just above halfway: up
+                  -(one + 2.0 ** -9)], dtype=np.float32)
+    got = synth.bf16_to_f32(synth.bf16_round(x))
+    np.testing.assert_array_equal(got, np.array([one, next_up + 2.0 ** -7, next_up, -one],
+                                                dtype=np.float32))
+
+
+def test_init_rows_are_distinct_sorted_and_in_range():
+    rows = synth.init_rows(10_000, 256, 2002)
+    assert rows.shape == (256,) and len(np.unique(rows)) == 256
+    assert np.all(np.diff(rows) > 0) and rows[0] >= 0 and rows[-1] < 10_000
+    np.testing.assert_array_equal(rows, synth.init_rows(10_000, 256, 2002))
+
+
+# ---------------------------------------------------------------- parity rules
+
+def _step(K=4, D=3, N=10_000.0):
+    w = np.array([0.5, 0.3, 0.2 - 5e-4, 5e-4])  # the last component: 5 points
+    mu = np.arange(K * D, dtype=np.float64).reshape(K, D) - 4.0
+    var = np.full((K, D), 2.0)
+    Nk = w * N
+    return (w, mu, var, -1234.5), Nk, N
+
+
+def test_weight_rule_is_relative_with_a_ten_point_floor():
+    ref, Nk, N = _step()
+    for k, scale in ((0, 1e-3 * ref[0][0]), (3, 1e-3 * 10 / N)):  # 5000 points; 5 points
+        for frac, ok in ((0.9, True), (1.1, False)):
+            w = ref[0].copy()
+            w[k] += frac * scale
+            rep = compare.compare_step(ref, (w, *ref[1:]), Nk, N)
+            assert rep["ok"] is ok, (k, frac, rep)
+            assert rep["w"] == pytest.approx(frac, rel=1e-6)
+
+
+def test_mean_rule_scales_with_max_of_mean_and_sigma():
+    ref, Nk, N = _step()
+    sigma = np.sqrt(2.0)
+    for (k, d), scale in (((1, 1), sigma), ((3, 2), 7.0)):  # mu = 0: sigma wins; mu = 7 wins
+        mu = ref[1].copy()
+        mu[k, d] += 0.9e-3 * scale
+        rep = compare.compare_step(ref, (ref[0], mu, *ref[2:]), Nk, N)
+        gated = Nk[k] >= compare.MIN_NK
+        assert rep["ok"], rep
+        assert (rep["mu"] if gated else rep["mu_ungated"]) == pytest.approx(0.9, rel=1e-6)
+    mu = ref[1].copy()
+    mu[1, 1] += 1.1e-3 * sigma
+    assert not compare.compare_step(ref, (ref[0], mu, *ref[2:]), Nk, N)["ok"]
+
+
+def test_mean_and_variance_are_gated_at_ten_points():
+    ref, Nk, N = _step()
+    var = ref[2].copy()
+    var[3] *= 1.5  # the 5-point component: reported, not judged
+    rep = compare.compare_step(ref, (ref[0], ref[1], var, ref[3]), Nk, N)
+    assert rep["ok"] and rep["var_ungated"] == pytest.approx(500.0)
+    assert rep["gated_components"] == 3
+    var = ref[2].copy()
+    var[2, 0] *= 1.0011  # a 1995-point component: judged at 1e-3 relative
+    assert not compare.compare_step(ref, (ref[0], ref[1], var, ref[3]), Nk, N)["ok"]
+
+
+def test_loglik_rule_is_relative_1e4():
+    ref, Nk, N = _step()
+    for frac, ok in ((0.9, True), (1.1, False)):
+        ll = ref[3] + frac * 1e-4 * abs(ref[3])
+        assert compare.compare_step(ref, (*ref[:3], ll), Nk, N)["ok"] is ok
+
+
+def test_topm_mismatch_is_excused_only_within_the_gap():
+    idx_ref = np.array([[0, 1], [2, 3]])
+    resp_ref = np.array([[0.6, 0.39], [0.5, 0.49]])
+    R_sorted = np.array([[0.6, 0.39, 0.01], [0.5, 0.49999, 0.00001]])
+    # row 1's second and third candidates are 0.49999 - 1e-5 apart: a swap there is excused
+    idx_got = np.array([[0, 1], [2, 4]])
+    bad, worst = compare.compare_topm(idx_ref, resp_ref, idx_got, resp_ref, R_sorted)
+    assert bad == 1  # only the excusal test: rank 1 of row 1 has gap 0.49998 >= 1e-5
+    R_close = np.array([[0.6, 0.39, 0.01], [0.5, 0.499995, 0.499990]])
+    bad, _ = compare.compare_topm(idx_ref, resp_ref, idx_got, resp_ref, R_close)
+    assert bad == 0
+    resp_got = resp_ref * np.array([[1.0009, 1.0], [1.0, 1.0]])
+    _, worst = compare.compare_topm(idx_ref, resp_ref, idx_ref, resp_got, R_sorted)
+    assert worst == pytest.approx(0.9, rel=1e-6)
+
+
+# ---------------------------------------------------------------- bench
+
+def test_stored_traffic_is_used_only_for_the_source_it_was_measured_on(monkeypatch):
+    import bench
+
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    stored = json.load(open(path))["uint8img"]
+    monkeypatch.setattr(bench, "fused_source_sha", lambda: stored["source_sha"])
+    assert bench.ncu_traffic("uint8img") == stored["dram_bytes_per_launch"]
+    assert bench.ncu_traffic("bf16stream") is None
+    monkeypatch.setattr(bench, "fused_source_sha", lambda: "0" * 16)
+    assert bench.ncu_traffic("uint8img") is None
