@@ -81,6 +81,7 @@ CASES = [
     ("uint8img", 20_011, 256, 3),
     ("sphere768", 3_001, 1024, 2),
     ("gauss4096", 20_000, 4096, 2),
+    ("gauss4096", 20_000, 512, 2),  # D = 96 on the tensor cores: 3 feature chunks, 4-CTA clusters
     ("bf16stream", 50_001, 1024, 3),
 ]
 
@@ -423,3 +424,19 @@ def test_split_dimensions_match_oracle(G):
     # the collapsed component keeps its 40 points and its zero spread in dimensions 0-3
     assert abs(got[0][0] * N - 40.0) < 0.05
     np.testing.assert_allclose(got[2][0][:4], 1e-6, rtol=1e-6)
+
+
+@pytest.mark.parametrize("D,K", [(48, 200), (96, 300)])
+def test_padded_and_odd_feature_chunks(G, D, K):
+    """2D not a multiple of 64 (D = 48: two chunks, the second half padding) and an odd
+    chunk count (D = 96: three chunks), with ragged K and N."""
+    rng = np.random.default_rng(D)
+    N = 5_003
+    centers = rng.uniform(-6, 6, size=(K, D))
+    z = rng.integers(0, K, size=N)
+    X = (centers[z] + rng.normal(size=(N, D))).astype(np.float32)
+    w = rng.dirichlet(np.ones(K))
+    mu = X[rng.choice(N, K, replace=False)]
+    ref, got = _tiny(G, X, w, mu, np.ones((K, D)))
+    rep = compare.compare_step(ref[:4], got, ref[4])
+    assert rep["ok"], rep
