@@ -82,6 +82,8 @@ CASES = [
     ("sphere768", 3_001, 1024, 2),
     ("gauss4096", 20_000, 4096, 2),
     ("gauss4096", 20_000, 512, 2),  # D = 96 on the tensor cores: 3 feature chunks, 4-CTA clusters
+    ("bf16stream", 30_001, 1536, 2),  # 12-CTA clusters (non-portable size)
+    ("bf16stream", 30_001, 2048, 2),  # 16-CTA clusters, the largest
     ("bf16stream", 50_001, 1024, 3),
 ]
 
