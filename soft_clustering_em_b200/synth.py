@@ -153,3 +153,37 @@ def init_rows(N: int, K: int, seed: int) -> np.ndarray:
     """K distinct row indices in [0, N), drawn uniformly with PCG64(seed)."""
     rng = np.random.Generator(np.random.PCG64(seed))
     return np.sort(rng.choice(N, size=K, replace=False)).astype(np.int64)
+
+
+def topm_inputs(N: int, K: int, m: int, seed: int, ties_at: float = None):
+    """A seeded stand-in for a top-m assignment: (idx N x m int32, resp N x m float32).
+
+    Each row holds m distinct component indices.  The first is skewed towards
+    low indices (u^2 scaling), so list sizes are uneven like those of a mixture
+    with unequal weights.  The others step forward from it modulo K.  resp is
+    descending along a row and sums to at most 1.  With ``ties_at`` set, about
+    one entry in 16 of ranks 2..m is then overwritten with exactly
+    float32(ties_at), which can break that order.
+    """
+    assert 1 <= m <= K
+    rng = np.random.Generator(np.random.PCG64(seed))
+    first = np.minimum(K - 1, (K * rng.random(N) ** 2).astype(np.int64))
+    idx = np.empty((N, m), dtype=np.int64)
+    idx[:, 0] = first
+    if m > 1:
+        steps = rng.integers(1, (K - 1) // (m - 1) + 1, size=(N, m - 1))
+        idx[:, 1:] = (first[:, None] + np.cumsum(steps, axis=1)) % K
+    resp = np.empty((N, m), dtype=np.float64)
+    resp[:, 0] = rng.uniform(0.3, 1.0, N)
+    rest = 1.0 - resp[:, 0]
+    for j in range(1, m):
+        resp[:, j] = rest * rng.random(N)
+        rest = rest - resp[:, j]
+    if m > 1:
+        resp[:, 1:] = -np.sort(-resp[:, 1:], axis=1)
+        resp[:, 1:] = np.minimum(resp[:, 1:], resp[:, :1])
+    resp = resp.astype(np.float32)
+    if ties_at is not None and m > 1:
+        hit = rng.random((N, m - 1)) < 1.0 / 16
+        resp[:, 1:][hit] = np.float32(ties_at)
+    return idx.astype(np.int32), resp
