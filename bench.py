@@ -57,6 +57,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--ivf", action="store_true",
+                    help="time the IVF list build (gmm_ivf_build) instead of the EM step")
+    ap.add_argument("--ivf-tau", type=float, default=0.1)
     return ap.parse_args()
 
 
@@ -419,10 +422,80 @@ def ours(args):
         dist.destroy_process_group()
 
 
+def ivf_bench(args):
+    """One GPU: the IVF list build on a seeded top-m assignment of the bf16stream size.
+
+    A step is one gmm_ivf_build (counter reset, count pass, two scans, fill pass)
+    over N points with m = 2 candidates each.  The inputs (N x m int32 + float32)
+    exceed L2, so no flush is needed.  Algorithmic bytes per build: the
+    assignment read once, the ids and offsets written once.
+    """
+    import torch
+
+    from oracle import ivf as ivf_oracle
+    from soft_clustering_em_b200 import gmm as G
+
+    wl = synth.WORKLOADS["bf16stream"]
+    N, K, m, tau = args.rows or wl.N, wl.K, wl.topm, args.ivf_tau
+    dev = torch.device("cuda", 0)
+    idx, resp = synth.topm_inputs(N, K, m, seed=wl.init_seed)
+    idx_d, resp_d = torch.from_numpy(idx).to(dev), torch.from_numpy(resp).to(dev)
+    ws = torch.zeros(G.gmm_ivf_workspace_size(N, K), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else None)
+    for _ in range(max(3, args.warmup)):
+        offsets, ids = G.gmm_ivf_build(idx_d, resp_d, K, tau, ws=ws)
+    torch.cuda.synchronize(dev)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    launches0 = G.gmm_launch_count()
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        starts[i].record(stream)
+        offsets, ids = G.gmm_ivf_build(idx_d, resp_d, K, tau, ws=ws)
+        stops[i].record(stream)
+    torch.cuda.synchronize(dev)
+    launches = G.gmm_launch_count() - launches0
+    clocks = sampler.stop()
+    ms = [a.elapsed_time(b) for a, b in zip(starts, stops)]
+    total_ms = sum(ms)
+    rc, flags = G.gmm_device_status(ws)
+    total = int(offsets[-1].item())
+    algo_bytes = N * m * 8 + total * 8 + (K + 1) * 8
+    pk, kind = peaks()
+    achieved = algo_bytes / (total_ms / args.steps * 1e-3) / 1e9
+    # oracle on a bounded sample of the same assignment, on the host
+    n_s = min(N, 10_000_000)
+    t0 = time.perf_counter()
+    ivf_oracle.ivf_lists(idx[:n_s], resp[:n_s], K, tau)
+    cpu_s = time.perf_counter() - t0
+    line = {
+        "metric": "IVF list build from a top-2 assignment, points/s on 1 B200",
+        "value": N * args.steps / (total_ms * 1e-3), "unit": "points/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+        "config": {"workload": "ivf_build", "N": N, "K": K, "m": m, "tau": tau,
+                   "entries": total, "list_inflation": total / N,
+                   "l2": "inputs larger than L2 (no flush)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                     "peak_kind": kind, "algorithmic_bytes_per_build": algo_bytes},
+        "cpu_baseline": {"value": n_s / cpu_s, "unit": "points/s", "cores": 1,
+                         "kind": "oracle", "sample": f"first {n_s} points of the assignment"},
+        "gpu_launches": launches, "device_status": rc, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         reference_arm(args)
+        return
+    if args.ivf:
+        ivf_bench(args)
         return
     ours(args)
 

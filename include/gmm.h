@@ -32,7 +32,8 @@
  *  - ws is a caller-owned device workspace of at least gmm_workspace_size()
  *    bytes, 256-byte aligned.  Its size depends on D, K, the dtype and the
  *    device, never on N.  Calls that share a workspace must be ordered on one
- *    stream.
+ *    stream.  (gmm_ivf_build, which files points into lists after the fit, has
+ *    a workspace of its own, sized by gmm_ivf_workspace_size.)
  *  - stream is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream).  Every entry point only enqueues work on it and returns without
  *    waiting, except gmm_device_status.
@@ -85,6 +86,8 @@ typedef struct {
 #define GMM_DEVFLAG_X_RANGE 0x8u         /* an element of X lies so far from the mixture mean
                                             (over 240 scale units, about 480 mixture standard
                                             deviations) that the tensor-core path clipped it */
+#define GMM_DEVFLAG_BAD_INDEX 0x10u      /* gmm_ivf_build: a component index outside [0, K)
+                                            or repeated within one point's row */
 
 /*
  * Bytes of device workspace needed for problem p on the CURRENT device.
@@ -197,10 +200,44 @@ gmm_status gmm_assign_topm(const gmm_problem* p, const void* X, const float* w,
                            float* resp, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Inverted lists of an IVF coarse quantizer from a top-m assignment: each point
+ * is filed under the clusters its responsibilities choose (Flash-GMM abstract:
+ * GMM responsibilities put border vectors into several clusters' lists).  The
+ * pages give no rule; this library's: point n joins the list of idx[n][0]
+ * always, and the list of idx[n][j] (j >= 1) when resp[n][j] >= tau, compared
+ * in float32.
+ *
+ *   idx, resp  device, N x m row-major, as gmm_assign_topm returns them
+ *              (1 <= m <= min(K, 8)); resp of rank 1 is not read.
+ *   tau        the threshold; not NaN (tau > 1 gives a plain partition by the
+ *              rank-1 component, tau <= 0 files every point m times).
+ *   offsets    device, K + 1 int64: list k is ids[offsets[k] .. offsets[k+1]),
+ *              offsets[K] is the number of entries.
+ *   ids        device, ids_capacity int64 point indices, ascending inside each
+ *              list; ids_capacity >= N * m (the most entries there can be).
+ *   ws         device workspace of gmm_ivf_workspace_size(N, K) bytes, 256-byte
+ *              aligned, its first word the status word (zero it once; a call
+ *              leaves it unchanged unless it raises a bit).  It grows with N up
+ *              to a cap: about 64 MiB of per-chunk counts plus 8 bytes per list.
+ *
+ * The result does not depend on the launch configuration or on timing.  An
+ * entry of idx outside [0, K), or repeating an earlier index of its row, is
+ * skipped and raises GMM_DEVFLAG_BAD_INDEX, which gmm_device_status reports as
+ * GMM_ERR_INVALID_ARG.  Host errors: GMM_ERR_INVALID_ARG (N < 1, K < 1, m out
+ * of range, a null pointer, NaN tau, ids_capacity < N * m),
+ * GMM_ERR_UNSUPPORTED (K > 65536 or N > 2^40), GMM_ERR_WORKSPACE.
+ */
+gmm_status gmm_ivf_workspace_size(int64_t N, int32_t K, size_t* bytes);
+gmm_status gmm_ivf_build(int64_t N, int32_t K, int32_t m, const int32_t* idx, const float* resp,
+                         float tau, int64_t* offsets, int64_t* ids, int64_t ids_capacity,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/*
  * Waits for stream, then reads the device status word of ws into *flags
  * (GMM_DEVFLAG_* bits; may be NULL) and, if clear != 0, resets it to 0.
- * Returns GMM_OK when no bit is set, GMM_ERR_NUMERIC for the data/parameter/range
- * bits, GMM_ERR_TIMEOUT for the wait bit.  The only entry point that blocks.
+ * Returns GMM_OK when no bit is set, GMM_ERR_TIMEOUT for the wait bit,
+ * GMM_ERR_NUMERIC for the data/parameter/range bits, GMM_ERR_INVALID_ARG for
+ * the index bit.  The only entry point that blocks.
  */
 gmm_status gmm_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* flags,
                              int32_t clear);

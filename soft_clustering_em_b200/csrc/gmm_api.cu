@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "gmm.h"
+#include "ivf.cuh"
 #include "simt_em.cuh"
 #include "tc_em.cuh"
 #include "tma_host.h"
@@ -120,6 +121,35 @@ void trace_end(cudaStream_t st) {
 gmm_status launched(int n) {
   g_launches += n;
   return launch_status();
+}
+
+// One walk of gmm_ivf_build over all chunks, for m candidates per point.
+template <int kM>
+void ivf_walk_m(bool fill, int64_t N, int K, const int32_t* idx, const float* resp, float tau,
+                const IvfLayout& L, int64_t* cnt, const int64_t* offsets, int64_t* ids,
+                unsigned int* status, cudaStream_t st) {
+  const int ctas = (L.B + kIvfWarps - 1) / kIvfWarps;
+  if (fill)
+    ivf_walk_kernel<kM, true><<<ctas, kIvfWarps * 32, 0, st>>>(N, K, idx, resp, tau, L.B, L.R,
+                                                               cnt, offsets, ids, status);
+  else
+    ivf_walk_kernel<kM, false><<<ctas, kIvfWarps * 32, 0, st>>>(N, K, idx, resp, tau, L.B, L.R,
+                                                                cnt, offsets, ids, status);
+}
+
+void ivf_walk(int m, bool fill, int64_t N, int K, const int32_t* idx, const float* resp,
+              float tau, const IvfLayout& L, int64_t* cnt, const int64_t* offsets, int64_t* ids,
+              unsigned int* status, cudaStream_t st) {
+  switch (m) {
+    case 1: return ivf_walk_m<1>(fill, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+    case 2: return ivf_walk_m<2>(fill, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+    case 3: return ivf_walk_m<3>(fill, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+    case 4: return ivf_walk_m<4>(fill, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+    case 5: return ivf_walk_m<5>(fill, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+    case 6: return ivf_walk_m<6>(fill, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+    case 7: return ivf_walk_m<7>(fill, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+    default: return ivf_walk_m<8>(fill, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+  }
 }
 
 template <typename XT, int MODE>
@@ -545,6 +575,39 @@ gmm_status gmm_assign_topm(const gmm_problem* p, const void* X, const float* w, 
   return fused_pass<kModeTopm>(p, X, wp, m, idx, resp, st);
 }
 
+gmm_status gmm_ivf_workspace_size(int64_t N, int32_t K, size_t* bytes) {
+  if (!bytes || N < 1 || K < 1) return GMM_ERR_INVALID_ARG;
+  if (K > kMaxK || (size_t)N > ((size_t)1 << 40)) return GMM_ERR_UNSUPPORTED;
+  *bytes = ivf_layout(N, K).total;
+  return GMM_OK;
+}
+
+gmm_status gmm_ivf_build(int64_t N, int32_t K, int32_t m, const int32_t* idx, const float* resp,
+                         float tau, int64_t* offsets, int64_t* ids, int64_t ids_capacity,
+                         void* ws, size_t ws_bytes, void* stream) {
+  size_t need = 0;
+  gmm_status s = gmm_ivf_workspace_size(N, K, &need);
+  if (s != GMM_OK) return s;
+  if (m < 1 || m > kMaxTopM || m > K) return GMM_ERR_INVALID_ARG;
+  if (!idx || !resp || !offsets || !ids || isnan(tau)) return GMM_ERR_INVALID_ARG;
+  if (ids_capacity < N * m) return GMM_ERR_INVALID_ARG;
+  if (!ws || ((uintptr_t)ws) % 256 != 0 || ws_bytes < need) return GMM_ERR_WORKSPACE;
+  const IvfLayout L = ivf_layout(N, K);
+  char* b = (char*)ws;
+  unsigned int* status = (unsigned int*)(b + L.status);
+  int64_t* tot = (int64_t*)(b + L.tot);
+  int64_t* cnt = (int64_t*)(b + L.cnt);
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemsetAsync(cnt, 0, (size_t)L.B * K * 8, st) != cudaSuccess)
+    return launch_status(), GMM_ERR_CUDA;
+  ivf_walk(m, false, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+  ivf_scan_chunks_kernel<<<(K + kIvfWarps - 1) / kIvfWarps, kIvfWarps * 32, 0, st>>>(K, L.B, cnt,
+                                                                                    tot);
+  ivf_offsets_kernel<<<1, kIvfScanThreads, 0, st>>>(K, tot, offsets);
+  ivf_walk(m, true, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+  return launched(4);
+}
+
 gmm_status gmm_launch_count(uint64_t* count) {
   if (!count) return GMM_ERR_INVALID_ARG;
   *count = g_launches;
@@ -572,6 +635,7 @@ gmm_status gmm_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* 
   if (f & GMM_DEVFLAG_WAIT_TIMEOUT) return GMM_ERR_TIMEOUT;
   if (f & (GMM_DEVFLAG_NONFINITE_X | GMM_DEVFLAG_BAD_PARAMS | GMM_DEVFLAG_X_RANGE))
     return GMM_ERR_NUMERIC;
+  if (f & GMM_DEVFLAG_BAD_INDEX) return GMM_ERR_INVALID_ARG;
   return GMM_OK;
 }
 

@@ -19,11 +19,12 @@ GMM_ERR_NUMERIC, GMM_ERR_TIMEOUT, GMM_ERR_WORKSPACE = 4, 5, 6
 GMM_F32, GMM_BF16 = 0, 1
 GMM_INIT_VAR_ONE, GMM_INIT_VAR_DATA = 0, 1
 GMM_DEVFLAG_NONFINITE_X, GMM_DEVFLAG_BAD_PARAMS, GMM_DEVFLAG_WAIT_TIMEOUT = 0x1, 0x2, 0x4
+GMM_DEVFLAG_X_RANGE, GMM_DEVFLAG_BAD_INDEX = 0x8, 0x10
 
 EXPORTS = ("gmm_workspace_size", "gmm_init", "gmm_em_step", "gmm_em_step_noalloc",
            "gmm_estep_stats", "gmm_mstep", "gmm_fit", "gmm_loglik",
-           "gmm_assign_topm", "gmm_device_status", "gmm_trace_fused", "gmm_launch_count",
-           "gmm_status_string")
+           "gmm_assign_topm", "gmm_ivf_workspace_size", "gmm_ivf_build", "gmm_device_status",
+           "gmm_trace_fused", "gmm_launch_count", "gmm_status_string")
 
 
 class gmm_problem(ctypes.Structure):
@@ -60,6 +61,8 @@ def load_library(path: str = LIB_PATH):
     lib.gmm_fit.argtypes = [PP, P, I32, P, P, P, P, P, SZ, P]
     lib.gmm_loglik.argtypes = [PP, P, P, P, P, P, P, SZ, P]
     lib.gmm_assign_topm.argtypes = [PP, P, P, P, P, I32, P, P, P, SZ, P]
+    lib.gmm_ivf_workspace_size.argtypes = [I64, I32, ctypes.POINTER(SZ)]
+    lib.gmm_ivf_build.argtypes = [I64, I32, I32, P, P, ctypes.c_float, P, P, I64, P, SZ, P]
     lib.gmm_device_status.argtypes = [P, SZ, P, ctypes.POINTER(ctypes.c_uint32), I32]
     lib.gmm_trace_fused.argtypes = [P, P]
     lib.gmm_launch_count.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
@@ -223,6 +226,37 @@ def gmm_assign_topm(X, w, mu, var, m, var_floor=1e-6, ws=None, stream=None):
                                           int(m), _ptr(idx), _ptr(resp), _ptr(ws), ws.numel(),
                                           _stream(stream)), "gmm_assign_topm")
     return idx, resp
+
+
+def gmm_ivf_workspace_size(N, K) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().gmm_ivf_workspace_size(int(N), int(K), ctypes.byref(n)),
+           "gmm_ivf_workspace_size")
+    return int(n.value)
+
+
+def gmm_ivf_build(idx, resp, K, tau, ws=None, stream=None):
+    """(offsets (K+1) int64, ids (N*m) int64): IVF lists from a top-m assignment.
+
+    idx (N x m int32) and resp (N x m float32) as gmm_assign_topm returns them.
+    List k is ids[offsets[k]:offsets[k+1]]; entries past offsets[K] are unused.
+    ws: a zeroed uint8 device tensor of gmm_ivf_workspace_size(N, K) bytes
+    (allocated here when None); its first word is the device status word.
+    """
+    if idx.dtype != torch.int32 or resp.dtype != torch.float32:
+        raise TypeError("idx must be int32 and resp float32")
+    if idx.dim() != 2 or resp.shape != idx.shape or not (idx.is_contiguous()
+                                                       and resp.is_contiguous()):
+        raise ValueError("idx and resp must be contiguous N x m tensors of the same shape")
+    N, m = idx.shape
+    if ws is None:
+        ws = torch.zeros(gmm_ivf_workspace_size(N, K), dtype=torch.uint8, device=idx.device)
+    offsets = torch.empty(int(K) + 1, dtype=torch.int64, device=idx.device)
+    ids = torch.empty(N * m, dtype=torch.int64, device=idx.device)
+    _check(load_library().gmm_ivf_build(int(N), int(K), int(m), _ptr(idx), _ptr(resp),
+                                        float(tau), _ptr(offsets), _ptr(ids), N * m, _ptr(ws),
+                                        ws.numel(), _stream(stream)), "gmm_ivf_build")
+    return offsets, ids
 
 
 def gmm_device_status(ws, clear=True, stream=None):

@@ -29,7 +29,8 @@ def test_header_declares_the_calls():
     names = declared_functions()
     for n in ("gmm_init", "gmm_em_step", "gmm_em_step_noalloc", "gmm_estep_stats", "gmm_mstep",
               "gmm_fit", "gmm_loglik",
-              "gmm_assign_topm", "gmm_workspace_size", "gmm_device_status", "gmm_trace_fused",
+              "gmm_assign_topm", "gmm_ivf_workspace_size", "gmm_ivf_build",
+              "gmm_workspace_size", "gmm_device_status", "gmm_trace_fused",
               "gmm_launch_count", "gmm_status_string"):
         assert n in names
 
@@ -123,3 +124,46 @@ def test_split_step_argument_checks(lib):
     bad = G.problem(0, 4, 3)
     assert lib.gmm_mstep(ctypes.byref(bad), P(16), 1, P(16), P(16), P(16), P(0), P(0)) == \
         G.GMM_ERR_INVALID_ARG
+
+
+def _ivf_ws(lib, N, K):
+    n = ctypes.c_size_t(0)
+    rc = lib.gmm_ivf_workspace_size(N, K, ctypes.byref(n))
+    return rc, n.value
+
+
+def test_ivf_workspace_grows_with_n_up_to_a_cap(lib):
+    assert _ivf_ws(lib, 0, 4)[0] == G.GMM_ERR_INVALID_ARG
+    assert _ivf_ws(lib, 10, 0)[0] == G.GMM_ERR_INVALID_ARG
+    assert _ivf_ws(lib, 10, 65537)[0] == G.GMM_ERR_UNSUPPORTED
+    assert _ivf_ws(lib, (1 << 40) + 1, 4)[0] == G.GMM_ERR_UNSUPPORTED
+    assert lib.gmm_ivf_workspace_size(10, 4, None) == G.GMM_ERR_INVALID_ARG
+    sizes = [_ivf_ws(lib, N, 1024)[1] for N in (1, 10**4, 10**6, 10**8, 10**10)]
+    assert sizes == sorted(sizes) and sizes[-2] == sizes[-1]  # capped chunk count
+    for K in (1024, 4096, 65536):
+        assert _ivf_ws(lib, 10**9, K)[1] <= (64 << 20) + 8 * K + 1024
+
+
+def test_ivf_build_argument_checks(lib):
+    P = ctypes.c_void_p
+    N, K, m = 100, 16, 2
+    ok_ws = _ivf_ws(lib, N, K)[1]
+
+    def call(N=N, K=K, m=m, idx=16, resp=16, tau=0.1, off=16, ids=16, cap=N * m, ws=256,
+             ws_bytes=ok_ws):
+        return lib.gmm_ivf_build(N, K, m, P(idx), P(resp), tau, P(off), P(ids), cap, P(ws),
+                                 ws_bytes, P(0))
+
+    assert call(N=0) == G.GMM_ERR_INVALID_ARG
+    assert call(K=0) == G.GMM_ERR_INVALID_ARG
+    assert call(K=65537) == G.GMM_ERR_UNSUPPORTED
+    for bad_m in (0, 9):
+        assert call(m=bad_m) == G.GMM_ERR_INVALID_ARG
+    assert call(K=1, m=2) == G.GMM_ERR_INVALID_ARG  # m > K
+    for name in ("idx", "resp", "off", "ids"):
+        assert call(**{name: 0}) == G.GMM_ERR_INVALID_ARG, name
+    assert call(tau=float("nan")) == G.GMM_ERR_INVALID_ARG
+    assert call(cap=N * m - 1) == G.GMM_ERR_INVALID_ARG
+    assert call(ws=0) == G.GMM_ERR_WORKSPACE
+    assert call(ws=128) == G.GMM_ERR_WORKSPACE
+    assert call(ws_bytes=ok_ws - 1) == G.GMM_ERR_WORKSPACE
