@@ -60,6 +60,9 @@ def parse():
     ap.add_argument("--ivf", action="store_true",
                     help="time the IVF list build (gmm_ivf_build) instead of the EM step")
     ap.add_argument("--ivf-tau", type=float, default=0.1)
+    ap.add_argument("--host-stream", action="store_true",
+                    help="time EM with X in pinned host memory (gmm_em_step_host)")
+    ap.add_argument("--chunk-rows", type=int, default=1 << 17)
     return ap.parse_args()
 
 
@@ -489,6 +492,77 @@ def ivf_bench(args):
     print(json.dumps(line), flush=True)
 
 
+def host_stream_bench(args):
+    """One GPU: EM iterations with X in pinned host memory, streamed in chunks.
+
+    A step is one gmm_em_step_host: every chunk of X crosses PCIe inside the
+    step (copy stream) while the previous chunk's E-step runs, then one M-step;
+    the step's LL is read back to pinned host memory.  Timed with CUDA events on
+    the compute stream; the copy stream waits on the start event.
+    """
+    import torch
+
+    from soft_clustering_em_b200 import gmm as G
+
+    wl = synth.WORKLOADS[args.workload]
+    N = args.rows or wl.N
+    dev = torch.device("cuda", 0)
+    X_np, _ = synth.make_data(wl, N)
+    Xh = torch.from_numpy(X_np.view(np.int16) if wl.dtype == "bf16" else X_np)
+    if wl.dtype == "bf16":
+        Xh = Xh.view(torch.bfloat16)
+    Xh = Xh.pin_memory()
+    Xd = Xh.to(dev)
+    mode = G.GMM_INIT_VAR_ONE if wl.var_init == "one" else G.GMM_INIT_VAR_DATA
+    p = G.problem_for(Xh, wl.K, wl.var_floor)
+    ws = G.workspace(p, dev)
+    w, mu, var = G.gmm_init(Xd, synth.init_rows(N, wl.K, wl.init_seed), wl.K, mode,
+                            wl.var_floor, ws=ws)
+    del Xd  # from here on X lives only in host memory
+    torch.cuda.empty_cache()
+    staging = torch.empty(G.gmm_host_staging_size(p, args.chunk_rows), dtype=torch.uint8,
+                          device=dev)
+    ll = torch.zeros(1, dtype=torch.float64, device=dev)
+    ll_host = torch.zeros(args.steps, dtype=torch.float64).pin_memory()
+    stream = torch.cuda.current_stream(dev)
+    cs = G.copy_stream_for(dev)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else None)
+    for _ in range(max(3, args.warmup)):
+        G.gmm_em_step_host(Xh, w, mu, var, ll, args.chunk_rows, wl.var_floor, staging=staging,
+                           ws=ws)
+    torch.cuda.synchronize(dev)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = G.gmm_launch_count()
+    start.record(stream)
+    cs.wait_event(start)
+    for i in range(args.steps):
+        G.gmm_em_step_host(Xh, w, mu, var, ll, args.chunk_rows, wl.var_floor, staging=staging,
+                           ws=ws)
+        ll_host[i].copy_(ll[0], non_blocking=True)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = G.gmm_launch_count() - launches0
+    clocks = sampler.stop()
+    ms = start.elapsed_time(stop)
+    rc, flags = G.gmm_device_status(ws)
+    h2d = N * wl.D * (2 if wl.dtype == "bf16" else 4)
+    line = {
+        "metric": "EM iterations/s with X streamed from pinned host memory (gmm_em_step_host)",
+        "value": args.steps / (ms * 1e-3), "unit": "EM iterations/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": dict(workload_config(wl, N), chunk_rows=args.chunk_rows,
+                       l2="X crosses PCIe every step"),
+        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 8,
+        "h2d_gbs": h2d * args.steps / (ms * 1e-3) / 1e9,
+        "gpu_launches": launches, "device_status": rc, "ll_last": float(ll_host[-1]),
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -496,6 +570,9 @@ def main():
         return
     if args.ivf:
         ivf_bench(args)
+        return
+    if args.host_stream:
+        host_stream_bench(args)
         return
     ours(args)
 

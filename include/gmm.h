@@ -182,6 +182,39 @@ gmm_status gmm_em_step_noalloc(const gmm_problem* p, const void* X, float* w, fl
 gmm_status gmm_fit(const gmm_problem* p, const void* X, int32_t iters, float* w, float* mu,
                    float* var, double* ll_history, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * One EM iteration with X in HOST memory: the out-of-core form, for data larger
+ * than the device (Flash-GMM abstract: datasets far larger than fit before on one
+ * device, since the method's device memory is O(K*D) whatever N is).
+ *
+ * X_host (N x D row-major, p->xdtype, HOST memory) is copied chunk_rows rows at
+ * a time into two device staging buffers on copy_stream, while stream runs the
+ * fused E-step and statistics pass on the other buffer.  Each chunk's fp64
+ * statistics are added, in chunk order, into one running total, and one
+ * M-step follows, so the result is the EM iteration of gmm_em_step on the same
+ * rows (the statistics are summed in another order: equal up to rounding, and
+ * deterministic for a given chunk_rows).  *loglik gets LL of the input
+ * parameters.
+ *
+ *   X_host       should be pinned (cudaHostAlloc / cudaHostRegister) for the
+ *                copies to overlap the E-step; pageable memory works, without
+ *                overlap.  It must stay valid and unchanged until stream has
+ *                completed the call's work.
+ *   chunk_rows   >= 1; rows per copy (the last chunk may hold fewer).
+ *   staging      device, 256-byte aligned, gmm_host_staging_size(p, chunk_rows)
+ *                bytes: two chunks of X plus two statistics buffers.
+ *   ws           the workspace of gmm_workspace_size(p), as for gmm_em_step.
+ *   stream, copy_stream  cudaStream_t as void*; they may be the same stream
+ *                (no overlap).  The call returns once everything is enqueued.
+ * Errors: as gmm_em_step, plus GMM_ERR_INVALID_ARG for chunk_rows < 1 or a null
+ * X_host and GMM_ERR_WORKSPACE for missing, misaligned or short staging.
+ */
+gmm_status gmm_host_staging_size(const gmm_problem* p, int64_t chunk_rows, size_t* bytes);
+gmm_status gmm_em_step_host(const gmm_problem* p, const void* X_host, int64_t chunk_rows,
+                            void* staging, size_t staging_bytes, float* w, float* mu, float* var,
+                            double* loglik, void* ws, size_t ws_bytes, void* stream,
+                            void* copy_stream);
+
 /* LL(theta) of the given parameters into *loglik (device, 1 double).  Parameters unchanged. */
 gmm_status gmm_loglik(const gmm_problem* p, const void* X, const float* w, const float* mu,
                       const float* var, double* loglik, void* ws, size_t ws_bytes,

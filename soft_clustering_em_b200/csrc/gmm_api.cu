@@ -302,16 +302,21 @@ gmm_status tc_pass(const gmm_problem* p, const void* X, char* ws, const TcLayout
 }
 
 // E-step and statistics of the rows of X into the canonical buffer `stats`.
+// n_prep is the point count the tensor-core prep sizes its small-component
+// rule by (pi_k * n_prep points): p->N, or the whole data's N when X is one
+// chunk of it.
 gmm_status estep_stats_impl(const gmm_problem* p, const void* X, const float* w,
                             const float* mu, const float* var, double* stats, void* ws_base,
-                            const Plan& P, cudaStream_t st) {
+                            const Plan& P, cudaStream_t st, int64_t n_prep) {
   char* ws = (char*)ws_base;
   gmm_status s;
   const size_t KD = (size_t)p->K * p->D;
   const unsigned blocks = (unsigned)((KD + 255) / 256);
   if (P.use_tc) {
     const TcLayout& T = P.tc;
-    if ((s = tc_prep(p, w, mu, var, ws, T, st)) != GMM_OK) return s;
+    gmm_problem pp = *p;
+    pp.N = n_prep;
+    if ((s = tc_prep(&pp, w, mu, var, ws, T, st)) != GMM_OK) return s;
     int nslots = 0;
     if ((s = tc_pass<kTcStats>(p, X, ws, T, st, &nslots)) != GMM_OK) return s;
     tc_reduce_stats_kernel<<<blocks, 256, 0, st>>>(
@@ -335,10 +340,50 @@ gmm_status mstep_impl(const gmm_problem* p, const double* stats, int nshards, fl
   return launched(1);
 }
 
+// total[i] += part[i]: one chunk's statistics into the running total (chunk order).
+__global__ void __launch_bounds__(256) stats_add_kernel(double* __restrict__ total,
+                                                        const double* __restrict__ part, size_t n) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) total[i] += part[i];
+}
+
+// Device staging of gmm_em_step_host: two chunk buffers, then the running and
+// the per-chunk statistics.
+struct HostStaging {
+  size_t buf_bytes, stats_bytes, total;
+};
+
+HostStaging host_staging(const gmm_problem* p, int64_t chunk_rows) {
+  HostStaging H;
+  H.buf_bytes = align_up((size_t)chunk_rows * p->D * elem_bytes(p->xdtype), 256);
+  H.stats_bytes = align_up(stats_doubles(p) * 8, 256);
+  H.total = 2 * H.buf_bytes + 2 * H.stats_bytes;
+  return H;
+}
+
+// Events of one gmm_em_step_host call, destroyed on every way out (a pending
+// event is released once the work it marks has completed).
+struct StagingEvents {
+  cudaEvent_t copied[2] = {nullptr, nullptr}, used[2] = {nullptr, nullptr};
+  bool create() {
+    for (int b = 0; b < 2; ++b)
+      if (cudaEventCreateWithFlags(&copied[b], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&used[b], cudaEventDisableTiming) != cudaSuccess)
+        return false;
+    return true;
+  }
+  ~StagingEvents() {
+    for (int b = 0; b < 2; ++b) {
+      if (copied[b]) cudaEventDestroy(copied[b]);
+      if (used[b]) cudaEventDestroy(used[b]);
+    }
+  }
+};
+
 gmm_status em_step_impl(const gmm_problem* p, const void* X, float* w, float* mu, float* var,
                         double* loglik, void* ws_base, const Plan& P, cudaStream_t st) {
   double* stats = (double*)((char*)ws_base + P.stats);
-  gmm_status s = estep_stats_impl(p, X, w, mu, var, stats, ws_base, P, st);
+  gmm_status s = estep_stats_impl(p, X, w, mu, var, stats, ws_base, P, st, p->N);
   if (s != GMM_OK) return s;
   return mstep_impl(p, stats, 1, w, mu, var, loglik, st);
 }
@@ -471,7 +516,7 @@ gmm_status gmm_estep_stats(const gmm_problem* p, const void* X, const float* w, 
   if (!w || !mu || !var || !stats) return GMM_ERR_INVALID_ARG;
   Plan P;
   if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
-  return estep_stats_impl(p, X, w, mu, var, stats, ws, P, (cudaStream_t)stream);
+  return estep_stats_impl(p, X, w, mu, var, stats, ws, P, (cudaStream_t)stream, p->N);
 }
 
 gmm_status gmm_mstep(const gmm_problem* p, const double* stats, int32_t nshards, float* w,
@@ -606,6 +651,65 @@ gmm_status gmm_ivf_build(int64_t N, int32_t K, int32_t m, const int32_t* idx, co
   ivf_offsets_kernel<<<1, kIvfScanThreads, 0, st>>>(K, tot, offsets);
   ivf_walk(m, true, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
   return launched(4);
+}
+
+gmm_status gmm_host_staging_size(const gmm_problem* p, int64_t chunk_rows, size_t* bytes) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if (!bytes || chunk_rows < 1) return GMM_ERR_INVALID_ARG;
+  if ((size_t)chunk_rows > ((size_t)1 << 40)) return GMM_ERR_UNSUPPORTED;
+  *bytes = host_staging(p, chunk_rows).total;
+  return GMM_OK;
+}
+
+gmm_status gmm_em_step_host(const gmm_problem* p, const void* X_host, int64_t chunk_rows,
+                            void* staging, size_t staging_bytes, float* w, float* mu, float* var,
+                            double* loglik, void* ws, size_t ws_bytes, void* stream,
+                            void* copy_stream) {
+  size_t need = 0;
+  gmm_status s = gmm_host_staging_size(p, chunk_rows, &need);
+  if (s != GMM_OK) return s;
+  if (!X_host || !w || !mu || !var) return GMM_ERR_INVALID_ARG;
+  if (!staging || ((uintptr_t)staging) % 256 != 0 || staging_bytes < need)
+    return GMM_ERR_WORKSPACE;
+  if ((s = check_x(p, staging)) != GMM_OK) return s;
+  Plan P;
+  if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  const HostStaging H = host_staging(p, chunk_rows);
+  const size_t row_bytes = (size_t)p->D * elem_bytes(p->xdtype);
+  char* base = (char*)staging;
+  char* buf[2] = {base, base + H.buf_bytes};
+  double* total = (double*)(base + 2 * H.buf_bytes);
+  double* part = (double*)(base + 2 * H.buf_bytes + H.stats_bytes);
+  const size_t S = stats_doubles(p);
+  cudaStream_t st = (cudaStream_t)stream, cs = (cudaStream_t)copy_stream;
+  StagingEvents ev;
+  if (!ev.create()) return launch_status(), GMM_ERR_CUDA;
+  const char* xh = (const char*)X_host;
+  const int64_t nchunks = (p->N + chunk_rows - 1) / chunk_rows;
+  for (int64_t i = 0; i < nchunks; ++i) {
+    const int b = (int)(i & 1);
+    const int64_t r0 = i * chunk_rows;
+    gmm_problem pc = *p;
+    pc.N = std::min(chunk_rows, p->N - r0);
+    // the copy into buffer b waits until the E-step of chunk i - 2 has read it
+    if (i >= 2 && cudaStreamWaitEvent(cs, ev.used[b], 0) != cudaSuccess)
+      return launch_status(), GMM_ERR_CUDA;
+    if (cudaMemcpyAsync(buf[b], xh + (size_t)r0 * row_bytes, (size_t)pc.N * row_bytes,
+                        cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+        cudaEventRecord(ev.copied[b], cs) != cudaSuccess ||
+        cudaStreamWaitEvent(st, ev.copied[b], 0) != cudaSuccess)
+      return launch_status(), GMM_ERR_CUDA;
+    if ((s = estep_stats_impl(&pc, buf[b], w, mu, var, i == 0 ? total : part, ws, P, st,
+                              p->N)) != GMM_OK)
+      return s;
+    if (i > 0) {
+      stats_add_kernel<<<(unsigned)((S + 255) / 256), 256, 0, st>>>(total, part, S);
+      if ((s = launched(1)) != GMM_OK) return s;
+    }
+    if (cudaEventRecord(ev.used[b], st) != cudaSuccess) return launch_status(), GMM_ERR_CUDA;
+  }
+  return mstep_impl(p, total, 1, w, mu, var, loglik, st);
 }
 
 gmm_status gmm_launch_count(uint64_t* count) {

@@ -22,6 +22,7 @@ GMM_DEVFLAG_NONFINITE_X, GMM_DEVFLAG_BAD_PARAMS, GMM_DEVFLAG_WAIT_TIMEOUT = 0x1,
 GMM_DEVFLAG_X_RANGE, GMM_DEVFLAG_BAD_INDEX = 0x8, 0x10
 
 EXPORTS = ("gmm_workspace_size", "gmm_init", "gmm_em_step", "gmm_em_step_noalloc",
+           "gmm_host_staging_size", "gmm_em_step_host",
            "gmm_estep_stats", "gmm_mstep", "gmm_fit", "gmm_loglik",
            "gmm_assign_topm", "gmm_ivf_workspace_size", "gmm_ivf_build", "gmm_device_status",
            "gmm_trace_fused", "gmm_launch_count", "gmm_status_string")
@@ -56,6 +57,8 @@ def load_library(path: str = LIB_PATH):
     lib.gmm_init.argtypes = [PP, P, ctypes.POINTER(I64), I32, P, P, P, P, SZ, P]
     lib.gmm_em_step.argtypes = [PP, P, P, P, P, P, P, SZ, P]
     lib.gmm_em_step_noalloc.argtypes = [PP, P, P, P, P, P, P, P]
+    lib.gmm_host_staging_size.argtypes = [PP, I64, ctypes.POINTER(SZ)]
+    lib.gmm_em_step_host.argtypes = [PP, P, I64, P, SZ, P, P, P, P, P, SZ, P, P]
     lib.gmm_estep_stats.argtypes = [PP, P, P, P, P, P, P, SZ, P]
     lib.gmm_mstep.argtypes = [PP, P, I32, P, P, P, P, P]
     lib.gmm_fit.argtypes = [PP, P, I32, P, P, P, P, P, SZ, P]
@@ -146,6 +149,48 @@ def gmm_em_step(X, w, mu, var, loglik=None, var_floor=1e-6, ws=None, stream=None
     _check(load_library().gmm_em_step(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu), _ptr(var),
                                       _ptr(loglik), _ptr(ws), ws.numel(), _stream(stream)),
            "gmm_em_step")
+
+
+_copy_streams = {}
+
+
+def copy_stream_for(device):
+    """A side stream per device for gmm_em_step_host's host-to-device copies."""
+    key = torch.device(device).index if torch.device(device).index is not None else \
+        torch.cuda.current_device()
+    if key not in _copy_streams:
+        _copy_streams[key] = torch.cuda.Stream(device=key)
+    return _copy_streams[key]
+
+
+def gmm_host_staging_size(p: gmm_problem, chunk_rows) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().gmm_host_staging_size(ctypes.byref(p), int(chunk_rows),
+                                                ctypes.byref(n)), "gmm_host_staging_size")
+    return int(n.value)
+
+
+def gmm_em_step_host(X_host, w, mu, var, loglik=None, chunk_rows=1 << 18, var_floor=1e-6,
+                     staging=None, ws=None, stream=None, copy_stream=None):
+    """One EM iteration in place with X in host memory (pinned for overlap).
+
+    X_host: contiguous CPU tensor, float32 or bfloat16, N x D.  The rows are
+    copied chunk_rows at a time through device staging on copy_stream (default:
+    a side stream of the parameters' device) while the E-step runs on stream.
+    """
+    if X_host.is_cuda or not X_host.is_contiguous():
+        raise ValueError("X_host must be a contiguous host tensor")
+    p = problem_for(X_host, w.numel(), var_floor)
+    ws = _ws(p, ws, w.device)
+    if staging is None:
+        staging = torch.empty(gmm_host_staging_size(p, chunk_rows), dtype=torch.uint8,
+                              device=w.device)
+    cs = copy_stream_for(w.device) if copy_stream is None else copy_stream
+    _check(load_library().gmm_em_step_host(ctypes.byref(p), ctypes.c_void_p(X_host.data_ptr()),
+                                           int(chunk_rows), _ptr(staging), staging.numel(),
+                                           _ptr(w), _ptr(mu), _ptr(var), _ptr(loglik), _ptr(ws),
+                                           ws.numel(), _stream(stream), _stream(cs)),
+           "gmm_em_step_host")
 
 
 def stats_size(K, D) -> int:

@@ -30,6 +30,7 @@ def test_header_declares_the_calls():
     for n in ("gmm_init", "gmm_em_step", "gmm_em_step_noalloc", "gmm_estep_stats", "gmm_mstep",
               "gmm_fit", "gmm_loglik",
               "gmm_assign_topm", "gmm_ivf_workspace_size", "gmm_ivf_build",
+              "gmm_host_staging_size", "gmm_em_step_host",
               "gmm_workspace_size", "gmm_device_status", "gmm_trace_fused",
               "gmm_launch_count", "gmm_status_string"):
         assert n in names
@@ -167,3 +168,46 @@ def test_ivf_build_argument_checks(lib):
     assert call(ws=0) == G.GMM_ERR_WORKSPACE
     assert call(ws=128) == G.GMM_ERR_WORKSPACE
     assert call(ws_bytes=ok_ws - 1) == G.GMM_ERR_WORKSPACE
+
+
+def _staging(lib, p, rows):
+    n = ctypes.c_size_t(0)
+    rc = lib.gmm_host_staging_size(ctypes.byref(p), rows, ctypes.byref(n))
+    return rc, n.value
+
+
+def test_host_staging_size_is_two_chunks_and_two_stats_buffers(lib):
+    def up(x):
+        return (x + 255) // 256 * 256
+
+    for N, D, K, dt, rows in ((10**6, 128, 256, 0, 65_536), (10**8, 32, 1024, 1, 1 << 20),
+                              (7, 4, 3, 0, 3)):
+        p = G.problem(N, D, K, dt)
+        rc, n = _staging(lib, p, rows)
+        S = K * (2 * D + 1) + 1
+        assert rc == G.GMM_OK and n == 2 * up(rows * D * (2 if dt else 4)) + 2 * up(S * 8)
+    assert _staging(lib, G.problem(10, 4, 2), 0)[0] == G.GMM_ERR_INVALID_ARG
+    assert _staging(lib, G.problem(0, 4, 2), 5)[0] == G.GMM_ERR_INVALID_ARG
+    assert lib.gmm_host_staging_size(ctypes.byref(G.problem(10, 4, 2)), 5, None) == \
+        G.GMM_ERR_INVALID_ARG
+
+
+def test_em_step_host_argument_checks(lib):
+    P = ctypes.c_void_p
+    p = G.problem(100, 4, 2)
+    need = _staging(lib, p, 10)[1]
+
+    def call(X=16, rows=10, staging=256, sbytes=need, w=16):
+        return lib.gmm_em_step_host(ctypes.byref(p), P(X), rows, P(staging), sbytes, P(w), P(16),
+                                    P(16), P(0), P(256), 1 << 30, P(0), P(0))
+
+    assert call(X=0) == G.GMM_ERR_INVALID_ARG
+    assert call(w=0) == G.GMM_ERR_INVALID_ARG
+    assert call(rows=0) == G.GMM_ERR_INVALID_ARG
+    assert call(staging=0) == G.GMM_ERR_WORKSPACE
+    assert call(staging=128) == G.GMM_ERR_WORKSPACE
+    assert call(sbytes=need - 1) == G.GMM_ERR_WORKSPACE
+    bad = G.problem(100, 2, 2)  # 8-byte rows: not a legal row pitch for the staged copy
+    assert lib.gmm_em_step_host(ctypes.byref(bad), P(16), 10, P(256), 1 << 20, P(16), P(16),
+                                P(16), P(0), P(256), 1 << 30, P(0), P(0)) == \
+        G.GMM_ERR_UNSUPPORTED
