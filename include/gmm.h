@@ -281,7 +281,8 @@ gmm_status gmm_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* 
  * records start_event on its stream just before that kernel's launch and
  * stop_event just after it, so the kernel's own duration can be read with
  * cudaEventElapsedTime.  Passing NULL, NULL turns it off.  The setting is
- * process-wide and not synchronised between host threads.
+ * process-wide; each handle is read and written atomically, but the pair is not
+ * swapped as one, so change it while no other host thread is launching.
  */
 gmm_status gmm_trace_fused(void* start_event, void* stop_event);
 

@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -97,7 +98,7 @@ gmm_status get_plan(const gmm_problem* p, void* ws, size_t ws_bytes, Plan* P) {
   return GMM_OK;
 }
 
-unsigned long long g_launches = 0;  // kernels enqueued by this library
+std::atomic<unsigned long long> g_launches{0};  // kernels enqueued by this library, all threads
 
 gmm_status launch_status() {
   cudaError_t e = cudaGetLastError();
@@ -108,13 +109,13 @@ gmm_status launch_status() {
   return GMM_OK;
 }
 
-cudaEvent_t g_trace_start = nullptr, g_trace_stop = nullptr;
+std::atomic<cudaEvent_t> g_trace_start{nullptr}, g_trace_stop{nullptr};
 
 void trace_begin(cudaStream_t st) {
-  if (g_trace_start) cudaEventRecord(g_trace_start, st);
+  if (cudaEvent_t e = g_trace_start.load()) cudaEventRecord(e, st);
 }
 void trace_end(cudaStream_t st) {
-  if (g_trace_stop) cudaEventRecord(g_trace_stop, st);
+  if (cudaEvent_t e = g_trace_stop.load()) cudaEventRecord(e, st);
 }
 
 // Status after enqueuing n kernels (counted for gmm_launch_count).
@@ -714,7 +715,7 @@ gmm_status gmm_em_step_host(const gmm_problem* p, const void* X_host, int64_t ch
 
 gmm_status gmm_launch_count(uint64_t* count) {
   if (!count) return GMM_ERR_INVALID_ARG;
-  *count = g_launches;
+  *count = g_launches.load();
   return GMM_OK;
 }
 
