@@ -141,3 +141,28 @@ def test_stored_traffic_is_used_only_for_the_source_it_was_measured_on(monkeypat
     assert bench.ncu_traffic("bf16stream") is None
     monkeypatch.setattr(bench, "fused_source_sha", lambda: "0" * 16)
     assert bench.ncu_traffic("uint8img") is None
+
+
+def test_reference_arm_prints_one_contract_line():
+    import subprocess
+    import sys
+
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+           "--workload", "gauss8", "--steps", "2", "--warmup", "1"]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=300, check=True,
+                         env={**os.environ, "RANK": "0"})
+    lines = [ln for ln in out.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["value"] > 0
+    assert d["config"]["workload"] == "gauss8"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["cpu_baseline"]["cores"] >= 1
+    # ranks other than 0 print nothing and exit 0
+    quiet = subprocess.run(cmd, capture_output=True, text=True, timeout=120, check=True,
+                           env={**os.environ, "RANK": "1"})
+    assert quiet.stdout.strip() == ""
