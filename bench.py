@@ -308,56 +308,86 @@ def ours(args):
     if rc != 0:
         raise SystemExit(f"device status {G.status_string(rc)} flags={flags:#x}")
 
-    # ---- end to end: X and parameters from pinned host memory every step ----
-    # Each step's X is copied host -> device on a copy stream into one of two
-    # device buffers while the previous step computes (as a pipeline feeding the
-    # library would); the timed region spans every copy, every step and every
-    # read-back of the results.
-    w_h = theta0[0].cpu().pin_memory()
-    mu_h = theta0[1].cpu().pin_memory()
-    var_h = theta0[2].cpu().pin_memory()
-    ll_h = torch.zeros(1, dtype=torch.float64).pin_memory()
-    xbuf = [torch.empty_like(Xd), torch.empty_like(Xd)]
-    cstream = torch.cuda.Stream(dev)
-    copied = [torch.cuda.Event(), torch.cuda.Event()]
-    used = [torch.cuda.Event(), torch.cuda.Event()]
+    # ---- end to end: X from pinned host memory every step -------------------
+    # One GPU: the public call for host-resident data, gmm_em_step_host. Every
+    # step streams all of X over PCIe in chunks (copy stream), overlapping the
+    # previous chunk's E-step, and the step's LL is read back to pinned host
+    # memory. Several GPUs: each rank's step is gmm_estep_stats + all-gather +
+    # gmm_mstep, so X and the parameters are copied per step on a copy stream
+    # into one of two device buffers, overlapping the previous step.
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-
-    def issue_copy(i):
-        b = i % 2
-        if i >= 2:
-            cstream.wait_event(used[b])  # the step that read this buffer is done
-        with torch.cuda.stream(cstream):
-            xbuf[b].copy_(Xh, non_blocking=True)
-        copied[b].record(cstream)
-
-    barrier()
-    torch.cuda.synchronize(dev)
-    e0.record(stream)
-    cstream.wait_event(e0)
-    issue_copy(0)
-    for i in range(args.steps):
-        b = i % 2
-        if i + 1 < args.steps:
-            issue_copy(i + 1)
-        stream.wait_event(copied[b])
-        w.copy_(w_h, non_blocking=True)
-        mu.copy_(mu_h, non_blocking=True)
-        var.copy_(var_h, non_blocking=True)
-        step(xbuf[b])
-        used[b].record(stream)
-        w_h.copy_(w, non_blocking=True)
-        mu_h.copy_(mu, non_blocking=True)
-        var_h.copy_(var, non_blocking=True)
-        ll_h.copy_(ll, non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
     pbytes = (w.numel() + mu.numel() + var.numel()) * 4
-    h2d = (Xd.numel() * Xd.element_size() + pbytes) * world
-    d2h = (pbytes + 8) * world
+    if world == 1:
+        chunk_rows = min(N, args.chunk_rows)
+        staging = torch.empty(G.gmm_host_staging_size(p, chunk_rows), dtype=torch.uint8,
+                              device=dev)
+        cs = G.copy_stream_for(dev)
+        ll_hist = torch.zeros(args.steps, dtype=torch.float64).pin_memory()
+        G.gmm_em_step_host(Xh, w, mu, var, ll, chunk_rows, wl.var_floor, staging=staging,
+                           ws=ws)  # warm-up, untimed
+        for t, t0 in zip((w, mu, var), theta0):
+            t.copy_(t0)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        cs.wait_event(e0)
+        for i in range(args.steps):
+            G.gmm_em_step_host(Xh, w, mu, var, ll, chunk_rows, wl.var_floor, staging=staging,
+                               ws=ws)
+            ll_hist[i].copy_(ll[0], non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / args.steps
+        h2d = Xh.numel() * Xh.element_size()
+        d2h = 8
+        pipeline = (f"gmm_em_step_host: X streamed from pinned host memory in chunks of "
+                    f"{chunk_rows} rows on a copy stream, overlapping the E-step; LL read back")
+    else:
+        w_h = theta0[0].cpu().pin_memory()
+        mu_h = theta0[1].cpu().pin_memory()
+        var_h = theta0[2].cpu().pin_memory()
+        ll_h = torch.zeros(1, dtype=torch.float64).pin_memory()
+        xbuf = [torch.empty_like(Xd), torch.empty_like(Xd)]
+        cstream = torch.cuda.Stream(dev)
+        copied = [torch.cuda.Event(), torch.cuda.Event()]
+        used = [torch.cuda.Event(), torch.cuda.Event()]
+
+        def issue_copy(i):
+            b = i % 2
+            if i >= 2:
+                cstream.wait_event(used[b])  # the step that read this buffer is done
+            with torch.cuda.stream(cstream):
+                xbuf[b].copy_(Xh, non_blocking=True)
+            copied[b].record(cstream)
+
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        cstream.wait_event(e0)
+        issue_copy(0)
+        for i in range(args.steps):
+            b = i % 2
+            if i + 1 < args.steps:
+                issue_copy(i + 1)
+            stream.wait_event(copied[b])
+            w.copy_(w_h, non_blocking=True)
+            mu.copy_(mu_h, non_blocking=True)
+            var.copy_(var_h, non_blocking=True)
+            step(xbuf[b])
+            used[b].record(stream)
+            w_h.copy_(w, non_blocking=True)
+            mu_h.copy_(mu, non_blocking=True)
+            var_h.copy_(var, non_blocking=True)
+            ll_h.copy_(ll, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.steps
+        h2d = (Xd.numel() * Xd.element_size() + pbytes) * world
+        d2h = (pbytes + 8) * world
+        pipeline = ("each step's X and parameters copied from pinned host memory on a second "
+                    "stream, double-buffered, overlapping the previous step; parameters and LL "
+                    "read back")
 
     ms = total_ms / args.steps
     # whole-job throughput in workload iterations: rows of all ranks per second / workload N
@@ -390,9 +420,7 @@ def ours(args):
                                     f"{'sustained' if sustained else 'burst'} "
                                     "(fp16 runs at the bf16 rate)"},
         "e2e": {"value": (N_total / wl.N) * 1e3 / e2e_ms, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h,
-                "pipeline": "each step's X copied from pinned host memory on a second stream, "
-                            "double-buffered, overlapping the previous step"},
+                "d2h_bytes_per_step": d2h, "pipeline": pipeline},
         "gpu_launches": launches,
         "clocks": clocks,
     }
