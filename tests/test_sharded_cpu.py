@@ -1,8 +1,8 @@
-"""Row-sharded EM orchestration on CPU: two gloo ranks, statistics from the oracle.
+"""Row-sharded EM orchestration on CPU: two and three gloo ranks, statistics from the oracle.
 
 Each rank computes the fp64 statistics of its contiguous block of rows with the
 oracle, the ranks all-gather them (soft_clustering_em_b200.sharded), and every
-rank applies the M-step to the rank-ordered sum.  After three iterations both
+rank applies the M-step to the rank-ordered sum.  After three iterations all
 ranks must hold identical parameters, equal (to fp64 rounding) to the oracle run
 on all rows in one process.  This covers the host logic of the multi-GPU path;
 on GPUs the same orchestration runs with gmm_estep_stats / gmm_mstep and NCCL.
@@ -78,23 +78,25 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_rank_sharded_em_matches_single_process(oracle_mod):
+@pytest.mark.parametrize("world", [2, 3])  # 3001 rows: shards of 1000/1000/1001 at world 3
+def test_sharded_em_matches_single_process(oracle_mod, world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     out = {}
-    for _ in range(2):
+    for _ in range(world):
         r, w, mu, var, ll = q.get(timeout=240)
         out[r] = (w, mu, var, ll)
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    # identical on both ranks
-    for a, b in zip(out[0], out[1]):
-        np.testing.assert_array_equal(np.asarray(a), np.asarray(b))
+    # identical on every rank
+    for r in range(1, world):
+        for a, b in zip(out[0], out[r]):
+            np.testing.assert_array_equal(np.asarray(a), np.asarray(b))
     # equal to one process over all rows
     wl, X = _data()
     from soft_clustering_em_b200 import synth
