@@ -166,3 +166,31 @@ def test_reference_arm_prints_one_contract_line():
     quiet = subprocess.run(cmd, capture_output=True, text=True, timeout=120, check=True,
                            env={**os.environ, "RANK": "1"})
     assert quiet.stdout.strip() == ""
+
+
+def test_tensor_core_shape_limits_and_f_buffers(tmp_path):
+    """The tensor-core kernel's shape rule and F-buffer choice, from the host-side
+    layout code itself (compiled for the host with nvcc; no device needed)."""
+    import subprocess
+
+    nvcc = "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    exe = str(tmp_path / "tc_layout_check")
+    subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O1", "-std=c++17",
+                    "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include"),
+                    "-I", os.path.join(ROOT, "soft_clustering_em_b200", "csrc"), "-o", exe,
+                    os.path.join(ROOT, "tests", "csrc", "tc_layout_check.cu")],
+                   check=True, capture_output=True, timeout=600)
+    rows = [list(map(int, ln.split())) for ln in
+            subprocess.run([exe], check=True, capture_output=True, text=True).stdout.split("\n")
+            if ln.strip()]
+    assert [r[0] for r in rows] == list(range(4, 129, 4))
+    for D, maxk, nfb256, nfb1024, nfbmax in rows:
+        assert maxk == (2048 if D <= 64 else 1280 if D <= 96 else 256), D
+        if D <= 32:  # two F buffers at every K
+            assert (nfb256, nfb1024, nfbmax) == (2, 2, 2), D
+        elif D <= 64:  # two only at small K, where the cluster is small enough
+            assert (nfb256, nfb1024, nfbmax) == (2, 1, 1), D
+        else:
+            assert nfb256 == 1 and nfbmax == 1 and nfb1024 == (1 if D <= 96 else 0), D
