@@ -211,3 +211,35 @@ def test_em_step_host_argument_checks(lib):
     assert lib.gmm_em_step_host(ctypes.byref(bad), P(16), 10, P(256), 1 << 20, P(16), P(16),
                                 P(16), P(0), P(256), 1 << 30, P(0), P(0)) == \
         G.GMM_ERR_UNSUPPORTED
+
+
+def test_header_is_plain_c99_and_the_c_example_links(lib, tmp_path):
+    """include/gmm.h compiles as pedantic C99, and a plain C program using the
+    ABI builds, links and runs: without a device it reports GMM_ERR_CUDA cleanly."""
+    import shutil
+    import subprocess
+
+    import torch
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    inc = os.path.join(ROOT, "include")
+    hdr = tmp_path / "hdr.c"
+    hdr.write_text('#include "gmm.h"\nint main(void) { return gmm_status_string(GMM_OK) == 0; }\n')
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", inc, "-c",
+                    str(hdr), "-o", str(tmp_path / "hdr.o")], check=True, capture_output=True)
+    cuda = "/usr/local/cuda"
+    libdir = os.path.dirname(G.LIB_PATH)
+    exe = str(tmp_path / "c_abi_example")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", inc, "-I",
+                    os.path.join(cuda, "include"), "-o", exe,
+                    os.path.join(ROOT, "tests", "csrc", "c_abi_example.c"), "-L", libdir,
+                    "-lscem_gmm", "-L", os.path.join(cuda, "lib64"), "-lcudart",
+                    "-Wl,-rpath," + libdir, "-Wl,-rpath," + os.path.join(cuda, "lib64")],
+                   check=True, capture_output=True)
+    out = subprocess.run([exe], capture_output=True, text=True, timeout=300)
+    if torch.cuda.is_available():
+        assert out.returncode == 0 and out.stdout.startswith("LL(theta_9)"), out.stdout
+    else:
+        assert out.returncode == 0 and "GMM_ERR_CUDA" in out.stdout, out.stdout
