@@ -103,7 +103,10 @@ gmm_status gmm_workspace_size(const gmm_problem* p, size_t* bytes);
  * [0, N)), w_k = 1/K, and var = 1 (GMM_INIT_VAR_ONE) or the per-dimension
  * biased sample variance of X, max(., var_floor), for every component
  * (GMM_INIT_VAR_DATA).  Writes w, mu, var.  The review page (section 3) gives
- * no initialisation; this one is the library's definition.
+ * no initialisation; this one is the library's definition.  The indices are
+ * copied to the workspace on `stream`: from pageable memory the copy has read
+ * them when the call returns; from pinned (page-locked) memory the array must
+ * stay unchanged until the stream has reached this call.
  */
 gmm_status gmm_init(const gmm_problem* p, const void* X, const int64_t* rows_host,
                     int32_t init_var, float* w, float* mu, float* var, void* ws,
