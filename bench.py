@@ -41,6 +41,9 @@ from soft_clustering_em_b200 import synth  # noqa: E402
 METRIC = "EM iterations/s and fused E+M N·K·D/s on 1 B200, % of roofline"
 UNIT = "EM iterations/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# N*K exponentials at 16 MUFU ex2 per clock per SM, 148 SMs, 1965 MHz: a floor
+# for the normalisation, reported beside the tensor roofline
+MUFU_EXP_PER_S = 16 * 148 * 1.965e9
 FUSED_SOURCES = ["soft_clustering_em_b200/csrc/tc_em.cuh",
                  "soft_clustering_em_b200/csrc/sm100_prims.cuh",
                  "soft_clustering_em_b200/csrc/common.cuh"]
@@ -416,6 +419,8 @@ def ours(args):
                      "kernel": "fused E-step + statistics pass (tc_fused_kernel)",
                      "algorithmic": "8*N*K*D flop per launch",
                      "fused_ms_per_launch": fused_avg,
+                     "frac_vs_tf32_dense": achieved / (peak / 2.0),
+                     "mufu_exp_floor_ms": N * wl.K / MUFU_EXP_PER_S * 1e3,
                      "peak_source": f"{pk_kind} bf16 dense "
                                     f"{'sustained' if sustained else 'burst'} "
                                     "(fp16 runs at the bf16 rate)"},
