@@ -144,6 +144,14 @@ def init(X, rows, K, var_mode, var_floor=1e-6):
     return w, mu, var
 
 
+def init_seeded(X, seed, K, var_mode, var_floor=1e-6):
+    """init() at the K rows the library's gmm_init picks from `seed`
+    (SplitMix64-driven Floyd sampling, oracle/sampling.py)."""
+    from .sampling import floyd_rows
+
+    return init(X, floyd_rows(len(X), K, seed), K, var_mode, var_floor)
+
+
 def fit(X, w, mu, var, iters, var_floor=1e-6):
     """iters EM steps; returns (w, mu, var, ll_history) with ll[t] = LL(theta_t)."""
     X, w, mu, var, N, D, K = _shapes(X, w, mu, var)

@@ -23,6 +23,7 @@ REL = 1e-3
 LL_REL = 1e-4
 MIN_NK = 10.0
 TOPM_GAP = 1e-5
+W_ABS = 1e-9
 
 
 def compare_step(ref, got, Nk_ref, N=None):
@@ -35,12 +36,16 @@ def compare_step(ref, got, Nk_ref, N=None):
     gate = Nk_ref >= MIN_NK
     N = float(Nk_ref.sum()) if N is None else float(N)
     rw = np.abs(w_g - w_r) / (REL * np.maximum(w_r, MIN_NK / max(N, 1.0)))
+    # the plain reading of "relative 1e-3 on weights": 1e-3 pi_ref + 1e-9
+    rw_plain = np.abs(w_g - w_r) / (REL * w_r + W_ABS)
     scale_mu = REL * np.maximum(np.abs(mu_r), np.sqrt(var_r))
     rmu = np.abs(mu_g - mu_r) / scale_mu
     rvar = np.abs(var_g - var_r) / (REL * var_r)
     rll = abs(float(ll_g) - float(ll_r)) / (LL_REL * abs(float(ll_r)))
     out = {
         "w": float(rw.max()),
+        "w_plain": float(rw_plain.max()),
+        "w_plain_worst_k": int(np.argmax(rw_plain)),
         "mu": float(rmu[gate].max()) if gate.any() else 0.0,
         "var": float(rvar[gate].max()) if gate.any() else 0.0,
         "ll": rll,
