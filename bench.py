@@ -4,13 +4,14 @@
 One step = one full EM iteration through the C ABI (gmm_em_step: parameter
 prep, the fused E-step + statistics pass over all N rows, the deterministic
 reduction and the M-step) on the resident synthetic workload.  Default
-workload: uint8img (N=1e6, D=128, K=256, fp32 X), the configuration the
-throughput metric is quoted on.
+workload: gauss4096 (N=1e7, D=96, K=4096, fp32 X), the largest single-GPU
+configuration by N*K*D; --workload picks any of the five.
 
 Prints ONE JSON line (rank 0).  Timing: W untimed warm-up steps, then exactly
 K steps between a barrier + synchronize on both sides, timed with CUDA events
-on the stream the library launches on; X (512 MB) is larger than the 126 MB
-L2, so no flush is needed between steps.
+on the stream the library launches on; X (3.84 GB for gauss4096) is larger than
+the 126 MB L2, so no flush is needed between steps (a 256 MB buffer is zeroed
+between steps for the one workload, gauss8, whose X fits in L2).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -52,10 +53,10 @@ FUSED_SOURCES = ["soft_clustering_em_b200/csrc/tc_em.cuh",
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="uint8img", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default="gauss4096", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--rows", type=int, default=0, help="override N (0: the workload's N)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -75,6 +76,34 @@ def peaks():
         d = json.load(open(path))
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def measure_tf32_tflops(dev):
+    """Dense TF32 rate of this GPU: torch fp32 matmul with TF32 allowed, 8192^3,
+    best of 10 after warm-up, CUDA events (the survey's planned measurement)."""
+    import torch
+
+    n = 8192
+    a = torch.randn(n, n, device=dev)
+    b = torch.randn(n, n, device=dev)
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = True
+    try:
+        for _ in range(3):
+            torch.matmul(a, b)
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch.matmul(a, b)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            best = min(best, e0.elapsed_time(e1))
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
+    del a, b
+    torch.cuda.empty_cache()
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
 
 
 def fused_source_sha():
@@ -191,9 +220,8 @@ def reference_arm(args):
     wl = synth.WORKLOADS[args.workload]
     N = args.rows or wl.N
     X_np, _ = synth.make_data(wl, N)
-    rows = synth.init_rows(N, wl.K, wl.init_seed)
     mode = 0 if wl.var_init == "one" else 1
-    theta = oracle.init(synth.x_as_f64(wl, X_np), rows, wl.K, mode, wl.var_floor)
+    theta = oracle.init_seeded(synth.x_as_f64(wl, X_np), wl.init_seed, wl.K, mode, wl.var_floor)
     per_step = min(10.0, 150.0 / max(1, args.steps + args.warmup))
     n = size_sample(wl, X_np, theta, per_step)
     for _ in range(args.warmup):
@@ -245,9 +273,8 @@ def ours(args):
     Xd = Xh.to(dev, non_blocking=False)
     p = G.problem_for(Xd, wl.K, wl.var_floor)
     ws = G.workspace(p, dev)
-    rows = synth.init_rows(N, wl.K, wl.init_seed)
     mode = G.GMM_INIT_VAR_ONE if wl.var_init == "one" else G.GMM_INIT_VAR_DATA
-    w, mu, var = G.gmm_init(Xd, rows, wl.K, mode, wl.var_floor, ws=ws)
+    w, mu, var = G.gmm_init(Xd, wl.init_seed, wl.K, mode, wl.var_floor, ws=ws)
     if world > 1:
         sharded.broadcast_params(w, mu, var)  # every rank starts from rank 0's parameters
     ll = torch.zeros(1, dtype=torch.float64, device=dev)
@@ -258,8 +285,15 @@ def ours(args):
     stats = torch.empty(G.stats_size(wl.K, wl.D), dtype=torch.float64, device=dev)
     xdt = G.xdtype_of(Xd)
 
+    plan = G.gmm_plan(p)
+    # a problem whose fit runs in one launch is timed as gmm_fit over the
+    # workload's iterations per step; every other as one gmm_em_step per step
+    iters_per_step = wl.iters if (world == 1 and plan["fit_one_launch"]) else 1
+
     def step(X):
-        if world == 1:
+        if iters_per_step > 1:
+            G.gmm_fit(X, w, mu, var, iters_per_step, wl.var_floor, ws=ws)
+        elif world == 1:
             G.gmm_em_step(X, w, mu, var, ll, wl.var_floor, ws=ws)
         else:
             G.gmm_estep_stats(X, w, mu, var, stats, wl.var_floor, ws=ws)
@@ -277,6 +311,7 @@ def ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
+    tf32 = measure_tf32_tflops(dev) if rank == 0 else None
     props = torch.cuda.get_device_properties(dev)
     sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else None)
     time.sleep(0.5)
@@ -394,8 +429,8 @@ def ours(args):
 
     ms = total_ms / args.steps
     # whole-job throughput in workload iterations: rows of all ranks per second / workload N
-    value = (N_total / wl.N) * 1e3 / ms
-    nkd = float(N) * wl.K * wl.D
+    value = (N_total / wl.N) * iters_per_step * 1e3 / ms
+    nkd = float(N) * wl.K * wl.D * iters_per_step  # per timed step (and per fused launch)
     pk, pk_kind = peaks()
     sustained = total_ms >= 1000.0
     peak = pk["bf16_tflops_sustained" if sustained else "bf16_tflops"]
@@ -403,23 +438,45 @@ def ours(args):
     achieved = 8.0 * nkd / (fused_avg * 1e-3) / 1e12
     traffic = ncu_traffic(wl.name)
     cfg = workload_config(wl, N)
+    cfg["em_iters_per_timed_step"] = iters_per_step
     if world > 1:
         cfg.update({"ranks": world, "rows_per_rank": N, "exchange": "NCCL all-gather of fp64 "
                     "statistics, M-step sums shards in rank order"})
+    if iters_per_step > 1:
+        dtype = "f32"
+        precision = ("fp32 direct form on the CUDA cores, fp64 statistics exchanged over "
+                     "distributed shared memory, M-step on chip")
+        kernel = (f"small_fit_kernel: all {iters_per_step} iterations of gmm_fit in one launch "
+                  "of one cluster, X resident in shared memory")
+    elif plan["tensor_cores"]:
+        dtype = "f16"
+        precision = ("fp16 hi/lo split operands on the tensor cores (tcgen05 kind::f16), fp32 "
+                     "accumulation in tensor memory, fp64 reductions and M-step")
+        if plan["groups"] == 1:
+            kernel = (f"tc_fused_kernel: one fused pass, {plan['cluster_ctas']}-CTA clusters "
+                      "exchanging each row's (max, sum-exp) over DSMEM")
+        else:
+            kernel = (f"tc_fused_kernel, {plan['groups']} component groups of "
+                      f"{plan['cluster_ctas']}-CTA clusters: per chunk of "
+                      f"{plan['chunk_rows']} rows tc_convert_kernel (features to HBM), the "
+                      "partial (max, sum-exp) pass and the statistics pass, features TMA-loaded")
+    else:
+        dtype = "f32"
+        precision = "fp32 direct form on the CUDA cores, fp64 reductions and M-step"
+        kernel = "simt_fused_kernel (CUDA cores, direct form; the shape has no tensor-core plan)"
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f16",
-        "precision": "fp16 hi/lo split operands on the tensor cores, fp32 accumulation, "
-                     "fp64 reductions and M-step",
+        "vs_baseline": None, "dtype": dtype, "precision": precision,
         "data": "synthetic", "config": cfg,
         "nkd_per_s": nkd * world * 1e3 / ms,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "fused E-step + statistics pass (tc_fused_kernel)",
-                     "algorithmic": "8*N*K*D flop per launch",
+                     "kernel": kernel, "plan": plan,
+                     "algorithmic": "8*N*K*D flop per fused pass (all its launches)",
                      "fused_ms_per_launch": fused_avg,
-                     "frac_vs_tf32_dense": achieved / (peak / 2.0),
+                     "tf32_tflops_measured": tf32,
+                     "frac_vs_tf32_measured": achieved / tf32 if tf32 else None,
                      "mufu_exp_floor_ms": N * wl.K / MUFU_EXP_PER_S * 1e3,
                      "peak_source": f"{pk_kind} bf16 dense "
                                     f"{'sustained' if sustained else 'burst'} "
@@ -549,7 +606,7 @@ def host_stream_bench(args):
     mode = G.GMM_INIT_VAR_ONE if wl.var_init == "one" else G.GMM_INIT_VAR_DATA
     p = G.problem_for(Xh, wl.K, wl.var_floor)
     ws = G.workspace(p, dev)
-    w, mu, var = G.gmm_init(Xd, synth.init_rows(N, wl.K, wl.init_seed), wl.K, mode,
+    w, mu, var = G.gmm_init(Xd, wl.init_seed, wl.K, mode,
                             wl.var_floor, ws=ws)
     del Xd  # from here on X lives only in host memory
     torch.cuda.empty_cache()

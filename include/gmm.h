@@ -89,6 +89,23 @@ typedef struct {
 #define GMM_DEVFLAG_BAD_INDEX 0x10u      /* gmm_ivf_build: a component index outside [0, K)
                                             or repeated within one point's row */
 
+/* How the library runs a problem on the current device (see gmm_plan). */
+typedef struct {
+  int32_t tensor_cores; /* 1: the tcgen05 tensor-core kernel; 0: the CUDA-core kernel
+                           (D > 128, D not a multiple of 4, or no cluster shape fits) */
+  int32_t cluster_ctas; /* tensor cores: CTAs per thread-block cluster, 128 components each */
+  int32_t groups;       /* tensor cores: component groups.  1: one fused pass, the row
+                           normalisation exchanged inside the cluster.  > 1: per chunk of
+                           rows, a pass that writes each group's (max, sum-exp) per row
+                           to a row buffer, then the statistics pass */
+  int32_t fit_one_launch; /* 1: gmm_fit runs all its iterations in one launch of one
+                             cluster, X held in the cluster's shared memory (small N * D) */
+  int64_t chunk_rows;   /* groups > 1: rows per chunk (fixed by D and K, not by N), else 0 */
+} gmm_plan_info;
+
+/* Fills *info for problem p on the current device.  Errors as gmm_workspace_size. */
+gmm_status gmm_plan(const gmm_problem* p, gmm_plan_info* info);
+
 /*
  * Bytes of device workspace needed for problem p on the CURRENT device.
  * The value depends on (D, K, xdtype) and the device's SM count only: it is
@@ -98,19 +115,36 @@ typedef struct {
 gmm_status gmm_workspace_size(const gmm_problem* p, size_t* bytes);
 
 /*
- * Initial parameters.  mu_k = X[rows_host[k]] (K row indices chosen by the
- * caller, e.g. uniformly without replacement; HOST array of K int64 in
- * [0, N)), w_k = 1/K, and var = 1 (GMM_INIT_VAR_ONE) or the per-dimension
- * biased sample variance of X, max(., var_floor), for every component
- * (GMM_INIT_VAR_DATA).  Writes w, mu, var.  The review page (section 3) gives
- * no initialisation; this one is the library's definition.  The indices are
- * copied to the workspace on `stream`: from pageable memory the copy has read
- * them when the call returns; from pinned (page-locked) memory the array must
- * stay unchanged until the stream has reached this call.
+ * Initial parameters from a seed.  The review page (section 3) gives no
+ * initialisation; this one is the library's definition.  mu_k = X[row_k] for
+ * K distinct rows drawn uniformly without replacement (requires K <= N),
+ * w_k = 1/K, and var = 1 (GMM_INIT_VAR_ONE) or the per-dimension biased sample
+ * variance of X, max(., var_floor), for every component (GMM_INIT_VAR_DATA).
+ * Writes w, mu, var.
+ *
+ * The rows are chosen on the host, reproducibly from `seed`: Floyd's sampling
+ * algorithm (for j = N-K .. N-1: t uniform in [0, j]; take t, or j if t was
+ * taken; row_k is the index taken at step k) drawing its uniform integers from
+ * SplitMix64 (Steele, Lea and Flood, OOPSLA 2014) started at state `seed`,
+ * output i = mix(seed + (i+1) * 0x9E3779B97F4A7C15); an output x gives
+ * x mod n when x < 2^64 - (2^64 mod n) and is redrawn otherwise.  Any other
+ * implementation of these two published definitions picks the same rows.
+ * Errors: as gmm_em_step, plus GMM_ERR_INVALID_ARG for K > N or a bad
+ * init_var.
  */
-gmm_status gmm_init(const gmm_problem* p, const void* X, const int64_t* rows_host,
-                    int32_t init_var, float* w, float* mu, float* var, void* ws,
-                    size_t ws_bytes, void* stream);
+gmm_status gmm_init(const gmm_problem* p, const void* X, uint64_t seed, int32_t init_var,
+                    float* w, float* mu, float* var, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * gmm_init with the K rows chosen by the caller: mu_k = X[rows_host[k]] (HOST
+ * array of K int64 in [0, N); repeats allowed), the rest as gmm_init.  The
+ * indices are copied to the workspace on `stream`: from pageable memory the
+ * copy has read them when the call returns; from pinned (page-locked) memory
+ * the array must stay unchanged until the stream has reached this call.
+ */
+gmm_status gmm_init_rows(const gmm_problem* p, const void* X, const int64_t* rows_host,
+                         int32_t init_var, float* w, float* mu, float* var, void* ws,
+                         size_t ws_bytes, void* stream);
 
 /*
  * One fused EM iteration, in place: (w, mu, var) <- M-step(E-step(X; w, mu, var)).
@@ -158,13 +192,18 @@ gmm_status gmm_mstep(const gmm_problem* p, const double* stats, int32_t nshards,
  * Scratch: a fixed 32 MiB array compiled into this library, present on every
  * device that loads the library until the process exits.  The first call on a
  * device looks up that array's device address (cudaGetSymbolAddress) and
- * caches it; make that first call before any stream capture.  When the
- * statistics slots of the regular workspace do not all fit, fewer CTAs (or
- * clusters) run the fused pass, one slot each, which is slower but gives the
- * same result up to summation order.  A tensor-core slot holds K*(4D+1)+1
- * doubles; when not even one fits next to the parameter tables, the call runs
- * the CUDA-core kernel, whose slot holds K*(2D+1)+1.  A problem for which not
- * even that fits is rejected with GMM_ERR_UNSUPPORTED and a message on stderr.
+ * caches it with the CUDA context that was current; a later call under
+ * another context (one created after cudaDeviceReset, or a non-primary driver
+ * context) looks it up again.  Make the first call on each device and context
+ * before any stream capture.  When the statistics slots of the regular
+ * workspace do not all fit, fewer CTAs (or clusters) run the fused pass, one
+ * slot each, which is slower but gives the same result up to summation order.
+ * A tensor-core slot holds K*(2D+1)+1 doubles beside the parameter tables;
+ * when not even one fits (and for shapes whose tensor-core plan has more than
+ * one component group, whose row-chunk buffers exceed the scratch), the call
+ * runs the CUDA-core kernel, whose slot holds K*(2D+1)+1.  A problem for which
+ * not even that fits is rejected with GMM_ERR_UNSUPPORTED and a message on
+ * stderr.
  *
  * Every call on a device uses the same array and it keeps the previous call's
  * contents; each call resets the status word and rewrites everything else it
@@ -178,9 +217,53 @@ gmm_status gmm_em_step_noalloc(const gmm_problem* p, const void* X, float* w, fl
                                float* var, double* loglik, uint32_t* dev_flags, void* stream);
 
 /*
+ * Neighbours of the diagonal EM step (the pages present the soft mixture as a
+ * replacement for k-means in an IVF coarse quantizer; they print none of
+ * these, so each is the textbook form).  All three run the same fused
+ * tensor-core E-step and statistics pass as gmm_em_step and take its
+ * workspace (gmm_workspace_size).
+ *
+ * gmm_em_step_hard: classification EM of the diagonal model.  Each point goes
+ * wholly to its most probable component (largest log-joint, ties to the lower
+ * index); the M-step is gmm_em_step's with those 0/1 responsibilities.
+ * labels (device, N int32, may be NULL) receives each point's component;
+ * loglik (may be NULL) the classification log-likelihood of the input
+ * parameters, sum_n max_k log(pi_k N(x_n | k)).  The decision is made on the
+ * tensor-core log-joints: points whose two best components lie within about
+ * 1e-3 nats may go to either.  GMM_ERR_UNSUPPORTED for shapes without a
+ * tensor-core plan (gmm_plan).
+ *
+ * gmm_em_step_spherical: soft EM with covariance s2_k * I: s2 is K floats
+ * (device, in place); the M-step variance is the mean over dimensions of the
+ * per-dimension variance about the new mean, floored at var_floor.  Any
+ * shape gmm_em_step takes.
+ *
+ * gmm_kmeans_step: one Lloyd step.  centers (device, K x D, in place) move to
+ * the mean of their points (a centre with no point stays); labels (may be
+ * NULL) gets each point's nearest centre (squared Euclidean distance, ties to
+ * the lower index, decided like gmm_em_step_hard's); inertia (device, 1
+ * double, may be NULL) the sum of squared distances to the input centres.
+ * Computed as hard EM with equal weights and one variance shared by every
+ * component and dimension.  GMM_ERR_UNSUPPORTED as gmm_em_step_hard.
+ */
+gmm_status gmm_em_step_hard(const gmm_problem* p, const void* X, float* w, float* mu,
+                            float* var, int32_t* labels, double* loglik, void* ws,
+                            size_t ws_bytes, void* stream);
+gmm_status gmm_em_step_spherical(const gmm_problem* p, const void* X, float* w, float* mu,
+                                 float* s2, double* loglik, void* ws, size_t ws_bytes,
+                                 void* stream);
+gmm_status gmm_kmeans_step(const gmm_problem* p, const void* X, float* centers, int32_t* labels,
+                           double* inertia, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * iters EM iterations in place.  ll_history (device, iters doubles, may be
  * NULL) receives LL(theta_t) for t = 0 .. iters-1, each of the parameters that
- * iteration started from.
+ * iteration started from.  When the data fit in the shared memory of one
+ * thread-block cluster (gmm_plan's fit_one_launch; about N * D <= 8e5 fp32
+ * values), all iterations run in a single launch: direct-form E-step on the
+ * CUDA cores, statistics in fp64 exchanged over distributed shared memory,
+ * the M-step on chip, parameters written back once.  Otherwise each iteration
+ * is gmm_em_step.
  */
 gmm_status gmm_fit(const gmm_problem* p, const void* X, int32_t iters, float* w, float* mu,
                    float* var, double* ll_history, void* ws, size_t ws_bytes, void* stream);
@@ -288,6 +371,21 @@ gmm_status gmm_device_status(void* ws, size_t ws_bytes, void* stream, uint32_t* 
  * swapped as one, so change it while no other host thread is launching.
  */
 gmm_status gmm_trace_fused(void* start_event, void* stop_event);
+
+/*
+ * Longest time, in nanoseconds, that any device-side wait of the tensor-core
+ * pass spins on a barrier for another warp or CTA before it gives up
+ * (default 1e9, one second; 0 restores the default).  A wait that gives up
+ * sets GMM_DEVFLAG_WAIT_TIMEOUT in the workspace status word; every other wait
+ * of the launch then gives up too, the kernel still waits (up to one second)
+ * for its own copies and MMAs in flight, releases its shared and tensor memory
+ * and returns, and gmm_device_status reports GMM_ERR_TIMEOUT.  The step's
+ * outputs are then not meaningful (restore the parameters), but the device
+ * context stays usable.  A budget below the time a tile takes (microseconds)
+ * makes every step give up: that is how the timeout path is tested.  The
+ * setting is process-wide and applies to launches enqueued after the call.
+ */
+gmm_status gmm_set_wait_budget(uint64_t ns);
 
 /*
  * Number of kernels this library has enqueued in this process so far (all

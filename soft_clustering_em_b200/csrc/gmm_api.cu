@@ -9,13 +9,17 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <unordered_set>
+#include <vector>
 
 #include "common.cuh"
 #include "gmm.h"
 #include "ivf.cuh"
 #include "simt_em.cuh"
+#include "small_fit.cuh"
 #include "tc_em.cuh"
 #include "tma_host.h"
+#include "variants.cuh"
 
 using namespace scem;
 
@@ -62,22 +66,18 @@ struct Plan {
   TcLayout tc;
   bool use_tc;
   size_t stats;  // canonical statistics buffer: K(2D+1)+1 doubles
+  size_t aux;    // the variants' parameters: K x D variances, K weights, one shared variance
   size_t total;
 };
 
 size_t stats_doubles(const gmm_problem* p) { return (size_t)p->K * (2 * (size_t)p->D + 1) + 1; }
-
-bool force_cuda_core_path() {
-  const char* e = getenv("SCEM_GMM_PATH");
-  return e && strcmp(e, "simt") == 0;
-}
 
 Plan make_plan(const gmm_problem* p, int sms, size_t cap) {
   Plan P;
   const size_t sbytes = align_up(stats_doubles(p) * 8, 256);
   const size_t c = cap ? (cap > sbytes ? cap - sbytes : 1) : 0;
   P.simt = c ? ws_layout_capped(p->D, p->K, sms, c) : ws_layout(p->D, p->K, sms);
-  P.use_tc = tc_shape_ok(p->D, p->K) && !force_cuda_core_path();
+  P.use_tc = tc_shape_ok(p->D, p->K, sms);
   if (P.use_tc) {
     P.tc = tc_layout(p->D, p->K, sms, c);
     if (P.tc.P < 1) P.use_tc = false;
@@ -85,7 +85,8 @@ Plan make_plan(const gmm_problem* p, int sms, size_t cap) {
   size_t body = P.simt.P >= 1 ? P.simt.total : 0;
   if (P.use_tc) body = std::max(body, P.tc.total);
   P.stats = align_up(body, 256);
-  P.total = P.stats + sbytes;
+  P.aux = P.stats + sbytes;
+  P.total = P.aux + align_up(((size_t)p->K * p->D + p->K + 1) * 4, 256);
   return P;
 }
 
@@ -187,15 +188,8 @@ gmm_status prep(const gmm_problem* p, const float* w, const float* mu, const flo
 // ---------------------------------------------------------------------------
 // Tensor-core path
 // ---------------------------------------------------------------------------
-constexpr uint64_t kWaitBudgetNs = 1000000000ull;  // 1 s per device-side wait
-
-// Tiles whose statistics accumulate in fp32 tensor memory before an fp64
-// drain (SCEM_GMM_DRAIN_TILES overrides the default, for tuning).
-int tc_drain_tiles() {
-  const char* e = getenv("SCEM_GMM_DRAIN_TILES");
-  const int v = e ? atoi(e) : 0;
-  return v >= 1 && v <= 1024 ? v : kTcDrainTiles;
-}
+constexpr uint64_t kWaitBudgetNs = 1000000000ull;  // default: 1 s per device-side wait
+std::atomic<uint64_t> g_wait_budget_ns{kWaitBudgetNs};  // gmm_set_wait_budget
 
 gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const float* var,
                    char* ws, const TcLayout& T, cudaStream_t st) {
@@ -207,25 +201,17 @@ gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const 
       (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.wsc), (int*)(ws + T.sharp),
       (int*)(ws + T.nsplit), (float*)(ws + T.muh), (float*)(ws + T.ph), (int*)(ws + T.precise),
       (float*)(ws + T.ci), (uint8_t*)(ws + T.perm), (float*)(ws + T.mhp), (float*)(ws + T.php),
-      (uint32_t*)(ws + T.pmask), (uint8_t*)(ws + T.rank), (unsigned int*)ws);
+      (uint32_t*)(ws + T.pmask), (uint8_t*)(ws + T.rank), (unsigned long long*)(ws + T.dirq),
+      (unsigned int*)ws);
   return launched(2);
 }
 
-template <typename XT, int MODE>
-gmm_status tc_launch(const gmm_problem* p, const void* X, char* ws, const TcLayout& T,
-                     cudaStream_t st, int* nslots) {
-  CUtensorMap mhi, mlo;
-  memset(&mhi, 0, sizeof(mhi));
-  memset(&mlo, 0, sizeof(mlo));
-  if (!make_tmap_16b_sw128(&mhi, ws + T.whi, (uint64_t)T.Fpad, (uint64_t)T.Kpad,
-                            (uint64_t)T.Fpad * 2, kTcComps) ||
-      !make_tmap_16b_sw128(&mlo, ws + T.wlo, (uint64_t)T.Fpad, (uint64_t)T.Kpad,
-                            (uint64_t)T.Fpad * 2, kTcComps))
-    return GMM_ERR_CUDA;
-  const TcSmem S = tc_smem_layout(p->D, T.C, T.nchunks);
-  // at least 120 KB so that exactly one CTA (and one 512-column TMEM allocation) sits on an SM
-  const size_t smem = std::max<size_t>(S.total, 120 * 1024);
-  auto kern = tc_fused_kernel<XT, MODE>;
+// Clusters of the fused pass: as many as fit at once, at most one per slot
+// (and, with one group, no more than there are tiles); with G > 1 groups a
+// whole number per group, the same for every chunk of a step.
+template <typename XT, int MODE, int FSRC>
+gmm_status tc_clusters(const TcLayout& T, int64_t ntiles, size_t smem, int* ncl_out) {
+  auto kern = tc_fused_kernel<XT, MODE, FSRC>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess) {
     cudaGetLastError();
@@ -246,7 +232,6 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, char* ws, const TcLayo
   cfg.numAttrs = 1;
   cfg.blockDim = dim3(kTcThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
   cfg.gridDim = dim3((unsigned)(T.C * T.P), 1, 1);
   int max_clusters = 0;
   if (cudaOccupancyMaxActiveClusters(&max_clusters, (void*)kern, &cfg) != cudaSuccess ||
@@ -254,12 +239,56 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, char* ws, const TcLayo
     cudaGetLastError();
     return GMM_ERR_UNSUPPORTED;
   }
-  const int64_t ntiles = (p->N + kTcRows - 1) / kTcRows;
-  const int ncl = (int)std::min<int64_t>(std::min(T.P, max_clusters), ntiles);
+  int ncl = std::min(T.P, max_clusters);
+  if (T.G == 1)
+    ncl = (int)std::min<int64_t>(ncl, ntiles);
+  else
+    ncl = ncl / T.G * T.G;
+  if (ncl < 1) return GMM_ERR_UNSUPPORTED;
+  *ncl_out = ncl;
+  return GMM_OK;
+}
+
+// One launch of the fused kernel over rows [0, N) of X with ncl clusters.
+// FSRC = 1: the rows' features are in the workspace's chunk buffer.
+template <typename XT, int MODE, int FSRC>
+gmm_status tc_launch(const gmm_problem* p, const void* X, int64_t N, char* ws, const TcLayout& T,
+                     int ncl, int accumulate, cudaStream_t st, int32_t* labels = nullptr,
+                     int ncand = 0) {
+  CUtensorMap mhi, mlo, fhi, flo;
+  memset(&mhi, 0, sizeof(mhi));
+  memset(&mlo, 0, sizeof(mlo));
+  memset(&fhi, 0, sizeof(fhi));
+  memset(&flo, 0, sizeof(flo));
+  if (!make_tmap_16b_sw128(&mhi, ws + T.whi, (uint64_t)T.Fpad, (uint64_t)T.Kpad,
+                            (uint64_t)T.Fpad * 2, kTcComps) ||
+      !make_tmap_16b_sw128(&mlo, ws + T.wlo, (uint64_t)T.Fpad, (uint64_t)T.Kpad,
+                            (uint64_t)T.Fpad * 2, kTcComps))
+    return GMM_ERR_CUDA;
+  if (FSRC && (!make_tmap_16b_sw128(&fhi, ws + T.fhi, (uint64_t)T.Fpad, (uint64_t)N,
+                                     (uint64_t)T.Fpad * 2, kTcRows) ||
+               !make_tmap_16b_sw128(&flo, ws + T.flo, (uint64_t)T.Fpad, (uint64_t)N,
+                                     (uint64_t)T.Fpad * 2, kTcRows)))
+    return GMM_ERR_CUDA;
+  const TcSmem S = tc_smem_layout(p->D, T.C, T.nchunks);
+  // at least 120 KB so that exactly one CTA (and one 512-column TMEM allocation) sits on an SM
+  const size_t smem = std::max<size_t>(S.total, 120 * 1024);
+  auto kern = tc_fused_kernel<XT, MODE, FSRC>;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)T.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.blockDim = dim3(kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
   cfg.gridDim = dim3((unsigned)(T.C * ncl), 1, 1);
   TcArgs args;
   args.X = X;
-  args.N = p->N;
+  args.N = N;
   args.D = p->D;
   args.K = p->K;
   args.C = T.C;
@@ -278,28 +307,98 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, char* ws, const TcLayo
   args.php = (const float*)(ws + T.php);
   args.slots = (double*)(ws + T.slots);
   args.slot_stride = T.slot_stride;
+  args.dirq = (unsigned long long*)(ws + T.dirq);
+  args.Kpad = T.Kpad;
+  args.G = T.G;
+  args.part = (float2*)(ws + T.part);
+  args.accumulate = accumulate;
+  args.labels = labels;
+  args.cand = (float2*)(ws + T.cand);
+  args.rowst = (float2*)(ws + T.rowst);
+  args.ncand = std::min(kTcCand, ncand);
   args.status = (unsigned int*)ws;
-  args.drain_tiles = tc_drain_tiles();
+  args.drain_tiles = kTcDrainTiles;
   args.precise = (const int*)(ws + T.precise);
   args.pmask = (const uint32_t*)(ws + T.pmask);
-  args.wait_ns = kWaitBudgetNs;
-  trace_begin(st);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args, mhi, mlo);
-  trace_end(st);
+  args.wait_ns = g_wait_budget_ns.load();
+  args.drain_ns = kWaitBudgetNs;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args, mhi, mlo, fhi, flo);
   if (e != cudaSuccess) {
     fprintf(stderr, "gmm: tensor-core launch failed: %s\n", cudaGetErrorString(e));
     cudaGetLastError();
     return GMM_ERR_CUDA;
   }
-  *nslots = ncl;
   return launched(1);
+}
+
+size_t tc_smem_bytes(const gmm_problem* p, const TcLayout& T) {
+  return std::max<size_t>(tc_smem_layout(p->D, T.C, T.nchunks).total, 120 * 1024);
+}
+
+// The fused pass over all rows of X: one launch with one component group;
+// with G > 1, chunk by chunk, the features converted, then the partial pass,
+// then the statistics (or, for MODE = kTcLoglik, the log-likelihood) pass.
+// *nslots receives the number of slots written.  The trace events bracket
+// the whole pass.
+template <typename XT, int MODE>
+gmm_status tc_pass_t(const gmm_problem* p, const void* X, char* ws, const TcLayout& T,
+                     cudaStream_t st, int* nslots, double* loglik, int32_t* labels) {
+  constexpr int PART = tc_mode_hard(MODE) ? kTcHardPartial : kTcPartial;
+  const int64_t ntiles = (p->N + kTcRows - 1) / kTcRows;
+  const size_t smem = tc_smem_bytes(p, T);
+  gmm_status s;
+  int ncl = 0;
+  if (T.G == 1) {
+    if ((s = tc_clusters<XT, MODE, 0>(T, ntiles, smem, &ncl)) != GMM_OK) return s;
+    trace_begin(st);
+    s = tc_launch<XT, MODE, 0>(p, X, p->N, ws, T, ncl, 0, st, labels);
+    trace_end(st);
+    *nslots = ncl;
+    return s;
+  }
+  if ((s = tc_clusters<XT, PART, 1>(T, ntiles, smem, &ncl)) != GMM_OK) return s;
+  if (tc_mode_stats(MODE)) {
+    int ncl2 = 0;
+    if ((s = tc_clusters<XT, MODE, 1>(T, ntiles, smem, &ncl2)) != GMM_OK) return s;
+    ncl = std::min(ncl, ncl2);
+  }
+  const size_t row_bytes = (size_t)p->D * sizeof(XT);
+  double* blocks = (double*)(ws + T.slots);  // log-likelihood mode: the slots are free
+  trace_begin(st);
+  int64_t i = 0;
+  for (int64_t r0 = 0; r0 < p->N; r0 += T.R, i++) {
+    const int64_t n = std::min<int64_t>(T.R, p->N - r0);
+    const XT* Xc = (const XT*)((const char*)X + (size_t)r0 * row_bytes);
+    const int64_t items = n * (p->D / 4);
+    const unsigned grid = (unsigned)std::min<int64_t>((items + 255) / 256, 148 * 16);
+    tc_convert_kernel<XT><<<grid, 256, 0, st>>>(Xc, n, p->D, T.Fpad, (const float*)(ws + T.m),
+                                               (const float*)(ws + T.isc), (__half*)(ws + T.fhi),
+                                               (__half*)(ws + T.flo), (unsigned int*)ws);
+    if ((s = launched(1)) != GMM_OK) return s;
+    if ((s = tc_launch<XT, PART, 1>(p, Xc, n, ws, T, ncl, 0, st)) != GMM_OK) return s;
+    if (tc_mode_stats(MODE)) {
+      if ((s = tc_launch<XT, MODE, 1>(p, Xc, n, ws, T, ncl, i > 0, st,
+                                      labels ? labels + r0 : nullptr)) != GMM_OK)
+        return s;
+    } else {
+      tc_part_loglik_kernel<<<kTcLseBlocks, 256, 0, st>>>((const float2*)(ws + T.part), n, T.G,
+                                                          blocks);
+      tc_sum_blocks_kernel<<<1, 1, 0, st>>>(blocks, i == 0, loglik);
+      if ((s = launched(2)) != GMM_OK) return s;
+    }
+  }
+  trace_end(st);
+  *nslots = ncl;
+  return GMM_OK;
 }
 
 template <int MODE>
 gmm_status tc_pass(const gmm_problem* p, const void* X, char* ws, const TcLayout& T,
-                   cudaStream_t st, int* nslots) {
-  if (p->xdtype == GMM_BF16) return tc_launch<__nv_bfloat16, MODE>(p, X, ws, T, st, nslots);
-  return tc_launch<float, MODE>(p, X, ws, T, st, nslots);
+                   cudaStream_t st, int* nslots, double* loglik = nullptr,
+                   int32_t* labels = nullptr) {
+  if (p->xdtype == GMM_BF16)
+    return tc_pass_t<__nv_bfloat16, MODE>(p, X, ws, T, st, nslots, loglik, labels);
+  return tc_pass_t<float, MODE>(p, X, ws, T, st, nslots, loglik, labels);
 }
 
 // E-step and statistics of the rows of X into the canonical buffer `stats`.
@@ -308,22 +407,27 @@ gmm_status tc_pass(const gmm_problem* p, const void* X, char* ws, const TcLayout
 // chunk of it.
 gmm_status estep_stats_impl(const gmm_problem* p, const void* X, const float* w,
                             const float* mu, const float* var, double* stats, void* ws_base,
-                            const Plan& P, cudaStream_t st, int64_t n_prep) {
+                            const Plan& P, cudaStream_t st, int64_t n_prep,
+                            bool hard = false, int32_t* labels = nullptr) {
   char* ws = (char*)ws_base;
   gmm_status s;
   const size_t KD = (size_t)p->K * p->D;
   const unsigned blocks = (unsigned)((KD + 255) / 256);
+  if (hard && !P.use_tc) return GMM_ERR_UNSUPPORTED;
   if (P.use_tc) {
     const TcLayout& T = P.tc;
     gmm_problem pp = *p;
     pp.N = n_prep;
     if ((s = tc_prep(&pp, w, mu, var, ws, T, st)) != GMM_OK) return s;
     int nslots = 0;
-    if ((s = tc_pass<kTcStats>(p, X, ws, T, st, &nslots)) != GMM_OK) return s;
+    s = hard ? tc_pass<kTcHardStats>(p, X, ws, T, st, &nslots, nullptr, labels)
+             : tc_pass<kTcStats>(p, X, ws, T, st, &nslots);
+    if (s != GMM_OK) return s;
     tc_reduce_stats_kernel<<<blocks, 256, 0, st>>>(
-        p->D, p->K, (const float*)(ws + T.m), (const float*)(ws + T.sc), mu,
-        (const uint8_t*)(ws + T.rank), (const int*)(ws + T.nsplit),
-        (const double*)(ws + T.slots), T.slot_stride, nslots, stats);
+        p->D, p->K, T.Kpad, (const float*)(ws + T.m), (const float*)(ws + T.sc), mu,
+        (const uint8_t*)(ws + T.rank), (const int*)(ws + T.nsplit), (const float*)(ws + T.ph),
+        (const unsigned long long*)(ws + T.dirq), (const double*)(ws + T.slots), T.slot_stride,
+        nslots, T.G, T.C * kTcComps, stats);
     return launched(1);
   }
   const WsPtrs wp = ws_ptrs(ws_base, P.simt);
@@ -331,6 +435,60 @@ gmm_status estep_stats_impl(const gmm_problem* p, const void* X, const float* w,
   if ((s = fused_pass<kModeStats>(p, X, wp, 0, nullptr, nullptr, st)) != GMM_OK) return s;
   simt_reduce_stats_kernel<<<blocks, 256, 0, st>>>(p->D, p->K, wp, stats);
   return launched(1);
+}
+
+// Top-m assignment on the tensor cores, chunk by chunk (Rt rows): with G > 1
+// groups the features are converted and the partial pass runs first; the
+// top-m pass writes each (CTA, column half)'s candidates and each row's
+// (max, sum-exp); tc_topm_refine_kernel finishes the rows in direct form.
+template <typename XT>
+gmm_status tc_topm_t(const gmm_problem* p, const void* X, const float* w, const float* mu,
+                     const float* var, int m, int32_t* idx, float* resp, char* ws, const Plan& P,
+                     cudaStream_t st) {
+  const TcLayout& T = P.tc;
+  gmm_status s;
+  if ((s = tc_prep(p, w, mu, var, ws, T, st)) != GMM_OK) return s;
+  float* iv = (float*)(ws + P.aux);
+  float* c0 = iv + (size_t)p->K * p->D;
+  tc_topm_prep_kernel<<<p->K, 128, 0, st>>>(p->D, w, var, iv, c0);
+  if ((s = launched(1)) != GMM_OK) return s;
+  const int nc = std::min(m + 2, kTcCand);
+  const size_t smem = tc_smem_bytes(p, T);
+  const size_t row_bytes = (size_t)p->D * sizeof(XT);
+  trace_begin(st);
+  for (int64_t r0 = 0; r0 < p->N; r0 += T.Rt) {
+    const int64_t n = std::min<int64_t>(T.Rt, p->N - r0);
+    const int64_t ntiles = (n + kTcRows - 1) / kTcRows;
+    const XT* Xc = (const XT*)((const char*)X + (size_t)r0 * row_bytes);
+    int ncl = 0;
+    if (T.G == 1) {
+      if ((s = tc_clusters<XT, kTcTopm, 0>(T, ntiles, smem, &ncl)) != GMM_OK) return s;
+      if ((s = tc_launch<XT, kTcTopm, 0>(p, Xc, n, ws, T, ncl, 0, st, nullptr, nc)) != GMM_OK)
+        return s;
+    } else {
+      int ncl2 = 0;
+      if ((s = tc_clusters<XT, kTcPartial, 1>(T, ntiles, smem, &ncl)) != GMM_OK ||
+          (s = tc_clusters<XT, kTcTopm, 1>(T, ntiles, smem, &ncl2)) != GMM_OK)
+        return s;
+      ncl = std::min(ncl, ncl2);
+      const int64_t items = n * (p->D / 4);
+      const unsigned grid = (unsigned)std::min<int64_t>((items + 255) / 256, 148 * 16);
+      tc_convert_kernel<XT><<<grid, 256, 0, st>>>(Xc, n, p->D, T.Fpad, (const float*)(ws + T.m),
+                                                 (const float*)(ws + T.isc),
+                                                 (__half*)(ws + T.fhi), (__half*)(ws + T.flo),
+                                                 (unsigned int*)ws);
+      if ((s = launched(1)) != GMM_OK) return s;
+      if ((s = tc_launch<XT, kTcPartial, 1>(p, Xc, n, ws, T, ncl, 0, st)) != GMM_OK ||
+          (s = tc_launch<XT, kTcTopm, 1>(p, Xc, n, ws, T, ncl, 0, st, nullptr, nc)) != GMM_OK)
+        return s;
+    }
+    tc_topm_refine_kernel<XT><<<(unsigned)((n + 127) / 128), 128, 0, st>>>(
+        Xc, n, p->D, p->K, T.G * T.C * 2, nc, m, (const float2*)(ws + T.cand),
+        (const float2*)(ws + T.rowst), mu, iv, c0, idx + (size_t)r0 * m, resp + (size_t)r0 * m);
+    if ((s = launched(1)) != GMM_OK) return s;
+  }
+  trace_end(st);
+  return GMM_OK;
 }
 
 gmm_status mstep_impl(const gmm_problem* p, const double* stats, int nshards, float* w,
@@ -389,6 +547,58 @@ gmm_status em_step_impl(const gmm_problem* p, const void* X, float* w, float* mu
   return mstep_impl(p, stats, 1, w, mu, var, loglik, st);
 }
 
+// All iterations of a small fit in one launch of one cluster (small_fit.cuh).
+// GMM_ERR_UNSUPPORTED when the cluster cannot be placed on this device.
+template <typename XT>
+gmm_status small_fit_t(const gmm_problem* p, const void* X, int iters, float* w, float* mu,
+                       float* var, double* ll, unsigned int* status, cudaStream_t st) {
+  const int C = sf_cluster(p->N, p->D, p->K);
+  const size_t smem = sf_layout(p->N, p->D, p->K, C).total;
+  auto kern = small_fit_kernel<XT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess ||
+      (C > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                    cudaSuccess)) {
+    cudaGetLastError();
+    return GMM_ERR_UNSUPPORTED;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.blockDim = dim3(kSfThreads, 1, 1);
+  cfg.gridDim = dim3((unsigned)C, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  int max_clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&max_clusters, (void*)kern, &cfg) != cudaSuccess ||
+      max_clusters < 1) {
+    cudaGetLastError();
+    return GMM_ERR_UNSUPPORTED;
+  }
+  trace_begin(st);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, (const XT*)X, p->N, p->D, p->K, iters,
+                                           p->var_floor, w, mu, var, ll, status);
+  trace_end(st);
+  if (e != cudaSuccess) {
+    fprintf(stderr, "gmm: small-fit launch failed: %s\n", cudaGetErrorString(e));
+    cudaGetLastError();
+    return GMM_ERR_CUDA;
+  }
+  return launched(1);
+}
+
+gmm_status small_fit(const gmm_problem* p, const void* X, int iters, float* w, float* mu,
+                     float* var, double* ll, unsigned int* status, cudaStream_t st) {
+  if (p->xdtype == GMM_BF16)
+    return small_fit_t<__nv_bfloat16>(p, X, iters, w, mu, var, ll, status, st);
+  return small_fit_t<float>(p, X, iters, w, mu, var, ll, status, st);
+}
+
 // ---------------------------------------------------------------------------
 // Scratch for gmm_em_step_noalloc: a fixed array in the module's own device
 // memory, so that entry point never asks for memory.  It exists on every
@@ -400,7 +610,37 @@ constexpr size_t kNoallocScratchBytes = (size_t)32 << 20;
 constexpr int kNoallocMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoallocMaxDevices] = {};
+// The address is looked up once per device and context: the context that was
+// current at the lookup is kept beside it, and a call made under another one
+// (a context created after cudaDeviceReset, or a non-primary driver context)
+// looks the address up again.
+struct NoallocEntry {
+  void* ctx;
+  void* ptr;
+};
+NoallocEntry g_noalloc_cache[kNoallocMaxDevices] = {};
+
+typedef int (*CtxGetCurrentFn)(void**);
+
+// The calling thread's current driver context (null if none or unknown),
+// fetched through the runtime so the library does not link libcuda.
+void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+    else
+      cudaGetLastError();
+    tried = true;
+  }
+  void* ctx = nullptr;
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
 
 gmm_status noalloc_scratch(void** out) {
   int dev = 0;
@@ -410,17 +650,61 @@ gmm_status noalloc_scratch(void** out) {
   }
   if (dev < 0 || dev >= kNoallocMaxDevices) return GMM_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  void* ctx = current_context();
+  NoallocEntry& e = g_noalloc_cache[dev];
+  if (!e.ptr || !ctx || e.ctx != ctx) {
     void* ptr = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    if (e != cudaSuccess || ptr == nullptr) {
+    const cudaError_t r = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (r != cudaSuccess || ptr == nullptr) {
       cudaGetLastError();
       return GMM_ERR_CUDA;
     }
-    g_noalloc_ptr[dev] = ptr;
+    e.ctx = ctx;
+    e.ptr = ptr;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = e.ptr;
   return GMM_OK;
+}
+
+
+// SplitMix64 in counter form (Steele, Lea and Flood, "Fast splittable
+// pseudorandom number generators", OOPSLA 2014): the i-th output (i = 0, 1, ...)
+// of the generator started from state `seed`.
+uint64_t splitmix64_at(uint64_t seed, uint64_t i) {
+  uint64_t z = seed + (i + 1) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Uniform integer in [0, n) from the stream's next outputs (*ctr counts the
+// outputs used): an output x is taken as x mod n when it lies below the
+// largest multiple of n that fits in 64 bits, otherwise the next one is drawn,
+// so every value is equally likely.
+uint64_t uniform_below(uint64_t seed, uint64_t* ctr, uint64_t n) {
+  const uint64_t rem = (0 - n) % n;  // 2^64 mod n
+  for (;;) {
+    const uint64_t x = splitmix64_at(seed, (*ctr)++);
+    if (x <= ~rem) return x % n;  // x < 2^64 - rem
+  }
+}
+
+// K distinct indices from [0, N), every K-subset equally likely: Floyd's
+// algorithm (Bentley and Floyd, "A sample of brilliance", Programming Pearls,
+// CACM 1987).  For j = N-K .. N-1 draw t uniform in [0, j]; take t, or j when t
+// was already taken.  rows[k] is the index taken at step k.
+void sample_rows(int64_t N, int K, uint64_t seed, std::vector<int64_t>* rows) {
+  rows->clear();
+  rows->reserve(K);
+  std::unordered_set<int64_t> taken;
+  taken.reserve(2 * (size_t)K);
+  uint64_t ctr = 0;
+  for (int64_t j = N - K; j < N; j++) {
+    const int64_t t = (int64_t)uniform_below(seed, &ctr, (uint64_t)j + 1);
+    const int64_t v = taken.count(t) ? j : t;
+    taken.insert(v);
+    rows->push_back(v);
+  }
 }
 
 }  // namespace
@@ -451,9 +735,9 @@ gmm_status gmm_workspace_size(const gmm_problem* p, size_t* bytes) {
   return GMM_OK;
 }
 
-gmm_status gmm_init(const gmm_problem* p, const void* X, const int64_t* rows_host,
-                    int32_t init_var, float* w, float* mu, float* var, void* ws, size_t ws_bytes,
-                    void* stream) {
+gmm_status gmm_init_rows(const gmm_problem* p, const void* X, const int64_t* rows_host,
+                         int32_t init_var, float* w, float* mu, float* var, void* ws,
+                         size_t ws_bytes, void* stream) {
   gmm_status s = check_problem(p);
   if (s != GMM_OK) return s;
   if ((s = check_x(p, X)) != GMM_OK) return s;
@@ -495,6 +779,35 @@ gmm_status gmm_init(const gmm_problem* p, const void* X, const int64_t* rows_hos
     }
   }
   return GMM_OK;
+}
+
+gmm_status gmm_plan(const gmm_problem* p, gmm_plan_info* info) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if (!info) return GMM_ERR_INVALID_ARG;
+  int sms = 0;
+  if ((s = device_sms(&sms)) != GMM_OK) return s;
+  const Plan P = make_plan(p, sms, 0);
+  memset(info, 0, sizeof(*info));
+  info->tensor_cores = P.use_tc ? 1 : 0;
+  info->fit_one_launch = sf_cluster(p->N, p->D, p->K) > 0 ? 1 : 0;
+  if (P.use_tc) {
+    info->cluster_ctas = P.tc.C;
+    info->groups = P.tc.G;
+    info->chunk_rows = P.tc.G > 1 ? P.tc.R : 0;
+  }
+  return GMM_OK;
+}
+
+gmm_status gmm_init(const gmm_problem* p, const void* X, uint64_t seed, int32_t init_var,
+                    float* w, float* mu, float* var, void* ws, size_t ws_bytes, void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if (p->K > p->N) return GMM_ERR_INVALID_ARG;  // K distinct rows are needed
+  std::vector<int64_t> rows;
+  sample_rows(p->N, p->K, seed, &rows);
+  // pageable source: the copy inside gmm_init_rows has read it when that call returns
+  return gmm_init_rows(p, X, rows.data(), init_var, w, mu, var, ws, ws_bytes, stream);
 }
 
 gmm_status gmm_em_step(const gmm_problem* p, const void* X, float* w, float* mu, float* var,
@@ -563,6 +876,68 @@ gmm_status gmm_em_step_noalloc(const gmm_problem* p, const void* X, float* w, fl
   return GMM_OK;
 }
 
+gmm_status gmm_em_step_hard(const gmm_problem* p, const void* X, float* w, float* mu,
+                            float* var, int32_t* labels, double* loglik, void* ws,
+                            size_t ws_bytes, void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if ((s = check_x(p, X)) != GMM_OK) return s;
+  if (!w || !mu || !var) return GMM_ERR_INVALID_ARG;
+  Plan P;
+  if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  if (!P.use_tc) return GMM_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  double* stats = (double*)((char*)ws + P.stats);
+  if ((s = estep_stats_impl(p, X, w, mu, var, stats, ws, P, st, p->N, true, labels)) != GMM_OK)
+    return s;
+  return mstep_impl(p, stats, 1, w, mu, var, loglik, st);
+}
+
+gmm_status gmm_em_step_spherical(const gmm_problem* p, const void* X, float* w, float* mu,
+                                 float* s2, double* loglik, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if ((s = check_x(p, X)) != GMM_OK) return s;
+  if (!w || !mu || !s2) return GMM_ERR_INVALID_ARG;
+  Plan P;
+  if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t KD = (size_t)p->K * p->D;
+  float* var = (float*)((char*)ws + P.aux);
+  double* stats = (double*)((char*)ws + P.stats);
+  sph_expand_kernel<<<(unsigned)((KD + 255) / 256), 256, 0, st>>>(p->D, p->K, s2, var);
+  if ((s = launched(1)) != GMM_OK) return s;
+  if ((s = estep_stats_impl(p, X, w, mu, var, stats, ws, P, st, p->N)) != GMM_OK) return s;
+  sph_mstep_kernel<<<p->K, 128, 0, st>>>(p->N, p->D, p->K, p->var_floor, stats, w, mu, s2, loglik);
+  return launched(1);
+}
+
+gmm_status gmm_kmeans_step(const gmm_problem* p, const void* X, float* centers, int32_t* labels,
+                           double* inertia, void* ws, size_t ws_bytes, void* stream) {
+  gmm_status s = check_problem(p);
+  if (s != GMM_OK) return s;
+  if ((s = check_x(p, X)) != GMM_OK) return s;
+  if (!centers) return GMM_ERR_INVALID_ARG;
+  Plan P;
+  if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  if (!P.use_tc) return GMM_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t KD = (size_t)p->K * p->D;
+  float* var = (float*)((char*)ws + P.aux);
+  float* w = var + KD;
+  float* v = w + p->K;
+  double* stats = (double*)((char*)ws + P.stats);
+  km_prep_kernel<<<1, 256, 0, st>>>(p->D, p->K, centers, w, var, v);
+  if ((s = launched(1)) != GMM_OK) return s;
+  if ((s = estep_stats_impl(p, X, w, centers, var, stats, ws, P, st, p->N, true, labels)) !=
+      GMM_OK)
+    return s;
+  km_mstep_kernel<<<(unsigned)((KD + 255) / 256), 256, 0, st>>>(p->N, p->D, p->K, stats, v,
+                                                                centers, inertia);
+  return launched(1);
+}
+
 gmm_status gmm_fit(const gmm_problem* p, const void* X, int32_t iters, float* w, float* mu,
                    float* var, double* ll_history, void* ws, size_t ws_bytes, void* stream) {
   gmm_status s = check_problem(p);
@@ -571,6 +946,10 @@ gmm_status gmm_fit(const gmm_problem* p, const void* X, int32_t iters, float* w,
   if (!w || !mu || !var || iters < 0) return GMM_ERR_INVALID_ARG;
   Plan P;
   if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  if (iters > 0 && sf_cluster(p->N, p->D, p->K) > 0) {
+    s = small_fit(p, X, iters, w, mu, var, ll_history, (unsigned int*)ws, (cudaStream_t)stream);
+    if (s != GMM_ERR_UNSUPPORTED) return s;  // else: no such cluster fits now; step by step
+  }
   for (int t = 0; t < iters; t++) {
     s = em_step_impl(p, X, w, mu, var, ll_history ? ll_history + t : nullptr, ws, P,
                      (cudaStream_t)stream);
@@ -593,7 +972,8 @@ gmm_status gmm_loglik(const gmm_problem* p, const void* X, const float* w, const
     const TcLayout& T = P.tc;
     if ((s = tc_prep(p, w, mu, var, wsb, T, st)) != GMM_OK) return s;
     int nslots = 0;
-    if ((s = tc_pass<kTcLoglik>(p, X, wsb, T, st, &nslots)) != GMM_OK) return s;
+    if ((s = tc_pass<kTcLoglik>(p, X, wsb, T, st, &nslots, loglik)) != GMM_OK) return s;
+    if (T.G > 1) return GMM_OK;  // the chunks' sums went straight into *loglik
     tc_reduce_loglik_kernel<<<1, 1, 0, st>>>(p->D, p->K, (const double*)(wsb + T.slots),
                                              T.slot_stride, nslots, loglik);
     return launched(1);
@@ -615,8 +995,13 @@ gmm_status gmm_assign_topm(const gmm_problem* p, const void* X, const float* w, 
   if (m < 1 || m > kMaxTopM || m > p->K) return GMM_ERR_INVALID_ARG;
   Plan P;
   if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
-  const WsPtrs wp = ws_ptrs(ws, P.simt);
   cudaStream_t st = (cudaStream_t)stream;
+  if (P.use_tc) {
+    if (p->xdtype == GMM_BF16)
+      return tc_topm_t<__nv_bfloat16>(p, X, w, mu, var, m, idx, resp, (char*)ws, P, st);
+    return tc_topm_t<float>(p, X, w, mu, var, m, idx, resp, (char*)ws, P, st);
+  }
+  const WsPtrs wp = ws_ptrs(ws, P.simt);
   if ((s = prep(p, w, mu, var, wp, st)) != GMM_OK) return s;
   return fused_pass<kModeTopm>(p, X, wp, m, idx, resp, st);
 }
@@ -711,6 +1096,11 @@ gmm_status gmm_em_step_host(const gmm_problem* p, const void* X_host, int64_t ch
     if (cudaEventRecord(ev.used[b], st) != cudaSuccess) return launch_status(), GMM_ERR_CUDA;
   }
   return mstep_impl(p, total, 1, w, mu, var, loglik, st);
+}
+
+gmm_status gmm_set_wait_budget(uint64_t ns) {
+  g_wait_budget_ns = ns == 0 ? kWaitBudgetNs : ns;
+  return GMM_OK;
 }
 
 gmm_status gmm_launch_count(uint64_t* count) {

@@ -69,6 +69,10 @@
 
 #include <math.h>
 
+#include <limits.h>
+
+#include <algorithm>
+
 #include "common.cuh"
 #include "sm100_prims.cuh"
 
@@ -103,8 +107,50 @@ constexpr float kTcXMax = 240.0f;                // |x^| beyond this cannot be s
 // of adding up; from zero they would grow with Q_k, which reaches 10^4 for
 // tight components far from the centring point.
 constexpr double kTcStartFrac = -0.625;
+// Fixed-point unit of the split dimensions' direct-form moments: each row's
+// r (x - mu) / sigma and r (x - mu)^2 / sigma^2 is rounded to a multiple of
+// 2^-32 and added as a signed 64-bit integer split into a high word
+// (q >> 32, signed) and a low word (q mod 2^32), each summed with a 64-bit
+// integer atomic.  Integer sums do not depend on the order of the additions,
+// so the result is deterministic whatever the scheduling; the rounding is
+// 2^-33 of a standard deviation per row, and the low-word sum stays exact for
+// up to 2^31 contributing rows per component.
+constexpr double kTcDirScale = 4294967296.0;  // 2^32
 
-enum TcMode { kTcStats = 0, kTcLoglik = 1 };
+// kTcStats: E-step, responsibilities and statistics (with G > 1 component
+//   groups, the rows' log-sum-exp comes from the groups' partials written by a
+//   kTcPartial pass over the same rows).
+// kTcLoglik: E-step and the log-likelihood only (one group).
+// kTcPartial: E-step of this cluster's component group; each row's (max,
+//   sum-exp) over the group's components goes to the row buffer.
+// kTcHardStats / kTcHardPartial: the same for hard (classification) EM: each
+//   row goes wholly to its most probable component (ties to the lower
+//   index); the exchanged partials are (max log-joint, its component index)
+//   instead of (max, sum-exp), the responsibilities one-hot, and the
+//   log-likelihood the classification one, sum_n max_k l_nk.
+// kTcTopm: E-step and row normalisation (with G > 1 groups, from the partial
+//   pass); each (CTA, column half) writes its kTcCand largest log-joints with
+//   their component indices to the candidate buffer, and the row's (max,
+//   sum-exp) to the row buffer, for tc_topm_refine_kernel.
+enum TcMode {
+  kTcStats = 0,
+  kTcLoglik = 1,
+  kTcPartial = 2,
+  kTcHardStats = 3,
+  kTcHardPartial = 4,
+  kTcTopm = 5
+};
+constexpr int kTcCand = 8;  // candidates per (CTA, column half) and row for top-m
+__host__ __device__ constexpr bool tc_mode_stats(int m) { return m == kTcStats || m == kTcHardStats; }
+__host__ __device__ constexpr bool tc_mode_partial(int m) {
+  return m == kTcPartial || m == kTcHardPartial;
+}
+__host__ __device__ constexpr bool tc_mode_hard(int m) {
+  return m == kTcHardStats || m == kTcHardPartial;
+}
+constexpr int kTcMaxGroups = 64;
+constexpr int64_t kTcChunkRowsMax = 1 << 18;       // rows per pass with component groups
+constexpr size_t kTcChunkFBytesMax = 256u << 20;   // cap on the chunk's feature buffer
 
 // Optional phase timestamps for performance work (off unless the library is
 // built with -DSCEM_PHASE_TRACE): slot `idx` of the first 64 tiles of cluster
@@ -166,7 +212,7 @@ __host__ __device__ inline TcSmem tc_smem_layout_n(int D, int C, int nchunks, ui
   L.xchg = off;
   off += 2u * 2u * C * kTcRows * 8;  // [parity][rank][column half][row]
   L.bars = off;
-  off += 8 * (2 * kTcStages + 12);
+  off += 8 * (2 * kTcStages + 16);
   L.tslot = off;
   off += 16;
   L.total = off + 1024;  // slack for aligning the dynamic base to 1024
@@ -196,29 +242,73 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //   mhp, php : [C*128 x D] f32 mu^ and 1/var^ in perm order
 //   whi, wlo : [C*128 x 64*nchunks] fp16 operand W (hi and lo parts)
 //   rank : [C*128 x D] u8 position of each dimension in perm
+//   dirq : [4D x C*128] u64 direct-form moments of split dimensions about the
+//          input means, by perm position i, as 64-bit fixed-point words (see
+//          kTcDirScale): rows i / D+i hold the high / low words of
+//          sum r (x - mu) / sigma, rows 2D+i / 3D+i those of
+//          sum r (x - mu)^2 / sigma^2.  One area for all clusters: integer
+//          additions commute, so the sums do not depend on the order in which
+//          rows or clusters add them.  Zeroed by tc_prep_w_kernel.
 //   slots: P per-cluster slots of slot_stride doubles:
 //          [(2D+1) x K] feature-major statistics (S1 rows 0..D-1, S2 rows
-//          D..2D-1, N_k row 2D), the cluster's LL, then [2D x K] direct-form
-//          moments of split dimensions about the input means, by perm position
-//          i: sum r (x - mu) in row i, sum r (x - mu)^2 in row D + i.
+//          D..2D-1, N_k row 2D), then the cluster's LL.
+//   With G > 1 component groups, also (after the slots):
+//   fhi, flo : [R x Fpad] fp16 features [x^, x^^2] (hi and lo parts) of one
+//              chunk of R rows, written by tc_convert_kernel, read by TMA
+//   part     : [R x G] float2 (max, sum-exp) of each row over each group
+//   Top-m assignment, for chunks of Rt rows:
+//   cand     : [Rt x (G C 2) x kTcCand] float2 (log-joint, index) candidates
+//   rowst    : [Rt] float2 (max, sum-exp) of each row
 struct TcLayout {
   size_t m, isc, sc, c, ci, wsc, sharp, nsplit, precise, pmask, muh, ph, perm, rank, mhp, php, whi,
-      wlo, slots, total, slot_stride;
-  int C, nchunks, Kpad, Fpad, P;
+      wlo, dirq, slots, fhi, flo, part, cand, rowst, total, slot_stride;
+  int C, G, nchunks, Kpad, Fpad, P;
+  int64_t R;   // rows per chunk (G > 1)
+  int64_t Rt;  // rows per chunk of the top-m assignment
 };
 
-inline bool tc_shape_ok(int D, int K) {
-  if (!(D >= 4 && D <= 128 && D % 4 == 0 && K >= 1 && K <= kTcComps * kTcMaxCluster))
-    return false;
-  return tc_smem_layout(D, tc_cluster(K), tc_nchunks(D)).total <= kTcMaxSmem;
+// Cluster size C and number of component groups G for a shape: the fewest
+// groups whose cluster (C = ceil(ceil(K/128) / G) CTAs of 128 components, at
+// most 16) fits the kernel's shared memory, and no more groups than the SMs
+// can hold one cluster each.  False if none does (or D is not a multiple of 4
+// up to 128): such shapes run on the CUDA cores.
+inline bool tc_shape(int D, int K, int num_sms, int* C_out, int* G_out) {
+  if (!(D >= 4 && D <= 128 && D % 4 == 0 && K >= 1)) return false;
+  const int cfull = tc_cluster(K);
+  for (int G = 1; G <= kTcMaxGroups; G++) {
+    const int C = (cfull + G - 1) / G;
+    if (C > kTcMaxCluster) continue;
+    if (tc_smem_layout(D, C, tc_nchunks(D)).total > kTcMaxSmem) continue;
+    if (G > 1 && num_sms / C < G) return false;
+    *C_out = C;
+    *G_out = G;
+    return true;
+  }
+  return false;
+}
+
+inline bool tc_shape_ok(int D, int K, int num_sms = 148) {
+  int C, G;
+  return tc_shape(D, K, num_sms, &C, &G);
+}
+
+// Rows per chunk with component groups: at most 2^18, the chunk's features
+// (4 Fpad bytes per row) at most 256 MiB, a multiple of the tile.
+inline int64_t tc_chunk_rows(int Fpad) {
+  int64_t r = (int64_t)(kTcChunkFBytesMax / (4u * (size_t)Fpad));
+  r = std::min<int64_t>(r, kTcChunkRowsMax);
+  return r / kTcRows * kTcRows;
 }
 
 inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   TcLayout L;
-  L.C = tc_cluster(K);
+  L.C = 1;
+  L.G = 1;
+  tc_shape(D, K, num_sms, &L.C, &L.G);
   L.nchunks = tc_nchunks(D);
-  L.Kpad = L.C * kTcComps;
+  L.Kpad = L.G * L.C * kTcComps;
   L.Fpad = L.nchunks * kTcChunk;
+  L.R = L.G > 1 ? tc_chunk_rows(L.Fpad) : 0;
   size_t off = 256;
   L.m = off;
   off = align_up(off + (size_t)D * 4, 256);
@@ -256,14 +346,40 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.pmask = off;
   off = align_up(off + (size_t)L.Kpad * (L.Fpad / 32) * 4, 256);
-  L.slot_stride = align_up((size_t)(4 * D + 1) * K + 1, 32);
+  L.dirq = off;
+  off = align_up(off + (size_t)4 * D * L.Kpad * 8, 256);
+  L.slot_stride = align_up((size_t)(2 * D + 1) * K + 1, 32);
+  // the chunk buffers of the two-pass form (G > 1), ahead of the slots
+  L.fhi = L.flo = L.part = off;
+  if (L.G > 1) {
+    L.fhi = off;
+    off = align_up(off + (size_t)L.R * L.Fpad * 2, 256);
+    L.flo = off;
+    off = align_up(off + (size_t)L.R * L.Fpad * 2, 256);
+    L.part = off;
+    off = align_up(off + (size_t)L.R * L.G * 8, 256);
+  }
+  // top-m candidates: at most 64 MiB, at most 2^18 rows (and R with groups)
+  {
+    const size_t per_row = (size_t)L.G * L.C * 2 * kTcCand * 8 + 8;
+    int64_t rt = (int64_t)((size_t)(64u << 20) / per_row) / kTcRows * kTcRows;
+    rt = std::max<int64_t>(kTcRows, std::min<int64_t>(rt, kTcChunkRowsMax));
+    if (L.G > 1) rt = std::min<int64_t>(rt, L.R);
+    L.Rt = rt;
+    L.cand = off;
+    off = align_up(off + (size_t)rt * (per_row - 8), 256);
+    L.rowst = off;
+    off = align_up(off + (size_t)rt * 8, 256);
+  }
   L.slots = off;
+  // one slot per cluster; with G > 1 a whole number of clusters per group
   L.P = num_sms / L.C;
   if (cap) {
     const size_t per = L.slot_stride * 8;
     const size_t fit = cap > off ? (cap - off) / per : 0;
     if ((size_t)L.P > fit) L.P = (int)fit;
   }
+  L.P = L.P / L.G * L.G;
   L.total = align_up(off + (size_t)L.P * L.slot_stride * 8, 256);
   return L;
 }
@@ -287,11 +403,23 @@ struct TcArgs {
   const float* php;     // 1/var^ in that order, C*128 x D
   double* slots;        // per-cluster statistic slots
   size_t slot_stride;   // doubles per slot: (2D+1)*K statistics + LL
+  unsigned long long* dirq;  // fixed-point direct-form moments of split dimensions, 4D x Kpad
+  int Kpad;
+  int G;                // component groups; cluster c serves group c % G
+  float2* part;         // G > 1: [rows x G] (max, sum-exp) per row and group
+  int accumulate;       // 1: add onto the slots (a later chunk of the same step)
+  int32_t* labels;      // hard EM: each row's component (may be null)
+  float2* cand;         // top-m: [rows x (G C 2) x kTcCand] (log-joint, index) candidates
+  float2* rowst;        // top-m: [rows] the row's (max, sum-exp) over all components
+  int ncand;            // top-m: candidates kept per (CTA, column half), <= kTcCand
   unsigned int* status;
   int drain_tiles;
   const int* precise;   // 1: some feature of the component is drained every tile, C*128
   const uint32_t* pmask;  // which features, C*128 x (Fpad/32) words
-  uint64_t wait_ns;
+  uint64_t wait_ns;   // budget of every wait for another warp or CTA (gmm_set_wait_budget)
+  uint64_t drain_ns;  // budget of the two waits for the CTA's own copies and MMAs in flight
+                      // before it may release shared and tensor memory (fixed, 1 s): these
+                      // complete in microseconds and ignore the abort bit
 };
 
 // A shared-memory descriptor advanced by `bytes` (start-address field only;
@@ -304,6 +432,14 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }
 
 __device__ __forceinline__ float round_half(float a) { return __half2float(__float2half_rn(a)); }
+
+// Adds v (already in units of 2^-32) to the fixed-point pair (hi, lo).
+__device__ __forceinline__ void fixed_add(unsigned long long* hi, unsigned long long* lo,
+                                          double v) {
+  const long long q = __double2ll_rn(v);
+  atomicAdd(hi, (unsigned long long)(q >> 32));
+  atomicAdd(lo, (unsigned long long)(q & 0xffffffffll));
+}
 
 // (a, b) -> fp16 pairs hi = fp16(a, b) and lo = fp16(a - hi_a, b - hi_b), packed:
 // three conversion instructions for two values.
@@ -350,11 +486,18 @@ __device__ __forceinline__ float load1<__nv_bfloat16>(const __nv_bfloat16* X, in
 
 // 10 warps put 3 on some of the 4 sub-partitions (16K registers each): 168 registers
 // per thread at most.
-template <typename XT, int MODE>
+// FSRC = 0: the compute warps convert X into the features F in shared memory.
+// FSRC = 1: F comes pre-converted (tc_convert_kernel) and the TMA warp loads
+//           each tile's F chunks (tm_fhi / tm_flo) next to the W stream.
+template <typename XT, int MODE, int FSRC>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fused_kernel(const TcArgs a, const __grid_constant__ CUtensorMap tm_whi,
-                    const __grid_constant__ CUtensorMap tm_wlo) {
+                    const __grid_constant__ CUtensorMap tm_wlo,
+                    const __grid_constant__ CUtensorMap tm_fhi,
+                    const __grid_constant__ CUtensorMap tm_flo) {
   using namespace sm100;
+  constexpr bool kStats = tc_mode_stats(MODE), kPartial = tc_mode_partial(MODE);
+  constexpr bool kHard = tc_mode_hard(MODE);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -385,17 +528,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* r_full1 = f_full + 8;  // second 64-row half of r^ written
   uint64_t* r_free = f_full + 9;   // MMAs of the first half done with the r^ buffer
   uint64_t* cbar = f_full + 10;    // rendezvous of the 256 compute threads
+  uint64_t* f_free = f_full + 11;  // [2] FSRC = 1: MMAs and epilogue done with an F buffer
+  uint64_t* f_tx = f_full + 13;    // [2] FSRC = 1: an F buffer's TMA loads have landed
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tslot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
-  const uint32_t cid = cluster_id_x(), ncl = nclusters_x();
+  // cluster c serves component group c % G and takes every (nclusters/G)-th tile
+  const uint32_t ngrp = (uint32_t)a.G;
+  const uint32_t grp = cluster_id_x() % ngrp;
+  const uint32_t cid = cluster_id_x() / ngrp, ncl = nclusters_x() / ngrp;
+  const uint32_t slot_id = cluster_id_x();
   const int64_t ntiles = (a.N + kTcRows - 1) / kTcRows;
   const int64_t my_tiles = ((int64_t)cid < ntiles) ? (ntiles - 1 - (int64_t)cid) / ncl + 1 : 0;
-  const int k0 = (int)rank * kTcComps;
+  const int k0 = (int)(grp * (uint32_t)C + rank) * kTcComps;
   volatile unsigned int* status = a.status;
   constexpr unsigned int kAbort = GMM_DEVFLAG_WAIT_TIMEOUT;
-  double* slot = a.slots + (size_t)cid * a.slot_stride;
+  double* slot = a.slots + (size_t)slot_id * a.slot_stride;
   const size_t ll_index = (size_t)(2 * D + 1) * K;
 
   // ---------------------------------------------------------------- set-up
@@ -404,7 +553,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(f_full, kTcComputeThreads);
+    mbar_init(f_full, kTcComputeThreads);  // start values stored (and, FSRC = 0, F written)
+    for (int b = 0; b < 2; b++) {
+      mbar_init(&f_free[b], 1);
+      mbar_init(&f_tx[b], 1);
+    }
     mbar_init(l_full, 1);
     mbar_init(r_full, kTcComputeThreads / 2);
     mbar_init(r_full1, kTcComputeThreads / 2);
@@ -444,23 +597,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   for (int i = tid; i < 2048; i += kTcThreads)
     reinterpret_cast<__half*>(sOnes)[i] = __float2half_rn(1.0f);
-  // padding features of F must read as zero in every MMA
-  for (uint32_t i = tid; i < L.nfb * L.fbytes / 16; i += kTcThreads)
-    reinterpret_cast<uint4*>(sF)[i] = make_uint4(0, 0, 0, 0);
-  if (MODE == kTcStats) {
+  // padding features of F must read as zero in every MMA (FSRC = 1: the
+  // pre-converted features hold zeros there)
+  if (!FSRC)
+    for (uint32_t i = tid; i < L.nfb * L.fbytes / 16; i += kTcThreads)
+      reinterpret_cast<uint4*>(sF)[i] = make_uint4(0, 0, 0, 0);
+  if (kStats && !a.accumulate) {
     for (int f = 0; f <= 2 * D; f++)
       for (int kk = tid; kk < kTcComps; kk += kTcThreads)
         if (k0 + kk < K) slot[(size_t)f * K + k0 + kk] = 0.0;
-    // the direct-form moments of split dimensions (the rows the reduction reads)
-    double* dir = slot + ll_index + 1;
-    for (int kk = tid; kk < kTcComps; kk += kTcThreads)
-      if (k0 + kk < K) {
-        const int ns = a.nsplit[k0 + kk];
-        for (int i = 0; i < ns; i++) {
-          dir[(size_t)i * K + k0 + kk] = 0.0;
-          dir[(size_t)(D + i) * K + k0 + kk] = 0.0;
-        }
-      }
   }
   fence_proxy_async_smem();
   tc_fence_before_sync();
@@ -477,12 +622,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_whi);
       tma_prefetch_desc(&tm_wlo);
+      if (FSRC) {
+        tma_prefetch_desc(&tm_fhi);
+        tma_prefetch_desc(&tm_flo);
+      }
       uint32_t stage = 0, phase = 0;
-      int64_t issued = 0;
+      int64_t issued = 0, fissued = 0;
       for (int64_t li = 0; li < my_tiles; li++) {
         bool ok = true;
+        // FSRC = 1: this tile's features into F buffer b, once the tile that
+        // used it last (li - nfb) is done with it.  Issued after the tile's
+        // first W stages, which the ring can take before that.
+        auto load_features = [&]() -> bool {
+          const uint32_t b = (uint32_t)(li % L.nfb);
+          const int64_t use = li / L.nfb;
+          if (use > 0 && !mbar_wait_bounded(&f_free[b], (uint32_t)((use - 1) & 1), status,
+                                            kAbort, a.wait_ns))
+            return false;
+          const int y = (int)(((int64_t)cid + li * ncl) * kTcRows);
+          uint8_t* dst = sF + b * L.fbytes;
+          mbar_arrive_expect_tx(&f_tx[b], 2u * (uint32_t)nch * kTcChunkBytes);
+          for (int c = 0; c < nch; c++) {
+            tma_load_2d(dst + (uint32_t)c * kTcChunkBytes, &tm_fhi, c * kTcChunk, y, &f_tx[b]);
+            tma_load_2d(dst + (uint32_t)(nch + c) * kTcChunkBytes, &tm_flo, c * kTcChunk, y,
+                        &f_tx[b]);
+          }
+          fissued++;
+          return true;
+        };
+        int wi = 0;  // W loads issued for this tile
         for (int c = 0; c < nch && ok; c++)
-          for (int part = 0; part < 2 && ok; part++) {
+          for (int part = 0; part < 2 && ok; part++, wi++) {
+            if (FSRC && wi == (2 * nch < kTcStages ? 2 * nch : kTcStages)) ok = load_features();
+            if (!ok) break;
             ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, status, kAbort, a.wait_ns);
             if (!ok) break;
             mbar_arrive_expect_tx(&full[stage], kTcChunkBytes);
@@ -494,12 +666,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               phase ^= 1u;
             }
           }
+        if (ok && FSRC && wi <= kTcStages && wi == 2 * nch) ok = load_features();
         if (!ok) break;
       }
       // every load issued must have landed before the CTA may exit
       for (int s = 0; s < kTcStages && s < issued; s++) {
         const int64_t uses = (issued - s + kTcStages - 1) / kTcStages;  // loads into stage s
-        mbar_wait_bounded(&full[s], (uint32_t)((uses - 1) & 1), status, 0u, a.wait_ns);
+        mbar_wait_bounded(&full[s], (uint32_t)((uses - 1) & 1), status, 0u, a.drain_ns);
+      }
+      for (int b = 0; b < (int)L.nfb && b < fissued; b++) {
+        const int64_t uses = (fissued - b + L.nfb - 1) / L.nfb;  // feature loads into buffer b
+        mbar_wait_bounded(&f_tx[b], (uint32_t)((uses - 1) & 1), status, 0u, a.drain_ns);
       }
     }
   } else if (warp == kTcMmaWarp) {
@@ -519,6 +696,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t stage = 0, phase = 0, ndrain = 0;
       for (int64_t li = 0; li < my_tiles; li++) {
         if (!mbar_wait_bounded(f_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) break;
+        if (FSRC && !mbar_wait_bounded(&f_tx[li % L.nfb], (uint32_t)((li / L.nfb) & 1), status,
+                                       kAbort, a.wait_ns))
+          break;
         SCEM_TRACE(li, 8);
         tc_fence_after_sync();
         bool ok = true;
@@ -552,7 +732,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         SCEM_TRACE(li, 10);
         tc_fence_after_sync();
         bool ok2 = true;
-        if (MODE == kTcStats) {
+        if (kStats) {
           const bool first = li == 0;  // later tiles add onto whatever the drains left
           if (li > 0) {
             if (!mbar_wait_bounded(drained, ndrain & 1u, status, kAbort, a.wait_ns)) break;
@@ -587,11 +767,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (!ok2) break;
         mma_commit(s_done);
+        if (FSRC) mma_commit(&f_free[li % L.nfb]);
         SCEM_TRACE(li, 11);
       }
       // every MMA issued must be complete before tensor memory is released
       mma_commit(final_bar);
-      mbar_wait_bounded(final_bar, 0, status, 0u, a.wait_ns);
+      mbar_wait_bounded(final_bar, 0, status, 0u, a.drain_ns);
     }
   } else {
     // ------------------------------------------------------------ compute warps
@@ -708,11 +889,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after_sync();
         return r;
       };
-      if (li > 0 && L.nfb == 1) {
+      if (!FSRC && li > 0 && L.nfb == 1) {
         ok = wait_prev_stats();
         if (!ok) break;
       }
       uint8_t* sFc = sF + (uint32_t)(li % L.nfb) * L.fbytes;  // this tile's F buffer
+      bool bad = false, wide = false;
+      if (!FSRC) {
       // ---- X tile -> F = [x^, x^^2] as fp16 hi/lo in the swizzled layout.
       // The next tile's rows (contiguous in X) are pulled into L2 now, so that
       // its loads meet L2 rather than DRAM latency; up to 16 16-byte loads per
@@ -724,7 +907,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           prefetch_l2_bulk(reinterpret_cast<const XT*>(a.X) + (size_t)nrow0 * D,
                            (uint32_t)((size_t)nrows * D * sizeof(XT)));
       }
-      bool bad = false, wide = false;
       constexpr int kBatch = 16;
       int nbatch = 0;
       for (int u0 = t; u0 < kTcRows * G; u0 += kTcComputeThreads * kBatch) {
@@ -780,6 +962,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (t == 0) SCEM_TRACE(li, 13);
         nbatch++;
       }
+      }  // !FSRC: conversion
       if (bad) atomicOr(a.status, GMM_DEVFLAG_NONFINITE_X);
       if (wide) atomicOr(a.status, GMM_DEVFLAG_X_RANGE);
       fence_proxy_async_smem();
@@ -787,14 +970,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before_sync();
       mbar_arrive(f_full);
       if (t == 0) SCEM_TRACE(li, 3);
-      if (li > 0 && L.nfb == 2) {
+      if (li > 0 && (FSRC || L.nfb == 2)) {
         ok = wait_prev_stats();
         if (!ok) break;
       }
       // Drain the previous tiles' statistics while the E-step MMAs run (they
       // write other tensor-memory columns); this tile's statistics MMAs wait
       // for it.
-      if (MODE == kTcStats && li > 0) {
+      if (kStats && li > 0) {
         ok = drain((li % a.drain_tiles) == 0, li);
         if (t == 0) SCEM_TRACE(li, 2);
         if (!ok) break;
@@ -936,7 +1119,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (t == 0) SCEM_TRACE(li, 5);
       float se = 0.f;
-      if (mx > -INFINITY) {
+      // hard EM: the first column of the thread's largest log-joint, as a
+      // component index (INT_MAX when none is finite)
+      int own_arg = INT_MAX;
+      if (kHard) {
+        float best = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 64; j++)
+          if (e[j] > best) {
+            best = e[j];
+            own_arg = k0 + col0 + j;
+          }
+        se = __int_as_float(own_arg);  // exchanged in place of the sum-exp
+      } else if (mx > -INFINITY) {
+        if (MODE == kTcTopm) {
+          // the thread's ncand largest log-joints (ties to the lower index),
+          // kept sorted in registers, before they become exponentials
+          float cv[kTcCand];
+          int ci[kTcCand];
+#pragma unroll
+          for (int q = 0; q < kTcCand; q++) {
+            cv[q] = -INFINITY;
+            ci[q] = INT_MAX;
+          }
+#pragma unroll
+          for (int j = 0; j < 64; j++) {
+            float v = e[j];
+            int ix = k0 + col0 + j;
+            if (v > cv[kTcCand - 1]) {
+#pragma unroll
+              for (int q = 0; q < kTcCand; q++)
+                if (v > cv[q]) {  // strictly larger: equal values keep the lower index first
+                  const float tv = cv[q];
+                  const int ti = ci[q];
+                  cv[q] = v;
+                  ci[q] = ix;
+                  v = tv;
+                  ix = ti;
+                }
+            }
+          }
+          if (row0 + row < a.N) {
+            float2* dst = a.cand + ((size_t)(row0 + row) * (ngrp * (uint32_t)C * 2u) +
+                                    ((grp * (uint32_t)C + rank) * 2u + (uint32_t)hf)) *
+                                       (size_t)a.ncand;
+#pragma unroll
+            for (int q = 0; q < kTcCand; q++)
+              if (q < a.ncand) dst[q] = make_float2(cv[q], __int_as_float(ci[q]));
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 64; j++) {
           e[j] = __expf(e[j] - mx);
@@ -947,33 +1178,79 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // row past N): its responsibilities are exactly 0, not -inf * 0
 #pragma unroll
         for (int j = 0; j < 64; j++) e[j] = 0.f;
+        if (MODE == kTcTopm && row0 + row < a.N) {
+          float2* dst = a.cand + ((size_t)(row0 + row) * (ngrp * (uint32_t)C * 2u) +
+                                  ((grp * (uint32_t)C + rank) * 2u + (uint32_t)hf)) *
+                                     (size_t)a.ncand;
+          for (int q = 0; q < a.ncand; q++) dst[q] = make_float2(-INFINITY, __int_as_float(INT_MAX));
+        }
       }
-      // every (CTA, column half) contributes one (max, sum-exp) partial per row
-      const uint32_t par = (uint32_t)(li & 1);
-      const uint32_t my_x = smem_u32(&xchg[((par * C + rank) * 2 + hf) * kTcRows + row]);
-      for (int r2 = 0; r2 < C; r2++) st_cluster_f32x2(map_to_rank(my_x, r2), mx, se);
-      __syncwarp();  // the warp's stores happen before lane 0's release-arrive
-      if (lane == 0) {
-        const uint32_t xb = smem_u32(&xbar[par]);
-        for (int r2 = 0; r2 < C; r2++) mbar_arrive_cluster(map_to_rank(xb, r2));
-      }
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&xbar[par], (uint32_t)((li >> 1) & 1),
-                                                     status, kAbort, a.wait_ns, true));
-      if (!ok) break;
-      if (t == 0) SCEM_TRACE(li, 6);
-      float M = -INFINITY;
-      for (int j = 0; j < 2 * C; j++) M = fmaxf(M, xchg[(par * C * 2 + j) * kTcRows + row].x);
-      float S = 0.f;
-      for (int j = 0; j < 2 * C; j++) {
-        const float2 p = xchg[(par * C * 2 + j) * kTcRows + row];
-        if (p.x > -INFINITY) S += p.y * __expf(p.x - M);
-      }
-      const float lse = M + __logf(S);
       const bool valid = row0 + row < a.N;
-      if (valid && rank == 0 && hf == 0) ll += (double)lse;
-      const float scale = (valid && mx > -INFINITY) ? __expf(mx - lse) * kTcRScale : 0.f;
+      float M = -INFINITY, S = 0.f;
+      int win = INT_MAX;  // hard EM: the row's component
+      // (max, sum-exp) partials combine as max and the sum rescaled to it;
+      // (max, index) partials as max and the lowest index attaining it
+      auto combine = [&](const float2 p) {
+        if (kHard) {
+          const int ix = __float_as_int(p.y);
+          if (p.x > M || (p.x == M && ix < win)) win = ix;
+          M = fmaxf(M, p.x);
+        } else {
+          M = fmaxf(M, p.x);
+        }
+      };
+      if ((kStats || MODE == kTcTopm) && ngrp > 1) {
+        // The row's partials of every group, from the partial pass over the
+        // same rows, combined in group order: the same value in every
+        // cluster, so the responsibilities of all groups sum to one.
+        const float2* pr = a.part + (size_t)(valid ? row0 + row : 0) * ngrp;
+        for (uint32_t g2 = 0; g2 < ngrp; g2++) combine(pr[g2]);
+        if (!kHard)
+          for (uint32_t g2 = 0; g2 < ngrp; g2++) {
+            const float2 p = pr[g2];
+            if (p.x > -INFINITY) S += p.y * __expf(p.x - M);
+          }
+      } else {
+        // every (CTA, column half) contributes one (max, sum-exp) partial per row
+        const uint32_t par = (uint32_t)(li & 1);
+        const uint32_t my_x = smem_u32(&xchg[((par * C + rank) * 2 + hf) * kTcRows + row]);
+        for (int r2 = 0; r2 < C; r2++) st_cluster_f32x2(map_to_rank(my_x, r2), mx, se);
+        __syncwarp();  // the warp's stores happen before lane 0's release-arrive
+        if (lane == 0) {
+          const uint32_t xb = smem_u32(&xbar[par]);
+          for (int r2 = 0; r2 < C; r2++) mbar_arrive_cluster(map_to_rank(xb, r2));
+        }
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&xbar[par], (uint32_t)((li >> 1) & 1),
+                                                       status, kAbort, a.wait_ns, true));
+        if (!ok) break;
+        if (t == 0) SCEM_TRACE(li, 6);
+        for (int j = 0; j < 2 * C; j++) combine(xchg[(par * C * 2 + j) * kTcRows + row]);
+        if (!kHard)
+          for (int j = 0; j < 2 * C; j++) {
+            const float2 p = xchg[(par * C * 2 + j) * kTcRows + row];
+            if (p.x > -INFINITY) S += p.y * __expf(p.x - M);
+          }
+        if (kPartial && valid && rank == 0 && hf == 0)
+          a.part[(size_t)(row0 + row) * ngrp + grp] =
+              make_float2(M, kHard ? __int_as_float(win) : S);
+      }
+      // soft: the row's log-sum-exp; hard: its largest log-joint
+      const float lse = kHard ? M : M + __logf(S);
+      if (MODE == kTcTopm && valid && rank == 0 && hf == 0 && grp == 0)
+        a.rowst[row0 + row] = make_float2(M, S);
+      if (!kPartial && MODE != kTcTopm && valid && rank == 0 && hf == 0 && grp == 0) {
+        ll += (double)lse;
+        if (kHard && a.labels) a.labels[row0 + row] = win < K ? win : -1;
+      }
+      float scale = (valid && mx > -INFINITY) ? __expf(mx - lse) * kTcRScale : 0.f;
+      if (kHard) {
+        // one-hot: exactly 2^15 in the winning column, zero elsewhere
+#pragma unroll
+        for (int j = 0; j < 64; j++) e[j] = (k0 + col0 + j == win) ? 1.f : 0.f;
+        scale = valid ? kTcRScale : 0.f;
+      }
       const int hr = row >> 6, rr = row & 63;  // which 64-row half of r^, row within it
-      if (MODE == kTcStats) {
+      if (kStats) {
         if (hr == 1) {
           // the first half's MMAs must be done with the buffer
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(r_free, (uint32_t)(li & 1), status,
@@ -1001,23 +1278,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // data units from X (no cancellation however narrow the dimension),
       // while the statistics MMAs run.  Only rows with a finite log-joint for
       // the component contribute: the few near it.  (X, not F: F may already
-      // hold the next tile once the statistics MMAs are done.)
-      if (MODE == kTcStats && (sm0 | sm1)) {
+      // hold the next tile once the statistics MMAs are done.)  They go into
+      // the shared fixed-point area (kTcDirScale), so the order in which rows
+      // and clusters add them does not change the sums.
+      if (kStats && (sm0 | sm1)) {
         const int nsh = shl[0];
         const XT* xrow = reinterpret_cast<const XT*>(a.X) + (size_t)(valid ? row0 + row : 0) * D;
-        double* dir = slot + ll_index + 1;  // [2D x K] after the LL
+        const size_t kp = (size_t)a.Kpad;
         for (int si = 0; si < nsh; si++) {
           const int j = shl[1 + si] & 255, ns = shl[1 + si] >> 8;
           if ((j >> 6) != hf) continue;
           const float l = tmem_ld1(tL + lane_base + (uint32_t)j);  // the finished log-joint
-          const double r = (valid && l > -INFINITY) ? (double)__expf(l - lse) : 0.0;
+          const double r = !(valid && l > -INFINITY) ? 0.0
+                           : kHard ? (k0 + j == win ? 1.0 : 0.0)
+                                   : (double)__expf(l - lse);
           if (r > 0.0) {
             const size_t base = (size_t)(k0 + j) * D;
+            unsigned long long* q = a.dirq + (k0 + j);
             for (int i = 0; i < ns; i++) {
               const int d = min((int)a.perm[base + i], D - 1);
-              const double dx = (double)load1<XT>(xrow, d) - (double)a.muh[base + i];
-              atomicAdd(dir + (size_t)i * K + (k0 + j), r * dx);
-              atomicAdd(dir + (size_t)(D + i) * K + (k0 + j), r * dx * dx);
+              const double p = (double)a.ph[base + i];  // 1/var of this dimension
+              const double u = ((double)load1<XT>(xrow, d) - (double)a.muh[base + i]) * sqrt(p);
+              const double ru = r * u * kTcDirScale;
+              fixed_add(q + (size_t)i * kp, q + (size_t)(D + i) * kp, ru);
+              fixed_add(q + (size_t)(2 * D + i) * kp, q + (size_t)(3 * D + i) * kp, ru * u);
             }
           }
         }
@@ -1028,7 +1312,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(s_done, (uint32_t)((my_tiles - 1) & 1),
                                                      status, kAbort, a.wait_ns));
       tc_fence_after_sync();
-      if (ok && MODE == kTcStats) ok = drain(true, my_tiles);
+      if (ok && kStats) ok = drain(true, my_tiles);
     }
     // LL of this CTA's rows (rank 0 of each cluster, column half 0): fixed-order sum
     ll = warp_sum(ll);
@@ -1036,10 +1320,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
     if (lane == 0) red[warp] = ok ? ll : 0.0;
     const bool met = rendezvous();
-    if (t == 0 && rank == 0) {
+    if (!kPartial && MODE != kTcTopm && t == 0 && rank == 0) {
       double s = 0.0;
       for (int w = 0; w < 8; w++) s += red[w];
-      slot[ll_index] = (ok && met) ? s : 0.0;
+      slot[ll_index] = (a.accumulate ? slot[ll_index] : 0.0) + ((ok && met) ? s : 0.0);
     }
   }
 
@@ -1125,7 +1409,7 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     float* __restrict__ muh, float* __restrict__ ph, int* __restrict__ precise_out,
     float* __restrict__ ci_out, uint8_t* __restrict__ perm_out, float* __restrict__ mhp_out,
     float* __restrict__ php_out, uint32_t* __restrict__ pmask_out, uint8_t* __restrict__ rank_out,
-    unsigned int* status) {
+    unsigned long long* __restrict__ dirq, unsigned int* status) {
   __shared__ double mh_s[kTcMaxD], vh_s[kTcMaxD], kd_s[kTcMaxD], ksort[kTcMaxD];
   __shared__ int rank_s[kTcMaxD];
   __shared__ double wv[kTcChunk * kTcMaxChunks];  // Fpad <= 256
@@ -1135,6 +1419,8 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
   const int k = blockIdx.x;
   const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
   const float wk = k < K ? w[k] : 0.f;
+  // the fused pass adds this component's split-dimension moments onto zero
+  for (int q = threadIdx.x; q < 4 * D; q += blockDim.x) dirq[(size_t)q * gridDim.x + k] = 0ull;
   const bool live = k < K && wk > 0.f;
   auto block_sum = [&](double v) -> double {
     v = warp_sum(v);
@@ -1274,18 +1560,25 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
   if (bad) atomicOr(status, GMM_DEVFLAG_BAD_PARAMS);
 }
 
+// Value of a fixed-point pair of sums (see kTcDirScale), in units of 2^-32.
+__device__ __forceinline__ double fixed_value(unsigned long long hi, unsigned long long lo) {
+  return (double)(long long)hi * kTcDirScale + (double)lo;
+}
+
 // Fixed-order fp64 sum of the per-cluster slots into the canonical
 // statistics buffer [ N_k | A | B | LL ] (component-major, moments about the
 // input means mu, data units).  The slots hold N' = 2^15 N_k and
 // S1' = 2^15 sum r x^, S2' = 2^15 sum r x^^2 with x^ = (x - m)/s, so with
 // dm = mu - m:  A = s S1 - dm N,  B = s^2 S2 - 2 s dm S1 + dm^2 N.  A split
-// dimension (perm position below nsplit_k) takes A and B from the direct-form
-// moments instead.
+// dimension (perm position below nsplit_k) takes A and B from the fixed-point
+// direct-form moments instead, scaled back by sigma = 1/sqrt(ph) with the same
+// stored ph the fused pass divided by.
 __global__ void __launch_bounds__(256) tc_reduce_stats_kernel(
-    int D, int K, const float* __restrict__ m, const float* __restrict__ sc,
+    int D, int K, int Kpad, const float* __restrict__ m, const float* __restrict__ sc,
     const float* __restrict__ mu, const uint8_t* __restrict__ rank,
-    const int* __restrict__ nsplit, const double* __restrict__ slots, size_t slot_stride,
-    int nslots, double* __restrict__ stats) {
+    const int* __restrict__ nsplit, const float* __restrict__ ph,
+    const unsigned long long* __restrict__ dirq, const double* __restrict__ slots,
+    size_t slot_stride, int nslots, int G, int group_comps, double* __restrict__ stats) {
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t KD = (size_t)K * D;
   if (i == 0) {
@@ -1296,7 +1589,8 @@ __global__ void __launch_bounds__(256) tc_reduce_stats_kernel(
   if (i >= KD) return;
   const int d = (int)(i / K), k = (int)(i - (size_t)d * K);
   double nks = 0.0, s1 = 0.0, s2 = 0.0;
-  for (int p = 0; p < nslots; p++) {
+  // the slots of the clusters that served component k's group: g, g + G, ...
+  for (int p = k / group_comps; p < nslots; p += G) {
     const double* s = slots + (size_t)p * slot_stride;
     nks += s[(size_t)(2 * D) * K + k];
     s1 += s[(size_t)d * K + k];
@@ -1309,19 +1603,236 @@ __global__ void __launch_bounds__(256) tc_reduce_stats_kernel(
   if (d == 0) stats[k] = n;
   const int r = rank[(size_t)k * D + d];
   if (r < nsplit[k]) {
-    const size_t dir = (size_t)(2 * D + 1) * K + 1;
-    double A = 0.0, B = 0.0;
-    for (int p = 0; p < nslots; p++) {
-      const double* s = slots + (size_t)p * slot_stride + dir;
-      A += s[(size_t)r * K + k];
-      B += s[(size_t)(D + r) * K + k];
-    }
-    stats[K + (size_t)k * D + d] = A;
-    stats[K + KD + (size_t)k * D + d] = B;
+    const size_t kp = (size_t)Kpad;
+    const double p = (double)ph[(size_t)k * D + r];  // 1/var, perm order
+    const double a1 = fixed_value(dirq[(size_t)r * kp + k], dirq[(size_t)(D + r) * kp + k]);
+    const double b1 =
+        fixed_value(dirq[(size_t)(2 * D + r) * kp + k], dirq[(size_t)(3 * D + r) * kp + k]);
+    stats[K + (size_t)k * D + d] = a1 / kTcDirScale / sqrt(p);
+    stats[K + KD + (size_t)k * D + d] = b1 / kTcDirScale / p;
     return;
   }
   stats[K + (size_t)k * D + d] = sd * S1 - dm * n;
   stats[K + KD + (size_t)k * D + d] = sd * sd * S2 - 2.0 * sd * dm * S1 + dm * dm * n;
+}
+
+// Features of a chunk of rows for the two-pass form: the same x^ = (x - m)/s,
+// clamp and fp16 hi/lo split as the fused kernel's own conversion, written
+// row-major [rows x Fpad] (x^ in features 0..D-1, x^^2 in D..2D-1, zeros
+// after), to be read back tile by tile by TMA in the 128-byte-swizzled
+// shared-memory layout.  Raises the same status bits.
+template <typename XT>
+__global__ void __launch_bounds__(256) tc_convert_kernel(
+    const XT* __restrict__ X, int64_t rows, int D, int Fpad, const float* __restrict__ m,
+    const float* __restrict__ isc, __half* __restrict__ fhi, __half* __restrict__ flo,
+    unsigned int* status) {
+  const int G4 = D / 4;
+  const int64_t items = rows * G4;
+  bool bad = false, wide = false;
+  for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < items;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = u / G4;
+    const int g = (int)(u - n * G4);
+    float xv[4];
+    load4<XT>(X, (size_t)n * D + 4 * g, xv);
+    float x[4];
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+      if (!isfinite(xv[j])) bad = true;
+      x[j] = (xv[j] - m[4 * g + j]) * isc[4 * g + j];
+      if (fabsf(x[j]) > kTcXMax) {
+        wide = true;
+        x[j] = copysignf(kTcXMax, x[j]);
+      }
+    }
+    uint32_t hx[2], lx[2], hs[2], ls[2];
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+      split_half2(x[2 * h], x[2 * h + 1], hx[h], lx[h]);
+      split_half2(x[2 * h] * x[2 * h], x[2 * h + 1] * x[2 * h + 1], hs[h], ls[h]);
+    }
+    const size_t o1 = (size_t)n * Fpad + 4 * g, o2 = o1 + D;
+    *reinterpret_cast<uint2*>(fhi + o1) = make_uint2(hx[0], hx[1]);
+    *reinterpret_cast<uint2*>(flo + o1) = make_uint2(lx[0], lx[1]);
+    *reinterpret_cast<uint2*>(fhi + o2) = make_uint2(hs[0], hs[1]);
+    *reinterpret_cast<uint2*>(flo + o2) = make_uint2(ls[0], ls[1]);
+  }
+  // padding features read as zero in every MMA
+  const int P4 = (Fpad - 2 * D) / 4;
+  for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < rows * P4;
+       u += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = u / P4;
+    const size_t o = (size_t)n * Fpad + 2 * D + 4 * (u - n * P4);
+    *reinterpret_cast<uint2*>(fhi + o) = make_uint2(0u, 0u);
+    *reinterpret_cast<uint2*>(flo + o) = make_uint2(0u, 0u);
+  }
+  if (bad) atomicOr(status, GMM_DEVFLAG_NONFINITE_X);
+  if (wide) atomicOr(status, GMM_DEVFLAG_X_RANGE);
+}
+
+// Top-m from the fused pass's candidates, one thread per row.  The row's
+// P = G C 2 candidate lists (each sorted by tensor-core log-joint, ties to the
+// lower index) are merged into its nc best.  Their log-joints are recomputed
+// in direct form in fp32, l_k = c0_k - 1/2 sum_d (x_d - mu_kd)^2 iv_kd with
+// c0_k = log pi_k - 1/2 sum_d log(2 pi var_kd) and iv = 1/var, and exchanged
+// for their tensor-core terms in the row's sum-exp (the candidates carry
+// almost all of a row's mass, so the normalisation comes out as precise as
+// the direct form).  r_k = exp(l_k - lse); the candidates are ordered by r,
+// descending, equal r to the lower index, and the first m written.  A row
+// with fewer than m finite candidates is completed, r = 0, by the lowest
+// indices not yet taken (the same order the definition gives).
+template <typename XT>
+__global__ void __launch_bounds__(128) tc_topm_refine_kernel(
+    const XT* __restrict__ X, int64_t rows, int D, int K, int P, int nc, int m,
+    const float2* __restrict__ cand, const float2* __restrict__ rowst,
+    const float* __restrict__ mu, const float* __restrict__ iv, const float* __restrict__ c0,
+    int32_t* __restrict__ idx_out, float* __restrict__ resp_out) {
+  const int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= rows) return;
+  float bv[kTcCand], bl[kTcCand];
+  int bi[kTcCand];
+#pragma unroll
+  for (int q = 0; q < kTcCand; q++) {
+    bv[q] = -INFINITY;
+    bi[q] = INT_MAX;
+  }
+  const float2* cr = cand + (size_t)n * P * nc;
+  for (int i = 0; i < P * nc; i++) {
+    const float2 c = cr[i];
+    float v = c.x;
+    int ix = __float_as_int(c.y);
+    if (!(v > -INFINITY)) continue;
+    // insert into the sorted best nc: (value desc, index asc)
+#pragma unroll
+    for (int q = 0; q < kTcCand; q++)
+      if (q < nc && (v > bv[q] || (v == bv[q] && ix < bi[q]))) {
+        const float tv = bv[q];
+        const int ti = bi[q];
+        bv[q] = v;
+        bi[q] = ix;
+        v = tv;
+        ix = ti;
+      }
+  }
+  const float2 st = rowst[n];
+  const float M = st.x;
+  float S = st.y;
+  const XT* xr = X + (size_t)n * D;
+#pragma unroll
+  for (int q = 0; q < kTcCand; q++) {
+    bl[q] = -INFINITY;
+    if (q < nc && bi[q] < K) {
+      const int k = bi[q];
+      const float* mk = mu + (size_t)k * D;
+      const float* ik = iv + (size_t)k * D;
+      float qd = 0.f;
+      for (int d = 0; d < D; d++) {
+        const float e = load1<XT>(xr, d) - mk[d];
+        qd = fmaf(e * e, ik[d], qd);
+      }
+      bl[q] = c0[k] - 0.5f * qd;
+      S += __expf(bl[q] - M) - __expf(bv[q] - M);
+    }
+  }
+  const float lse = M + __logf(S);
+  float r[kTcCand];
+#pragma unroll
+  for (int q = 0; q < kTcCand; q++) r[q] = bl[q] > -INFINITY ? __expf(bl[q] - lse) : 0.f;
+  // order the candidates by (r desc, index asc): insertion sort of nc <= 8
+#pragma unroll
+  for (int a1 = 1; a1 < kTcCand; a1++)
+#pragma unroll
+    for (int b1 = a1; b1 > 0; b1--)
+      if (b1 < nc && (r[b1] > r[b1 - 1] || (r[b1] == r[b1 - 1] && bi[b1] < bi[b1 - 1]))) {
+        const float tr = r[b1];
+        r[b1] = r[b1 - 1];
+        r[b1 - 1] = tr;
+        const int ti = bi[b1];
+        bi[b1] = bi[b1 - 1];
+        bi[b1 - 1] = ti;
+      }
+  int32_t* io = idx_out + (size_t)n * m;
+  float* ro = resp_out + (size_t)n * m;
+  int j = 0;
+  for (int q = 0; q < nc && j < m; q++)
+    if (bi[q] < K && r[q] > 0.f) {
+      io[j] = bi[q];
+      ro[j] = r[q];
+      j++;
+    }
+  // zero responsibilities: the lowest indices not taken yet
+  for (int k = 0; j < m && k < K; k++) {
+    bool taken = false;
+    for (int q = 0; q < j; q++) taken |= io[q] == k;
+    if (!taken) {
+      io[j] = k;
+      ro[j] = 0.f;
+      j++;
+    }
+  }
+}
+
+// 1/var and c0_k = log pi_k - 1/2 sum_d log(2 pi var_kd) (-inf for pi_k = 0)
+// for the refinement, one block per component.
+__global__ void __launch_bounds__(128) tc_topm_prep_kernel(int D, const float* __restrict__ w,
+                                                           const float* __restrict__ var,
+                                                           float* __restrict__ iv,
+                                                           float* __restrict__ c0) {
+  __shared__ double red[128];
+  const int k = blockIdx.x;
+  double s = 0.0;
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    const float v = var[(size_t)k * D + d];
+    iv[(size_t)k * D + d] = 1.0f / v;
+    s += log(2.0 * M_PI * (double)v);
+  }
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int h = 64; h > 0; h >>= 1) {
+    if ((int)threadIdx.x < h) red[threadIdx.x] += red[threadIdx.x + h];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) c0[k] = w[k] > 0.f ? (float)(log((double)w[k]) - 0.5 * red[0]) : -INFINITY;
+}
+
+constexpr int kTcLseBlocks = 128;
+
+// Log-likelihood of a chunk from the groups' partials: each row's log-sum-exp
+// combined exactly as the statistics pass combines it, summed in a fixed
+// order -- rows [b*per, (b+1)*per) by block b, strided by thread, then a
+// fixed tree -- into out[b].
+__global__ void __launch_bounds__(256) tc_part_loglik_kernel(const float2* __restrict__ part,
+                                                             int64_t rows, int G,
+                                                             double* __restrict__ out) {
+  __shared__ double red[256];
+  const int64_t per = (rows + gridDim.x - 1) / gridDim.x;
+  const int64_t lo = (int64_t)blockIdx.x * per, hi = min(rows, lo + per);
+  double s = 0.0;
+  for (int64_t n = lo + threadIdx.x; n < hi; n += blockDim.x) {
+    const float2* pr = part + (size_t)n * G;
+    float M = -INFINITY, S = 0.f;
+    for (int g = 0; g < G; g++) M = fmaxf(M, pr[g].x);
+    for (int g = 0; g < G; g++) {
+      const float2 p = pr[g];
+      if (p.x > -INFINITY) S += p.y * __expf(p.x - M);
+    }
+    s += (double)(M + __logf(S));
+  }
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[blockIdx.x] = red[0];
+}
+
+// *acc (+)= sum of the kTcLseBlocks block sums, in block order.
+__global__ void tc_sum_blocks_kernel(const double* __restrict__ blocks, int first,
+                                     double* __restrict__ acc) {
+  double s = 0.0;
+  for (int b = 0; b < kTcLseBlocks; b++) s += blocks[b];
+  *acc = (first ? 0.0 : *acc) + s;
 }
 
 __global__ void tc_reduce_loglik_kernel(int D, int K, const double* __restrict__ slots,

@@ -21,16 +21,23 @@ GMM_INIT_VAR_ONE, GMM_INIT_VAR_DATA = 0, 1
 GMM_DEVFLAG_NONFINITE_X, GMM_DEVFLAG_BAD_PARAMS, GMM_DEVFLAG_WAIT_TIMEOUT = 0x1, 0x2, 0x4
 GMM_DEVFLAG_X_RANGE, GMM_DEVFLAG_BAD_INDEX = 0x8, 0x10
 
-EXPORTS = ("gmm_workspace_size", "gmm_init", "gmm_em_step", "gmm_em_step_noalloc",
+EXPORTS = ("gmm_workspace_size", "gmm_plan", "gmm_init", "gmm_init_rows", "gmm_em_step",
+           "gmm_em_step_hard", "gmm_em_step_spherical", "gmm_kmeans_step", "gmm_em_step_noalloc",
            "gmm_host_staging_size", "gmm_em_step_host",
            "gmm_estep_stats", "gmm_mstep", "gmm_fit", "gmm_loglik",
            "gmm_assign_topm", "gmm_ivf_workspace_size", "gmm_ivf_build", "gmm_device_status",
-           "gmm_trace_fused", "gmm_launch_count", "gmm_status_string")
+           "gmm_trace_fused", "gmm_set_wait_budget", "gmm_launch_count", "gmm_status_string")
 
 
 class gmm_problem(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int64), ("D", ctypes.c_int32), ("K", ctypes.c_int32),
                 ("xdtype", ctypes.c_int32), ("var_floor", ctypes.c_float)]
+
+
+class gmm_plan_info(ctypes.Structure):
+    _fields_ = [("tensor_cores", ctypes.c_int32), ("cluster_ctas", ctypes.c_int32),
+                ("groups", ctypes.c_int32), ("fit_one_launch", ctypes.c_int32),
+                ("chunk_rows", ctypes.c_int64)]
 
 
 class GmmError(RuntimeError):
@@ -54,9 +61,14 @@ def load_library(path: str = LIB_PATH):
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     PP = ctypes.POINTER(gmm_problem)
     lib.gmm_workspace_size.argtypes = [PP, ctypes.POINTER(SZ)]
-    lib.gmm_init.argtypes = [PP, P, ctypes.POINTER(I64), I32, P, P, P, P, SZ, P]
+    lib.gmm_plan.argtypes = [PP, ctypes.POINTER(gmm_plan_info)]
+    lib.gmm_init.argtypes = [PP, P, ctypes.c_uint64, I32, P, P, P, P, SZ, P]
+    lib.gmm_init_rows.argtypes = [PP, P, ctypes.POINTER(I64), I32, P, P, P, P, SZ, P]
     lib.gmm_em_step.argtypes = [PP, P, P, P, P, P, P, SZ, P]
     lib.gmm_em_step_noalloc.argtypes = [PP, P, P, P, P, P, P, P]
+    lib.gmm_em_step_hard.argtypes = [PP, P, P, P, P, P, P, P, SZ, P]
+    lib.gmm_em_step_spherical.argtypes = [PP, P, P, P, P, P, P, SZ, P]
+    lib.gmm_kmeans_step.argtypes = [PP, P, P, P, P, P, SZ, P]
     lib.gmm_host_staging_size.argtypes = [PP, I64, ctypes.POINTER(SZ)]
     lib.gmm_em_step_host.argtypes = [PP, P, I64, P, SZ, P, P, P, P, P, SZ, P, P]
     lib.gmm_estep_stats.argtypes = [PP, P, P, P, P, P, P, SZ, P]
@@ -68,6 +80,7 @@ def load_library(path: str = LIB_PATH):
     lib.gmm_ivf_build.argtypes = [I64, I32, I32, P, P, ctypes.c_float, P, P, I64, P, SZ, P]
     lib.gmm_device_status.argtypes = [P, SZ, P, ctypes.POINTER(ctypes.c_uint32), I32]
     lib.gmm_trace_fused.argtypes = [P, P]
+    lib.gmm_set_wait_budget.argtypes = [ctypes.c_uint64]
     lib.gmm_launch_count.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
     lib.gmm_status_string.argtypes = [ctypes.c_int]
     lib.gmm_status_string.restype = ctypes.c_char_p
@@ -119,6 +132,13 @@ def gmm_workspace_size(p: gmm_problem) -> int:
     return int(n.value)
 
 
+def gmm_plan(p: gmm_problem) -> dict:
+    """How the library runs problem p on the current device."""
+    info = gmm_plan_info()
+    _check(load_library().gmm_plan(ctypes.byref(p), ctypes.byref(info)), "gmm_plan")
+    return {f: int(getattr(info, f)) for f, _ in gmm_plan_info._fields_}
+
+
 def workspace(p: gmm_problem, device=None) -> torch.Tensor:
     """A zero-filled device workspace for problem p (caller-owned, reusable)."""
     return torch.zeros(gmm_workspace_size(p), dtype=torch.uint8, device=device or "cuda")
@@ -128,17 +148,32 @@ def _ws(p, ws, device):
     return workspace(p, device) if ws is None else ws
 
 
-def gmm_init(X, rows, K, init_var=GMM_INIT_VAR_DATA, var_floor=1e-6, ws=None, stream=None):
+def _init_out(X, K):
+    w = torch.empty(K, dtype=torch.float32, device=X.device)
+    mu = torch.empty(K, X.shape[1], dtype=torch.float32, device=X.device)
+    return w, mu, torch.empty_like(mu)
+
+
+def gmm_init(X, seed, K, init_var=GMM_INIT_VAR_DATA, var_floor=1e-6, ws=None, stream=None):
+    """Initial (w, mu, var): means at K distinct rows of X chosen from `seed`."""
+    p = problem_for(X, K, var_floor)
+    ws = _ws(p, ws, X.device)
+    w, mu, var = _init_out(X, K)
+    _check(load_library().gmm_init(ctypes.byref(p), _ptr(X), int(seed) & ((1 << 64) - 1),
+                                   int(init_var), _ptr(w), _ptr(mu), _ptr(var), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "gmm_init")
+    return w, mu, var
+
+
+def gmm_init_rows(X, rows, K, init_var=GMM_INIT_VAR_DATA, var_floor=1e-6, ws=None, stream=None):
     """Initial (w, mu, var) from the K chosen rows of X (host int64 indices)."""
     p = problem_for(X, K, var_floor)
     ws = _ws(p, ws, X.device)
     rows = (ctypes.c_int64 * K)(*[int(r) for r in rows])
-    w = torch.empty(K, dtype=torch.float32, device=X.device)
-    mu = torch.empty(K, X.shape[1], dtype=torch.float32, device=X.device)
-    var = torch.empty_like(mu)
-    _check(load_library().gmm_init(ctypes.byref(p), _ptr(X), rows, int(init_var), _ptr(w),
-                                   _ptr(mu), _ptr(var), _ptr(ws), ws.numel(), _stream(stream)),
-           "gmm_init")
+    w, mu, var = _init_out(X, K)
+    _check(load_library().gmm_init_rows(ctypes.byref(p), _ptr(X), rows, int(init_var), _ptr(w),
+                                        _ptr(mu), _ptr(var), _ptr(ws), ws.numel(),
+                                        _stream(stream)), "gmm_init_rows")
     return w, mu, var
 
 
@@ -149,6 +184,34 @@ def gmm_em_step(X, w, mu, var, loglik=None, var_floor=1e-6, ws=None, stream=None
     _check(load_library().gmm_em_step(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu), _ptr(var),
                                       _ptr(loglik), _ptr(ws), ws.numel(), _stream(stream)),
            "gmm_em_step")
+
+
+def gmm_em_step_hard(X, w, mu, var, labels=None, loglik=None, var_floor=1e-6, ws=None,
+                     stream=None):
+    """One classification-EM step in place; labels (N int32) and loglik optional outputs."""
+    p = problem_for(X, w.numel(), var_floor)
+    ws = _ws(p, ws, X.device)
+    _check(load_library().gmm_em_step_hard(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu),
+                                           _ptr(var), _ptr(labels), _ptr(loglik), _ptr(ws),
+                                           ws.numel(), _stream(stream)), "gmm_em_step_hard")
+
+
+def gmm_em_step_spherical(X, w, mu, s2, loglik=None, var_floor=1e-6, ws=None, stream=None):
+    """One soft EM step in place with covariances s2_k * I (s2: K floats)."""
+    p = problem_for(X, w.numel(), var_floor)
+    ws = _ws(p, ws, X.device)
+    _check(load_library().gmm_em_step_spherical(ctypes.byref(p), _ptr(X), _ptr(w), _ptr(mu),
+                                                _ptr(s2), _ptr(loglik), _ptr(ws), ws.numel(),
+                                                _stream(stream)), "gmm_em_step_spherical")
+
+
+def gmm_kmeans_step(X, centers, labels=None, inertia=None, ws=None, stream=None):
+    """One Lloyd step in place on centers (K x D); optional labels (N int32) and inertia."""
+    p = problem_for(X, centers.shape[0])
+    ws = _ws(p, ws, X.device)
+    _check(load_library().gmm_kmeans_step(ctypes.byref(p), _ptr(X), _ptr(centers), _ptr(labels),
+                                          _ptr(inertia), _ptr(ws), ws.numel(), _stream(stream)),
+           "gmm_kmeans_step")
 
 
 _copy_streams = {}
@@ -322,6 +385,11 @@ def gmm_trace_fused(start=None, stop=None):
             e.record()  # torch creates the CUDA event lazily, on its first record
     _check(load_library().gmm_trace_fused(ctypes.c_void_p(start.cuda_event),
                                           ctypes.c_void_p(stop.cuda_event)), "gmm_trace_fused")
+
+
+def gmm_set_wait_budget(ns=0):
+    """Budget of every device-side wait in nanoseconds (0: the default, one second)."""
+    _check(load_library().gmm_set_wait_budget(int(ns)), "gmm_set_wait_budget")
 
 
 def gmm_launch_count() -> int:

@@ -60,8 +60,8 @@ int main(void) {
     goto done;
   }
   cudaMemcpy(dX, X, sizeof(float) * NPTS * DIM, cudaMemcpyHostToDevice);
-  if (check(gmm_init(&p, dX, rows, GMM_INIT_VAR_DATA, (float*)dw, (float*)dmu, (float*)dvar, ws,
-                     ws_bytes, NULL), "gmm_init") ||
+  if (check(gmm_init_rows(&p, dX, rows, GMM_INIT_VAR_DATA, (float*)dw, (float*)dmu, (float*)dvar, ws,
+                     ws_bytes, NULL), "gmm_init_rows") ||
       check(gmm_fit(&p, dX, 10, (float*)dw, (float*)dmu, (float*)dvar, (double*)dll, ws,
                     ws_bytes, NULL), "gmm_fit") ||
       check(gmm_device_status(ws, ws_bytes, NULL, NULL, 1), "gmm_device_status")) {

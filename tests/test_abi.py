@@ -27,7 +27,9 @@ def declared_functions():
 
 def test_header_declares_the_calls():
     names = declared_functions()
-    for n in ("gmm_init", "gmm_em_step", "gmm_em_step_noalloc", "gmm_estep_stats", "gmm_mstep",
+    for n in ("gmm_plan", "gmm_init", "gmm_init_rows", "gmm_em_step_hard",
+              "gmm_em_step_spherical", "gmm_kmeans_step", "gmm_em_step", "gmm_em_step_noalloc",
+              "gmm_estep_stats", "gmm_mstep", "gmm_set_wait_budget",
               "gmm_fit", "gmm_loglik",
               "gmm_assign_topm", "gmm_ivf_workspace_size", "gmm_ivf_build",
               "gmm_host_staging_size", "gmm_em_step_host",
@@ -87,12 +89,18 @@ def test_topm_and_init_argument_checks(lib):
                                  P(256), 1 << 30, P(0))
         assert rc == G.GMM_ERR_INVALID_ARG, m
     rows = (ctypes.c_int64 * 3)(0, 5, 10)  # 10 is out of range for N = 10
-    rc = lib.gmm_init(ctypes.byref(p), P(16), rows, 1, P(16), P(16), P(16), P(256), 1 << 30, P(0))
+    rc = lib.gmm_init_rows(ctypes.byref(p), P(16), rows, 1, P(16), P(16), P(16), P(256), 1 << 30, P(0))
     assert rc == G.GMM_ERR_INVALID_ARG
     rows = (ctypes.c_int64 * 3)(0, 5, 9)
-    rc = lib.gmm_init(ctypes.byref(p), P(16), rows, 2, P(16), P(16), P(16), P(256), 1 << 30, P(0))
+    rc = lib.gmm_init_rows(ctypes.byref(p), P(16), rows, 2, P(16), P(16), P(16), P(256), 1 << 30, P(0))
     assert rc == G.GMM_ERR_INVALID_ARG
     rc = lib.gmm_fit(ctypes.byref(p), P(16), -1, P(16), P(16), P(16), P(0), P(256), 1 << 30, P(0))
+    assert rc == G.GMM_ERR_INVALID_ARG
+    # seeded init: K distinct rows need K <= N; the variance mode is checked too
+    few = G.problem(2, 4, 3)
+    rc = lib.gmm_init(ctypes.byref(few), P(16), 5, 1, P(16), P(16), P(16), P(256), 1 << 30, P(0))
+    assert rc == G.GMM_ERR_INVALID_ARG
+    rc = lib.gmm_init(ctypes.byref(p), P(16), 5, 2, P(16), P(16), P(16), P(256), 1 << 30, P(0))
     assert rc == G.GMM_ERR_INVALID_ARG
 
 

@@ -40,7 +40,7 @@ def _setup(G, name, N, K):
     Xh = Xh.pin_memory()
     Xd = Xh.cuda()
     mode = G.GMM_INIT_VAR_ONE if wl.var_init == "one" else G.GMM_INIT_VAR_DATA
-    w, mu, var = G.gmm_init(Xd, synth.init_rows(N, K, wl.init_seed), K, mode, wl.var_floor)
+    w, mu, var = G.gmm_init_rows(Xd, synth.init_rows(N, K, wl.init_seed), K, mode, wl.var_floor)
     return wl, Xh, Xd, synth.x_as_f64(wl, X), (w, mu, var)
 
 
@@ -51,6 +51,7 @@ def _setup(G, name, N, K):
     ("gauss8", 1_000, 8, 1_000),         # exactly one chunk
     ("gauss8", 999, 8, 5_000),           # chunk larger than N
     ("sphere768", 2_003, 1024, 500),     # the CUDA-core kernel
+    ("gauss4096", 20_000, 4096, 6_000),  # component groups: two passes per host chunk
 ])
 def test_host_streamed_step_matches_oracle(G, name, N, K, chunk):
     import torch

@@ -49,7 +49,7 @@ def test_noalloc_matches_workspace_step_twice(G, name, N):
         Xd = torch.from_numpy(X).cuda()
     ws = G.workspace(G.problem_for(Xd, wl.K, wl.var_floor))
     mode = G.GMM_INIT_VAR_ONE if wl.var_init == "one" else G.GMM_INIT_VAR_DATA
-    w, mu, var = G.gmm_init(Xd, synth.init_rows(N, wl.K, wl.init_seed), wl.K, mode,
+    w, mu, var = G.gmm_init_rows(Xd, synth.init_rows(N, wl.K, wl.init_seed), wl.K, mode,
                             wl.var_floor, ws=ws)
     ref = [w.clone(), mu.clone(), var.clone()]
     got = [w.clone(), mu.clone(), var.clone()]
