@@ -194,11 +194,11 @@ std::atomic<uint64_t> g_wait_budget_ns{kWaitBudgetNs};  // gmm_set_wait_budget
 gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const float* var,
                    char* ws, const TcLayout& T, cudaStream_t st) {
   float* m = (float*)(ws + T.m);
-  tc_center_kernel<<<(p->D + 127) / 128, 128, 0, st>>>(p->D, p->K, w, mu, var, m,
+  tc_center_kernel<<<p->D, 256, 0, st>>>(p->D, p->K, w, mu, var, m,
                                                        (float*)(ws + T.isc), (float*)(ws + T.sc));
   tc_prep_w_kernel<<<T.Kpad, 128, 0, st>>>(
       p->N, p->D, p->K, T.Fpad, w, mu, var, m, (const float*)(ws + T.sc), (__half*)(ws + T.whi),
-      (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.wsc), (int*)(ws + T.sharp),
+      (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.wsc), (int*)(ws + T.ndir),
       (int*)(ws + T.nsplit), (float*)(ws + T.muh), (float*)(ws + T.ph), (int*)(ws + T.precise),
       (float*)(ws + T.ci), (uint8_t*)(ws + T.perm), (float*)(ws + T.mhp), (float*)(ws + T.php),
       (uint32_t*)(ws + T.pmask), (uint8_t*)(ws + T.rank), (unsigned long long*)(ws + T.dirq),
@@ -298,7 +298,7 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, int64_t N, char* ws, c
   args.c = (const float*)(ws + T.c);
   args.ci = (const float*)(ws + T.ci);
   args.wsc = (const float*)(ws + T.wsc);
-  args.sharp = (const int*)(ws + T.sharp);
+  args.ndir = (const int*)(ws + T.ndir);
   args.nsplit = (const int*)(ws + T.nsplit);
   args.muh = (const float*)(ws + T.muh);
   args.ph = (const float*)(ws + T.ph);
@@ -425,7 +425,7 @@ gmm_status estep_stats_impl(const gmm_problem* p, const void* X, const float* w,
     if (s != GMM_OK) return s;
     tc_reduce_stats_kernel<<<blocks, 256, 0, st>>>(
         p->D, p->K, T.Kpad, (const float*)(ws + T.m), (const float*)(ws + T.sc), mu,
-        (const uint8_t*)(ws + T.rank), (const int*)(ws + T.nsplit), (const float*)(ws + T.ph),
+        (const uint8_t*)(ws + T.rank), (const int*)(ws + T.ndir), (const float*)(ws + T.ph),
         (const unsigned long long*)(ws + T.dirq), (const double*)(ws + T.slots), T.slot_stride,
         nslots, T.G, T.C * kTcComps, stats);
     return launched(1);

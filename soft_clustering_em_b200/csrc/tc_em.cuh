@@ -93,9 +93,25 @@ constexpr double kTcRhoPrecise = 64.0;  // mu^^2/var^ of a dimension above which
                                         // drain after every tile with mass
 constexpr uint32_t kTcChunkBytes = 128u * 128u;  // one [128 x 64] 16-bit operand chunk
 constexpr float kTcRScale = 32768.0f;            // r is stored as fp16(r * 2^15)
-constexpr double kTcSharpKappa = 1e7;            // split dimensions above this kappa_k ...
+// Split dimensions above this kappa_k: the expanded form's logit bias, about
+// 4e-8 kappa_k nats with the accumulator start value below, stays under the
+// 4e-3 nats the weight tolerance allows ...
+constexpr double kTcSharpKappa = 1e5;
 constexpr double kTcSmallKappa = 2.0e4;          // ... or above this one for a component
 constexpr double kTcSmallPoints = 50.0;          //     expecting fewer points than this
+// Dimensions whose kappa_kd = (mu^^2 + 1)/var^ exceeds this take their moments
+// in direct form (exact, fixed point) even when the contraction keeps them for
+// the logits.  The tensor-core statistics give var to a relative error of
+// about 1e-7 (mu^^2/var^) of the NEW variance (fp32 accumulation that rounds
+// toward zero, 22-bit features); on data clipped to a range, a dimension's
+// variance can shrink several-fold in one step, so the margin is wide: at 500
+// the error stays near 3e-4 even after a tenfold shrink.
+constexpr double kTcDirectKappa = 500.0;
+// Rows whose responsibility for a component is below this add nothing to its
+// direct-form moments: r (x - mu)^2 / var stays below ~2e-10 for such a row
+// (its log-joint carries -(x - mu)^2 / (2 var)), negligible next to the second
+// moment of a component holding ten or more points.
+constexpr float kTcDirRmin = 1e-12f;
 constexpr float kTcXMax = 240.0f;                // |x^| beyond this cannot be split into fp16
 // Start value of the E-step accumulator, as a multiple of Q_k = sum_d mu^^2/var^.
 // For a point the component explains, the linear K-steps add about +Q_k and
@@ -149,6 +165,10 @@ __host__ __device__ constexpr bool tc_mode_hard(int m) {
   return m == kTcHardStats || m == kTcHardPartial;
 }
 constexpr int kTcMaxGroups = 64;
+// Largest cluster of a component group when there are several (G > 1): the
+// grid must hold a whole number of clusters per group, and smaller clusters
+// pack more of the SMs into it (8-CTA clusters left a third of a B200 idle).
+constexpr int kTcGroupClusterMax = 16;
 constexpr int64_t kTcChunkRowsMax = 1 << 18;       // rows per pass with component groups
 constexpr size_t kTcChunkFBytesMax = 256u << 20;   // cap on the chunk's feature buffer
 
@@ -212,7 +232,7 @@ __host__ __device__ inline TcSmem tc_smem_layout_n(int D, int C, int nchunks, ui
   L.xchg = off;
   off += 2u * 2u * C * kTcRows * 8;  // [parity][rank][column half][row]
   L.bars = off;
-  off += 8 * (2 * kTcStages + 16);
+  off += 8 * (2 * kTcStages + 20);
   L.tslot = off;
   off += 16;
   L.total = off + 1024;  // slack for aligning the dynamic base to 1024
@@ -232,8 +252,9 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //   ci   : C*128 f32 the part of that constant the accumulator starts from, in
 //          units of the W row scale
 //   wsc  : C*128 f32 power-of-two scale of each W row
-//   sharp: C*128 int32 1 if some of the component's dimensions are summed in
-//          direct form (nsplit: C*128 int32, how many: the first nsplit of perm)
+//   ndir : C*128 int32 how many of the component's leading dimensions (in perm
+//          order) take their moments in direct form; the first nsplit of
+//          them (nsplit: C*128 int32) also leave the contraction for the logits
 //   pmask: [C*128 x Fpad/32] u32 per feature of each component, 1 if it is
 //          drained after every tile with mass (see tc_prep_w_kernel)
 //   perm : [C*128 x D] u8 dimensions of each component by decreasing
@@ -260,7 +281,7 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //   cand     : [Rt x (G C 2) x kTcCand] float2 (log-joint, index) candidates
 //   rowst    : [Rt] float2 (max, sum-exp) of each row
 struct TcLayout {
-  size_t m, isc, sc, c, ci, wsc, sharp, nsplit, precise, pmask, muh, ph, perm, rank, mhp, php, whi,
+  size_t m, isc, sc, c, ci, wsc, ndir, nsplit, precise, pmask, muh, ph, perm, rank, mhp, php, whi,
       wlo, dirq, slots, fhi, flo, part, cand, rowst, total, slot_stride;
   int C, G, nchunks, Kpad, Fpad, P;
   int64_t R;   // rows per chunk (G > 1)
@@ -277,7 +298,7 @@ inline bool tc_shape(int D, int K, int num_sms, int* C_out, int* G_out) {
   const int cfull = tc_cluster(K);
   for (int G = 1; G <= kTcMaxGroups; G++) {
     const int C = (cfull + G - 1) / G;
-    if (C > kTcMaxCluster) continue;
+    if (C > kTcMaxCluster || (G > 1 && C > kTcGroupClusterMax)) continue;
     if (tc_smem_layout(D, C, tc_nchunks(D)).total > kTcMaxSmem) continue;
     if (G > 1 && num_sms / C < G) return false;
     *C_out = C;
@@ -322,7 +343,7 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.wsc = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
-  L.sharp = off;
+  L.ndir = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.nsplit = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
@@ -394,8 +415,8 @@ struct TcArgs {
                         // (-inf for padding / pi = 0)
   const float* ci;      // accumulator start values (W-row-scale units), C*128
   const float* wsc;     // W row scales, C*128
-  const int* sharp;     // 1: some dimensions in direct form, C*128
-  const int* nsplit;    // how many (the first of perm), C*128
+  const int* ndir;      // leading perm dimensions with direct-form moments, C*128
+  const int* nsplit;    // how many of those also leave the contraction, C*128
   const float* muh;     // mu (data units) in perm order, C*128 x D
   const float* ph;      // 1/var (data units) in perm order, C*128 x D
   const uint8_t* perm;  // dimensions by decreasing (mu^^2 + 1)/var^, C*128 x D
@@ -498,6 +519,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using namespace sm100;
   constexpr bool kStats = tc_mode_stats(MODE), kPartial = tc_mode_partial(MODE);
   constexpr bool kHard = tc_mode_hard(MODE);
+  // A pass without statistics on pre-converted features overlaps tiles: two
+  // logit buffers in tensor memory (columns [0, 128) and [128, 256), free of
+  // statistics here), so the E-step of tile i+1 runs while the epilogue of
+  // tile i reads the other buffer; the F buffer is released as soon as the
+  // E-step is done with it (after the epilogue when split dimensions' filter
+  // reads it too).
+  constexpr bool kOverlap = !kStats && FSRC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -530,6 +558,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* cbar = f_full + 10;    // rendezvous of the 256 compute threads
   uint64_t* f_free = f_full + 11;  // [2] FSRC = 1: MMAs and epilogue done with an F buffer
   uint64_t* f_tx = f_full + 13;    // [2] FSRC = 1: an F buffer's TMA loads have landed
+  uint64_t* f_full2 = f_full + 15;  // [2] overlap: start values in logit buffer b stored
+  uint64_t* l_full2 = f_full + 17;  // [2] overlap: E-step into logit buffer b done
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tslot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -557,6 +587,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int b = 0; b < 2; b++) {
       mbar_init(&f_free[b], 1);
       mbar_init(&f_tx[b], 1);
+      mbar_init(&f_full2[b], kTcComputeThreads);
+      mbar_init(&l_full2[b], 1);
     }
     mbar_init(l_full, 1);
     mbar_init(r_full, kTcComputeThreads / 2);
@@ -587,13 +619,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     int n = 0;
     uint32_t mw[4] = {0u, 0u, 0u, 0u};
+    // every component with direct-form moments: local index | split count << 8
+    // | direct count << 16; the mask marks those with split dimensions
     for (int j = 0; j < kTcComps; j++)
-      if (a.sharp[k0 + j]) {
-        shl[1 + n++] = j | (a.nsplit[k0 + j] << 8);  // local index | split count
-        mw[j >> 5] |= 1u << (j & 31);
+      if (a.ndir[k0 + j] > 0) {
+        const int ns = a.nsplit[k0 + j];
+        shl[1 + n++] = j | (ns << 8) | (a.ndir[k0 + j] << 16);
+        if (ns > 0) mw[j >> 5] |= 1u << (j & 31);
       }
     shl[0] = n;
-    for (int q = 0; q < 4; q++) shl[kTcComps + q] = (int)mw[q];  // bit j: local component j
+    // after the list (entries 1..128): bit j of word q is local component 32q + j
+    for (int q = 0; q < 4; q++) shl[kTcComps + 1 + q] = (int)mw[q];
   }
   for (int i = tid; i < 2048; i += kTcThreads)
     reinterpret_cast<__half*>(sOnes)[i] = __float2half_rn(1.0f);
@@ -694,8 +730,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint64_t dR = sw128_desc(rb, 8192, 1024);      // r^ as the MN-major statistics A
       const uint64_t dOnes = sw128_desc(ob, 16, 1024);
       uint32_t stage = 0, phase = 0, ndrain = 0;
+      const bool has_split = (shl[kTcComps + 1] | shl[kTcComps + 2] | shl[kTcComps + 3] |
+                              shl[kTcComps + 4]) != 0;
       for (int64_t li = 0; li < my_tiles; li++) {
-        if (!mbar_wait_bounded(f_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) break;
+        const uint32_t lb = kOverlap ? (uint32_t)(li & 1) : 0u;  // logit buffer
+        const uint32_t tLb = tL + 128u * lb;
+        if (kOverlap) {
+          if (!mbar_wait_bounded(&f_full2[lb], (uint32_t)((li >> 1) & 1), status, kAbort,
+                                 a.wait_ns))
+            break;
+        } else if (!mbar_wait_bounded(f_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) {
+          break;
+        }
         if (FSRC && !mbar_wait_bounded(&f_tx[li % L.nfb], (uint32_t)((li / L.nfb) & 1), status,
                                        kAbort, a.wait_ns))
           break;
@@ -715,8 +761,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int ks = 0; ks < 4; ks++) {
               const uint64_t bd = desc_add(wd, 32u * ks);
-              mma_bf16(tL, desc_add(fhd, 32u * ks), bd, idE, true);  // onto the start values
-              if (part == 0) mma_bf16(tL, desc_add(fld, 32u * ks), bd, idE, true);
+              mma_bf16(tLb, desc_add(fhd, 32u * ks), bd, idE, true);  // onto the start values
+              if (part == 0) mma_bf16(tLb, desc_add(fld, 32u * ks), bd, idE, true);
             }
             mma_commit(&empty[stage]);
             if (++stage == kTcStages) {
@@ -726,6 +772,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
         if (!ok) break;
+        if (kOverlap) {
+          mma_commit(&l_full2[lb]);
+          // the F buffer is free once the E-step is done with it -- or, where
+          // split dimensions' filter reads it, once both row halves' epilogues are
+          if (has_split &&
+              !(mbar_wait_bounded(r_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns) &&
+                mbar_wait_bounded(r_full1, (uint32_t)(li & 1), status, kAbort, a.wait_ns)))
+            break;
+          mma_commit(&f_free[li % L.nfb]);
+          continue;
+        }
         mma_commit(l_full);
         SCEM_TRACE(li, 9);
         if (!mbar_wait_bounded(r_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) break;
@@ -857,7 +914,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // epilogue) rather than from zero, so that its rounding errors cancel.
     // Each thread writes its own row and column half; the stores are waited
     // on before the F-full arrive.
-    auto store_start = [&]() {
+    auto store_start = [&](uint32_t lbuf) {
 #pragma unroll
       for (int q = 0; q < 2; q++) {
         float v[32];
@@ -869,10 +926,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           v[4 * j4 + 2] = c4.z;
           v[4 * j4 + 3] = c4.w;
         }
-        tmem_st32_nowait(tL + lane_base + (uint32_t)(col0 + 32 * q), v);
+        tmem_st32_nowait(tL + 128u * lbuf + lane_base + (uint32_t)(col0 + 32 * q), v);
       }
     };
-    if (my_tiles > 0) store_start();
+    if (my_tiles > 0) {
+      store_start(0);
+      if (kOverlap) {
+        tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(&f_full2[0]);
+      }
+    }
 
     for (int64_t li = 0; li < my_tiles && ok; li++) {
       const int64_t row0 = ((int64_t)cid + li * ncl) * kTcRows;
@@ -894,6 +958,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!ok) break;
       }
       uint8_t* sFc = sF + (uint32_t)(li % L.nfb) * L.fbytes;  // this tile's F buffer
+      const uint32_t tLc = tL + (kOverlap ? 128u * (uint32_t)(li & 1) : 0u);  // its logits
+      if (kOverlap && li + 1 < my_tiles) {
+        // the next tile's start values into the other logit buffer, read last
+        // by the tile before this one
+        store_start((uint32_t)((li + 1) & 1));
+        tmem_wait_st();
+        tc_fence_before_sync();
+        mbar_arrive(&f_full2[(li + 1) & 1]);
+      }
       bool bad = false, wide = false;
       if (!FSRC) {
       // ---- X tile -> F = [x^, x^^2] as fp16 hi/lo in the swizzled layout.
@@ -965,12 +1038,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }  // !FSRC: conversion
       if (bad) atomicOr(a.status, GMM_DEVFLAG_NONFINITE_X);
       if (wide) atomicOr(a.status, GMM_DEVFLAG_X_RANGE);
-      fence_proxy_async_smem();
-      tmem_wait_st();  // the accumulator's start values are in place
-      tc_fence_before_sync();
-      mbar_arrive(f_full);
+      if (!kOverlap) {
+        fence_proxy_async_smem();
+        tmem_wait_st();  // the accumulator's start values are in place
+        tc_fence_before_sync();
+        mbar_arrive(f_full);
+      }
       if (t == 0) SCEM_TRACE(li, 3);
-      if (li > 0 && (FSRC || L.nfb == 2)) {
+      if (!kOverlap && li > 0 && (FSRC || L.nfb == 2)) {
         ok = wait_prev_stats();
         if (!ok) break;
       }
@@ -986,8 +1061,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
 
       // ---- epilogue: logits -> row max / sum-exp -> cluster exchange -> r^
+      const bool valid = row0 + row < a.N;
+      float M = -INFINITY, S = 0.f;
+      int win = INT_MAX;  // hard EM: the row's component
+      // (max, sum-exp) partials combine as max and the sum rescaled to it;
+      // (max, index) partials as max and the lowest index attaining it
+      auto combine = [&](const float2 p) {
+        if (kHard) {
+          const int ix = __float_as_int(p.y);
+          if (p.x > M || (p.x == M && ix < win)) win = ix;
+          M = fmaxf(M, p.x);
+        } else {
+          M = fmaxf(M, p.x);
+        }
+      };
+      if ((kStats || MODE == kTcTopm) && ngrp > 1) {
+        // The row's partials of every group, from the partial pass over the
+        // same rows, combined in group order: the same value in every
+        // cluster, so the responsibilities of all groups sum to one.  Read
+        // while the E-step MMAs run.
+        const float2* pr = a.part + (size_t)(valid ? row0 + row : 0) * ngrp;
+        for (uint32_t g2 = 0; g2 < ngrp; g2++) combine(pr[g2]);
+        if (!kHard)
+          for (uint32_t g2 = 0; g2 < ngrp; g2++) {
+            const float2 p = pr[g2];
+            if (p.x > -INFINITY) S += p.y * __expf(p.x - M);
+          }
+      }
       ok = __all_sync(0xffffffffu,
-                      mbar_wait_bounded(l_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns));
+                      kOverlap ? mbar_wait_bounded(&l_full2[li & 1], (uint32_t)((li >> 1) & 1),
+                                                   status, kAbort, a.wait_ns)
+                               : mbar_wait_bounded(l_full, (uint32_t)(li & 1), status, kAbort,
+                                                   a.wait_ns));
       if (!ok) break;
       if (t == 0) SCEM_TRACE(li, 4);
       tc_fence_after_sync();
@@ -1002,7 +1107,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int q = 0; q < 2; q++) {
           float v[32];
-          tmem_ld32(tL + lane_base + (uint32_t)(col0 + 32 * q), v);
+          tmem_ld32(tLc + lane_base + (uint32_t)(col0 + 32 * q), v);
           const uint32_t mq = q ? m1 : m0;
 #pragma unroll
           for (int j = 0; j < 32; j++) {
@@ -1013,7 +1118,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       };
-      const uint32_t sm0 = (uint32_t)shl[kTcComps + 2 * hf], sm1 = (uint32_t)shl[kTcComps + 2 * hf + 1];
+      const uint32_t sm0 = (uint32_t)shl[kTcComps + 1 + 2 * hf],
+                     sm1 = (uint32_t)shl[kTcComps + 2 + 2 * hf];
       load_logits(false, sm0, sm1);
       if (sm0 | sm1) {
         // Components of this column half with split dimensions: the tensor
@@ -1029,16 +1135,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // the filter tables of every split component head for L1 now (one lane
         // per component), so the per-component loop below meets L1, not L2
         for (int sj = lane; sj < nsh; sj += 32) {
+          if (((shl[1 + sj] >> 8) & 255) == 0) continue;
           const size_t base = (size_t)(k0 + (shl[1 + sj] & 255)) * D;
           prefetch_l1(a.perm + base);
           prefetch_l1(a.mhp + base);
           prefetch_l1(a.php + base);
         }
         for (int si = 0; si < nsh; si++) {
-          const int j = shl[1 + si] & 255, ns = shl[1 + si] >> 8;
-          if ((j >> 6) != hf) continue;
+          const int j = shl[1 + si] & 255, ns = (shl[1 + si] >> 8) & 255;
+          if ((j >> 6) != hf || ns == 0) continue;
           const size_t base = (size_t)(k0 + j) * D;
-          const float v0 = tmem_ld1(tL + lane_base + (uint32_t)j);
+          const float v0 = tmem_ld1(tLc + lane_base + (uint32_t)j);
           const float lr = fmaf(v0, wscs[j], csm[j]);  // log-joint over the kept dimensions
           const float qmax = 2.f * (lr - floor_l);      // split sum beyond this: below the floor
           // Filter: the row's own features x^ = F_hi + F_lo (shared memory).
@@ -1113,7 +1220,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
           }
           // the finished log-joint (the second load_logits takes it as is)
-          tmem_st1(tL + lane_base + (uint32_t)j, q <= qmax ? lr - 0.5f * q : -INFINITY);
+          tmem_st1(tLc + lane_base + (uint32_t)j, q <= qmax ? lr - 0.5f * q : -INFINITY);
         }
         load_logits(true, sm0, sm1);
       }
@@ -1185,31 +1292,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int q = 0; q < a.ncand; q++) dst[q] = make_float2(-INFINITY, __int_as_float(INT_MAX));
         }
       }
-      const bool valid = row0 + row < a.N;
-      float M = -INFINITY, S = 0.f;
-      int win = INT_MAX;  // hard EM: the row's component
-      // (max, sum-exp) partials combine as max and the sum rescaled to it;
-      // (max, index) partials as max and the lowest index attaining it
-      auto combine = [&](const float2 p) {
-        if (kHard) {
-          const int ix = __float_as_int(p.y);
-          if (p.x > M || (p.x == M && ix < win)) win = ix;
-          M = fmaxf(M, p.x);
-        } else {
-          M = fmaxf(M, p.x);
-        }
-      };
       if ((kStats || MODE == kTcTopm) && ngrp > 1) {
-        // The row's partials of every group, from the partial pass over the
-        // same rows, combined in group order: the same value in every
-        // cluster, so the responsibilities of all groups sum to one.
-        const float2* pr = a.part + (size_t)(valid ? row0 + row : 0) * ngrp;
-        for (uint32_t g2 = 0; g2 < ngrp; g2++) combine(pr[g2]);
-        if (!kHard)
-          for (uint32_t g2 = 0; g2 < ngrp; g2++) {
-            const float2 p = pr[g2];
-            if (p.x > -INFINITY) S += p.y * __expf(p.x - M);
-          }
+        // combined above, before the wait for the E-step
       } else {
         // every (CTA, column half) contributes one (max, sum-exp) partial per row
         const uint32_t par = (uint32_t)(li & 1);
@@ -1250,6 +1334,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         scale = valid ? kTcRScale : 0.f;
       }
       const int hr = row >> 6, rr = row & 63;  // which 64-row half of r^, row within it
+      uint64_t rbits = 0;  // the thread's columns whose r exceeds kTcDirRmin
       if (kStats) {
         if (hr == 1) {
           // the first half's MMAs must be done with the buffer
@@ -1269,6 +1354,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           *reinterpret_cast<uint4*>(sR + off) = ph4;
           *reinterpret_cast<uint4*>(sR + 16384u + off) = pl4;
         }
+        if (shl[0] > 0) {
+#pragma unroll
+          for (int j = 0; j < 64; j++)
+            if (e[j] * scale > kTcDirRmin * kTcRScale) rbits |= 1ull << j;
+        }
         fence_proxy_async_smem();
       }
       tc_fence_before_sync();
@@ -1281,21 +1371,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // hold the next tile once the statistics MMAs are done.)  They go into
       // the shared fixed-point area (kTcDirScale), so the order in which rows
       // and clusters add them does not change the sums.
-      if (kStats && (sm0 | sm1)) {
+      if (kStats && shl[0] > 0) {
         const int nsh = shl[0];
         const XT* xrow = reinterpret_cast<const XT*>(a.X) + (size_t)(valid ? row0 + row : 0) * D;
         const size_t kp = (size_t)a.Kpad;
         for (int si = 0; si < nsh; si++) {
-          const int j = shl[1 + si] & 255, ns = shl[1 + si] >> 8;
-          if ((j >> 6) != hf) continue;
-          const float l = tmem_ld1(tL + lane_base + (uint32_t)j);  // the finished log-joint
+          const int j = shl[1 + si] & 255, ns = (shl[1 + si] >> 8) & 255, nd = shl[1 + si] >> 16;
+          if ((j >> 6) != hf || !((rbits >> (j & 63)) & 1ull)) continue;
+          // the log-joint: finished in tensor memory for a component with split
+          // dimensions, the raw accumulator (scaled as the epilogue scales it) otherwise
+          const float v0 = tmem_ld1(tLc + lane_base + (uint32_t)j);
+          const float l = ns > 0 ? v0 : fmaf(v0, wscs[j], csm[j]);
           const double r = !(valid && l > -INFINITY) ? 0.0
                            : kHard ? (k0 + j == win ? 1.0 : 0.0)
                                    : (double)__expf(l - lse);
-          if (r > 0.0) {
+          if (r > (double)kTcDirRmin) {
             const size_t base = (size_t)(k0 + j) * D;
             unsigned long long* q = a.dirq + (k0 + j);
-            for (int i = 0; i < ns; i++) {
+            for (int i = 0; i < nd; i++) {
               const int d = min((int)a.perm[base + i], D - 1);
               const double p = (double)a.ph[base + i];  // 1/var of this dimension
               const double u = ((double)load1<XT>(xrow, d) - (double)a.muh[base + i]) * sqrt(p);
@@ -1306,9 +1399,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
-      if (li + 1 < my_tiles) store_start();  // L is no longer read in this tile
+      if (!kOverlap && li + 1 < my_tiles) store_start(0);  // L is no longer read in this tile
     }
-    if (ok && my_tiles > 0) {
+    if (!kOverlap && ok && my_tiles > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(s_done, (uint32_t)((my_tiles - 1) & 1),
                                                      status, kAbort, a.wait_ns));
       tc_fence_after_sync();
@@ -1339,19 +1432,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Prep for the tensor-core pass, one thread per dimension:
+// Prep for the tensor-core pass, per dimension:
 //   m_d = sum_k pi_k mu_kd / sum_k pi_k                  (centring, fp64)
 //   v_d = sum_k pi_k (var_kd + mu_kd^2) / sum_k pi_k - m_d^2   (mixture variance)
 //   s_d = 2^(round(log2 sqrt(v_d)) + 1)                  (exact power-of-two scale)
 // ---------------------------------------------------------------------------
-__global__ void tc_center_kernel(int D, int K, const float* __restrict__ w,
-                                 const float* __restrict__ mu, const float* __restrict__ var,
-                                 float* __restrict__ m_out, float* __restrict__ isc_out,
-                                 float* __restrict__ sc_out) {
-  const int d = blockIdx.x * blockDim.x + threadIdx.x;
-  if (d >= D) return;
+// One block of 256 threads per dimension: thread t sums components t, t + 256,
+// ... in order, then a fixed tree combines the threads (deterministic).
+__global__ void __launch_bounds__(256) tc_center_kernel(int D, int K, const float* __restrict__ w,
+                                                        const float* __restrict__ mu,
+                                                        const float* __restrict__ var,
+                                                        float* __restrict__ m_out,
+                                                        float* __restrict__ isc_out,
+                                                        float* __restrict__ sc_out) {
+  __shared__ double red[3][256];
+  const int d = blockIdx.x;
   double s = 0.0, s2 = 0.0, sw = 0.0;
-  for (int k = 0; k < K; k++) {
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
     const double wk = (double)w[k];
     if (wk > 0.0) {
       const double mk = (double)mu[(size_t)k * D + d];
@@ -1360,6 +1457,19 @@ __global__ void tc_center_kernel(int D, int K, const float* __restrict__ w,
       sw += wk;
     }
   }
+  red[0][threadIdx.x] = s;
+  red[1][threadIdx.x] = s2;
+  red[2][threadIdx.x] = sw;
+  __syncthreads();
+  for (int h = 128; h > 0; h >>= 1) {
+    if ((int)threadIdx.x < h)
+      for (int q = 0; q < 3; q++) red[q][threadIdx.x] += red[q][threadIdx.x + h];
+    __syncthreads();
+  }
+  if (threadIdx.x != 0) return;
+  s = red[0][0];
+  s2 = red[1][0];
+  sw = red[2][0];
   const double m = sw > 0.0 ? s / sw : 0.0;
   const double v = sw > 0.0 ? s2 / sw - m * m : 0.0;
   int e = 0;
@@ -1405,7 +1515,7 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     int64_t N, int D, int K, int Fpad, const float* __restrict__ w, const float* __restrict__ mu,
     const float* __restrict__ var, const float* __restrict__ m, const float* __restrict__ sc,
     __half* __restrict__ whi, __half* __restrict__ wlo, float* __restrict__ c_out,
-    float* __restrict__ wsc_out, int* __restrict__ sharp_out, int* __restrict__ nsplit_out,
+    float* __restrict__ wsc_out, int* __restrict__ ndir_out, int* __restrict__ nsplit_out,
     float* __restrict__ muh, float* __restrict__ ph, int* __restrict__ precise_out,
     float* __restrict__ ci_out, uint8_t* __restrict__ perm_out, float* __restrict__ mhp_out,
     float* __restrict__ php_out, uint32_t* __restrict__ pmask_out, uint8_t* __restrict__ rank_out,
@@ -1415,7 +1525,7 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
   __shared__ double wv[kTcChunk * kTcMaxChunks];  // Fpad <= 256
   __shared__ double ef[kTcChunk * kTcMaxChunks];  // E[F] under the component
   __shared__ double red[4][4];
-  __shared__ int ns_s;
+  __shared__ int ns_s, nd_s;
   const int k = blockIdx.x;
   const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
   const float wk = k < K ? w[k] : 0.f;
@@ -1491,6 +1601,11 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
       while (ns < D && rem > thr) rem -= ksort[ns++];
     }
     ns_s = ns;
+    // and the further leading dimensions whose moments are taken in direct form
+    int nd = ns;
+    if (live)
+      while (nd < D && ksort[nd] > kTcDirectKappa) nd++;
+    nd_s = nd;
   }
   __syncthreads();
   const int ns = ns_s;
@@ -1553,7 +1668,7 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     ci_out[k] = cstart;
     c_out[k] = live ? (float)(cfull - ldexp((double)cstart, g)) : -INFINITY;
     wsc_out[k] = ldexpf(1.0f, g);
-    sharp_out[k] = ns > 0 ? 1 : 0;
+    ndir_out[k] = nd_s;
     nsplit_out[k] = ns;
     precise_out[k] = live && (Rho > kTcRhoPrecise || small) ? 1 : 0;  // some pmask bit set
   }
@@ -1569,14 +1684,14 @@ __device__ __forceinline__ double fixed_value(unsigned long long hi, unsigned lo
 // statistics buffer [ N_k | A | B | LL ] (component-major, moments about the
 // input means mu, data units).  The slots hold N' = 2^15 N_k and
 // S1' = 2^15 sum r x^, S2' = 2^15 sum r x^^2 with x^ = (x - m)/s, so with
-// dm = mu - m:  A = s S1 - dm N,  B = s^2 S2 - 2 s dm S1 + dm^2 N.  A split
-// dimension (perm position below nsplit_k) takes A and B from the fixed-point
-// direct-form moments instead, scaled back by sigma = 1/sqrt(ph) with the same
+// dm = mu - m:  A = s S1 - dm N,  B = s^2 S2 - 2 s dm S1 + dm^2 N.  A
+// dimension with direct-form moments (perm position below ndir_k) takes A and
+// B from the fixed-point sums instead, scaled back by sigma = 1/sqrt(ph) with the same
 // stored ph the fused pass divided by.
 __global__ void __launch_bounds__(256) tc_reduce_stats_kernel(
     int D, int K, int Kpad, const float* __restrict__ m, const float* __restrict__ sc,
     const float* __restrict__ mu, const uint8_t* __restrict__ rank,
-    const int* __restrict__ nsplit, const float* __restrict__ ph,
+    const int* __restrict__ ndir, const float* __restrict__ ph,
     const unsigned long long* __restrict__ dirq, const double* __restrict__ slots,
     size_t slot_stride, int nslots, int G, int group_comps, double* __restrict__ stats) {
   const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -1602,7 +1717,7 @@ __global__ void __launch_bounds__(256) tc_reduce_stats_kernel(
   const double dm = (double)mu[(size_t)k * D + d] - (double)m[d];
   if (d == 0) stats[k] = n;
   const int r = rank[(size_t)k * D + d];
-  if (r < nsplit[k]) {
+  if (r < ndir[k]) {
     const size_t kp = (size_t)Kpad;
     const double p = (double)ph[(size_t)k * D + r];  // 1/var, perm order
     const double a1 = fixed_value(dirq[(size_t)r * kp + k], dirq[(size_t)(D + r) * kp + k]);

@@ -66,15 +66,20 @@ def _step(K=4, D=3, N=10_000.0):
     return (w, mu, var, -1234.5), Nk, N
 
 
-def test_weight_rule_is_relative_with_a_ten_point_floor():
+def test_weight_rule_is_relative_plus_1e9():
+    """|dpi| <= 1e-3 pi + 1e-9, for a 5000-point and a 5-point component alike
+    (no floor at ten points); the looser 10-point reading is reported beside it."""
     ref, Nk, N = _step()
-    for k, scale in ((0, 1e-3 * ref[0][0]), (3, 1e-3 * 10 / N)):  # 5000 points; 5 points
+    for k in (0, 3):  # 5000 points; 5 points
+        scale = 1e-3 * ref[0][k] + 1e-9
         for frac, ok in ((0.9, True), (1.1, False)):
             w = ref[0].copy()
             w[k] += frac * scale
             rep = compare.compare_step(ref, (w, *ref[1:]), Nk, N)
             assert rep["ok"] is ok, (k, frac, rep)
             assert rep["w"] == pytest.approx(frac, rel=1e-6)
+            floor = 1e-3 * max(ref[0][k], 10 / N)
+            assert rep["w_floor10"] == pytest.approx(frac * scale / floor, rel=1e-6)
 
 
 def test_mean_rule_scales_with_max_of_mean_and_sigma():
