@@ -196,12 +196,19 @@ gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const 
   float* m = (float*)(ws + T.m);
   tc_center_kernel<<<p->D, 256, 0, st>>>(p->D, p->K, w, mu, var, m,
                                                        (float*)(ws + T.isc), (float*)(ws + T.sc));
-  tc_prep_w_kernel<<<T.Kpad, 128, 0, st>>>(
+  const size_t psmem = tc_prep_smem_bytes(p->D, T.Fpad);
+  if (psmem > 48 * 1024 &&
+      cudaFuncSetAttribute(tc_prep_w_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)psmem) != cudaSuccess) {
+    cudaGetLastError();
+    return GMM_ERR_UNSUPPORTED;
+  }
+  tc_prep_w_kernel<<<T.Kpad, 128, psmem, st>>>(
       p->N, p->D, p->K, T.Fpad, w, mu, var, m, (const float*)(ws + T.sc), (__half*)(ws + T.whi),
       (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.wsc), (int*)(ws + T.ndir),
       (int*)(ws + T.nsplit), (float*)(ws + T.muh), (float*)(ws + T.ph), (int*)(ws + T.precise),
-      (float*)(ws + T.ci), (uint8_t*)(ws + T.perm), (float*)(ws + T.mhp), (float*)(ws + T.php),
-      (uint32_t*)(ws + T.pmask), (uint8_t*)(ws + T.rank), (unsigned long long*)(ws + T.dirq),
+      (float*)(ws + T.ci), (uint16_t*)(ws + T.perm), (float*)(ws + T.mhp), (float*)(ws + T.php),
+      (uint32_t*)(ws + T.pmask), (uint16_t*)(ws + T.rank), (unsigned long long*)(ws + T.dirq),
       (unsigned int*)ws);
   return launched(2);
 }
@@ -254,7 +261,7 @@ gmm_status tc_clusters(const TcLayout& T, int64_t ntiles, size_t smem, int* ncl_
 template <typename XT, int MODE, int FSRC>
 gmm_status tc_launch(const gmm_problem* p, const void* X, int64_t N, char* ws, const TcLayout& T,
                      int ncl, int accumulate, cudaStream_t st, int32_t* labels = nullptr,
-                     int ncand = 0) {
+                     int ncand = 0, int fg0 = 0, int nfgc = 0) {
   CUtensorMap mhi, mlo, fhi, flo;
   memset(&mhi, 0, sizeof(mhi));
   memset(&mlo, 0, sizeof(mlo));
@@ -302,7 +309,7 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, int64_t N, char* ws, c
   args.nsplit = (const int*)(ws + T.nsplit);
   args.muh = (const float*)(ws + T.muh);
   args.ph = (const float*)(ws + T.ph);
-  args.perm = (const uint8_t*)(ws + T.perm);
+  args.perm = (const uint16_t*)(ws + T.perm);
   args.mhp = (const float*)(ws + T.mhp);
   args.php = (const float*)(ws + T.php);
   args.slots = (double*)(ws + T.slots);
@@ -316,6 +323,9 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, int64_t N, char* ws, c
   args.cand = (float2*)(ws + T.cand);
   args.rowst = (float2*)(ws + T.rowst);
   args.ncand = std::min(kTcCand, ncand);
+  args.fg0 = fg0;
+  args.nfgc = nfgc > 0 ? nfgc : T.nfg;
+  args.nfg = T.nfg;
   args.status = (unsigned int*)ws;
   args.drain_tiles = kTcDrainTiles;
   args.precise = (const int*)(ws + T.precise);
@@ -335,61 +345,86 @@ size_t tc_smem_bytes(const gmm_problem* p, const TcLayout& T) {
   return std::max<size_t>(tc_smem_layout(p->D, T.C, T.nchunks).total, 120 * 1024);
 }
 
-// The fused pass over all rows of X: one launch with one component group;
-// with G > 1, chunk by chunk, the features converted, then the partial pass,
-// then the statistics (or, for MODE = kTcLoglik, the log-likelihood) pass.
-// *nslots receives the number of slots written.  The trace events bracket
-// the whole pass.
-template <typename XT, int MODE>
-gmm_status tc_pass_t(const gmm_problem* p, const void* X, char* ws, const TcLayout& T,
-                     cudaStream_t st, int* nslots, double* loglik, int32_t* labels) {
+// Converts rows [r0, r0 + n) of X into the chunk's feature buffer.
+template <typename XT>
+gmm_status tc_convert(const gmm_problem* p, const XT* Xc, int64_t n, char* ws, const TcLayout& T,
+                      cudaStream_t st) {
+  const int64_t items = n * (p->D / 4);
+  const unsigned grid = (unsigned)std::min<int64_t>((items + 255) / 256, 148 * 16);
+  tc_convert_kernel<XT><<<grid, 256, 0, st>>>(Xc, n, p->D, T.Fpad, (const float*)(ws + T.m),
+                                             (const float*)(ws + T.isc), (__half*)(ws + T.fhi),
+                                             (__half*)(ws + T.flo), (unsigned int*)ws);
+  return launched(1);
+}
+
+// The fused pass over pre-converted features (FS = 1: resident per tile;
+// FS = 2: streamed in rounds), chunk by chunk: the features converted, the
+// partial pass when there are several component groups, then the statistics
+// pass once per feature group (or the log-likelihood).
+template <typename XT, int MODE, int FS>
+gmm_status tc_pass_chunked(const gmm_problem* p, const void* X, char* ws, const TcLayout& T,
+                           cudaStream_t st, int* nslots, double* loglik, int32_t* labels) {
   constexpr int PART = tc_mode_hard(MODE) ? kTcHardPartial : kTcPartial;
   const int64_t ntiles = (p->N + kTcRows - 1) / kTcRows;
   const size_t smem = tc_smem_bytes(p, T);
   gmm_status s;
-  int ncl = 0;
-  if (T.G == 1) {
-    if ((s = tc_clusters<XT, MODE, 0>(T, ntiles, smem, &ncl)) != GMM_OK) return s;
-    trace_begin(st);
-    s = tc_launch<XT, MODE, 0>(p, X, p->N, ws, T, ncl, 0, st, labels);
-    trace_end(st);
-    *nslots = ncl;
-    return s;
+  int ncl = 1 << 30, c2 = 0;
+  if (T.G > 1) {
+    if ((s = tc_clusters<XT, PART, FS>(T, ntiles, smem, &c2)) != GMM_OK) return s;
+    ncl = std::min(ncl, c2);
   }
-  if ((s = tc_clusters<XT, PART, 1>(T, ntiles, smem, &ncl)) != GMM_OK) return s;
-  if (tc_mode_stats(MODE)) {
-    int ncl2 = 0;
-    if ((s = tc_clusters<XT, MODE, 1>(T, ntiles, smem, &ncl2)) != GMM_OK) return s;
-    ncl = std::min(ncl, ncl2);
-  }
+  if ((s = tc_clusters<XT, MODE, FS>(T, ntiles, smem, &c2)) != GMM_OK) return s;
+  ncl = std::min(ncl, c2);
   const size_t row_bytes = (size_t)p->D * sizeof(XT);
-  double* blocks = (double*)(ws + T.slots);  // log-likelihood mode: the slots are free
+  double* blocks = (double*)(ws + T.slots);  // log-likelihood mode with groups: the slots are free
   trace_begin(st);
   int64_t i = 0;
   for (int64_t r0 = 0; r0 < p->N; r0 += T.R, i++) {
     const int64_t n = std::min<int64_t>(T.R, p->N - r0);
     const XT* Xc = (const XT*)((const char*)X + (size_t)r0 * row_bytes);
-    const int64_t items = n * (p->D / 4);
-    const unsigned grid = (unsigned)std::min<int64_t>((items + 255) / 256, 148 * 16);
-    tc_convert_kernel<XT><<<grid, 256, 0, st>>>(Xc, n, p->D, T.Fpad, (const float*)(ws + T.m),
-                                               (const float*)(ws + T.isc), (__half*)(ws + T.fhi),
-                                               (__half*)(ws + T.flo), (unsigned int*)ws);
-    if ((s = launched(1)) != GMM_OK) return s;
-    if ((s = tc_launch<XT, PART, 1>(p, Xc, n, ws, T, ncl, 0, st)) != GMM_OK) return s;
+    if ((s = tc_convert<XT>(p, Xc, n, ws, T, st)) != GMM_OK) return s;
+    if (T.G > 1 && (s = tc_launch<XT, PART, FS>(p, Xc, n, ws, T, ncl, 0, st)) != GMM_OK)
+      return s;
     if (tc_mode_stats(MODE)) {
-      if ((s = tc_launch<XT, MODE, 1>(p, Xc, n, ws, T, ncl, i > 0, st,
-                                      labels ? labels + r0 : nullptr)) != GMM_OK)
-        return s;
-    } else {
+      for (int fg = 0; fg < T.NFG; fg++) {
+        const int fg0 = fg * T.nfg;
+        if ((s = tc_launch<XT, MODE, FS>(p, Xc, n, ws, T, ncl, !(i == 0 && fg == 0), st,
+                                         labels ? labels + r0 : nullptr, 0, fg0,
+                                         std::min(T.nfg, T.nchunks - fg0))) != GMM_OK)
+          return s;
+      }
+    } else if (T.G > 1) {
       tc_part_loglik_kernel<<<kTcLseBlocks, 256, 0, st>>>((const float2*)(ws + T.part), n, T.G,
                                                           blocks);
       tc_sum_blocks_kernel<<<1, 1, 0, st>>>(blocks, i == 0, loglik);
       if ((s = launched(2)) != GMM_OK) return s;
+    } else if ((s = tc_launch<XT, MODE, FS>(p, Xc, n, ws, T, ncl, i > 0, st)) != GMM_OK) {
+      return s;  // one group, streamed features: each chunk's LL adds into the slots
     }
   }
   trace_end(st);
   *nslots = ncl;
   return GMM_OK;
+}
+
+// The fused pass over all rows of X: one launch with one component group and
+// resident features; otherwise chunk by chunk (tc_pass_chunked).  *nslots
+// receives the number of slots written.  The trace events bracket the pass.
+template <typename XT, int MODE>
+gmm_status tc_pass_t(const gmm_problem* p, const void* X, char* ws, const TcLayout& T,
+                     cudaStream_t st, int* nslots, double* loglik, int32_t* labels) {
+  if (tc_streamed(T.nchunks))
+    return tc_pass_chunked<XT, MODE, 2>(p, X, ws, T, st, nslots, loglik, labels);
+  if (T.G > 1) return tc_pass_chunked<XT, MODE, 1>(p, X, ws, T, st, nslots, loglik, labels);
+  const int64_t ntiles = (p->N + kTcRows - 1) / kTcRows;
+  gmm_status s;
+  int ncl = 0;
+  if ((s = tc_clusters<XT, MODE, 0>(T, ntiles, tc_smem_bytes(p, T), &ncl)) != GMM_OK) return s;
+  trace_begin(st);
+  s = tc_launch<XT, MODE, 0>(p, X, p->N, ws, T, ncl, 0, st, labels);
+  trace_end(st);
+  *nslots = ncl;
+  return s;
 }
 
 template <int MODE>
@@ -425,7 +460,7 @@ gmm_status estep_stats_impl(const gmm_problem* p, const void* X, const float* w,
     if (s != GMM_OK) return s;
     tc_reduce_stats_kernel<<<blocks, 256, 0, st>>>(
         p->D, p->K, T.Kpad, (const float*)(ws + T.m), (const float*)(ws + T.sc), mu,
-        (const uint8_t*)(ws + T.rank), (const int*)(ws + T.ndir), (const float*)(ws + T.ph),
+        (const uint16_t*)(ws + T.rank), (const int*)(ws + T.ndir), (const float*)(ws + T.ph),
         (const unsigned long long*)(ws + T.dirq), (const double*)(ws + T.slots), T.slot_stride,
         nslots, T.G, T.C * kTcComps, stats);
     return launched(1);
@@ -437,10 +472,30 @@ gmm_status estep_stats_impl(const gmm_problem* p, const void* X, const float* w,
   return launched(1);
 }
 
-// Top-m assignment on the tensor cores, chunk by chunk (Rt rows): with G > 1
-// groups the features are converted and the partial pass runs first; the
-// top-m pass writes each (CTA, column half)'s candidates and each row's
-// (max, sum-exp); tc_topm_refine_kernel finishes the rows in direct form.
+// One chunk of the top-m pass over pre-converted features (FS = 1 or 2).
+template <typename XT, int FS>
+gmm_status tc_topm_chunk(const gmm_problem* p, const XT* Xc, int64_t n, char* ws,
+                         const TcLayout& T, int nc, cudaStream_t st) {
+  const int64_t ntiles = (n + kTcRows - 1) / kTcRows;
+  const size_t smem = tc_smem_bytes(p, T);
+  gmm_status s;
+  int ncl = 1 << 30, c2 = 0;
+  if (T.G > 1) {
+    if ((s = tc_clusters<XT, kTcPartial, FS>(T, ntiles, smem, &c2)) != GMM_OK) return s;
+    ncl = c2;
+  }
+  if ((s = tc_clusters<XT, kTcTopm, FS>(T, ntiles, smem, &c2)) != GMM_OK) return s;
+  ncl = std::min(ncl, c2);
+  if ((s = tc_convert<XT>(p, Xc, n, ws, T, st)) != GMM_OK) return s;
+  if (T.G > 1 && (s = tc_launch<XT, kTcPartial, FS>(p, Xc, n, ws, T, ncl, 0, st)) != GMM_OK)
+    return s;
+  return tc_launch<XT, kTcTopm, FS>(p, Xc, n, ws, T, ncl, 0, st, nullptr, nc);
+}
+
+// Top-m assignment on the tensor cores, chunk by chunk (Rt rows): the top-m
+// pass (after the features are converted and the partial pass, when the
+// shape needs them) writes each (CTA, column half)'s candidates and each
+// row's (max, sum-exp); tc_topm_refine_kernel finishes the rows in direct form.
 template <typename XT>
 gmm_status tc_topm_t(const gmm_problem* p, const void* X, const float* w, const float* mu,
                      const float* var, int m, int32_t* idx, float* resp, char* ws, const Plan& P,
@@ -455,33 +510,21 @@ gmm_status tc_topm_t(const gmm_problem* p, const void* X, const float* w, const 
   const int nc = std::min(m + 2, kTcCand);
   const size_t smem = tc_smem_bytes(p, T);
   const size_t row_bytes = (size_t)p->D * sizeof(XT);
+  const bool streamed = tc_streamed(T.nchunks);
   trace_begin(st);
   for (int64_t r0 = 0; r0 < p->N; r0 += T.Rt) {
     const int64_t n = std::min<int64_t>(T.Rt, p->N - r0);
-    const int64_t ntiles = (n + kTcRows - 1) / kTcRows;
     const XT* Xc = (const XT*)((const char*)X + (size_t)r0 * row_bytes);
-    int ncl = 0;
-    if (T.G == 1) {
-      if ((s = tc_clusters<XT, kTcTopm, 0>(T, ntiles, smem, &ncl)) != GMM_OK) return s;
-      if ((s = tc_launch<XT, kTcTopm, 0>(p, Xc, n, ws, T, ncl, 0, st, nullptr, nc)) != GMM_OK)
-        return s;
+    if (streamed) {
+      s = tc_topm_chunk<XT, 2>(p, Xc, n, ws, T, nc, st);
+    } else if (T.G > 1) {
+      s = tc_topm_chunk<XT, 1>(p, Xc, n, ws, T, nc, st);
     } else {
-      int ncl2 = 0;
-      if ((s = tc_clusters<XT, kTcPartial, 1>(T, ntiles, smem, &ncl)) != GMM_OK ||
-          (s = tc_clusters<XT, kTcTopm, 1>(T, ntiles, smem, &ncl2)) != GMM_OK)
-        return s;
-      ncl = std::min(ncl, ncl2);
-      const int64_t items = n * (p->D / 4);
-      const unsigned grid = (unsigned)std::min<int64_t>((items + 255) / 256, 148 * 16);
-      tc_convert_kernel<XT><<<grid, 256, 0, st>>>(Xc, n, p->D, T.Fpad, (const float*)(ws + T.m),
-                                                 (const float*)(ws + T.isc),
-                                                 (__half*)(ws + T.fhi), (__half*)(ws + T.flo),
-                                                 (unsigned int*)ws);
-      if ((s = launched(1)) != GMM_OK) return s;
-      if ((s = tc_launch<XT, kTcPartial, 1>(p, Xc, n, ws, T, ncl, 0, st)) != GMM_OK ||
-          (s = tc_launch<XT, kTcTopm, 1>(p, Xc, n, ws, T, ncl, 0, st, nullptr, nc)) != GMM_OK)
-        return s;
+      int ncl = 0;
+      s = tc_clusters<XT, kTcTopm, 0>(T, (n + kTcRows - 1) / kTcRows, smem, &ncl);
+      if (s == GMM_OK) s = tc_launch<XT, kTcTopm, 0>(p, Xc, n, ws, T, ncl, 0, st, nullptr, nc);
     }
+    if (s != GMM_OK) return s;
     tc_topm_refine_kernel<XT><<<(unsigned)((n + 127) / 128), 128, 0, st>>>(
         Xc, n, p->D, p->K, T.G * T.C * 2, nc, m, (const float2*)(ws + T.cand),
         (const float2*)(ws + T.rowst), mu, iv, c0, idx + (size_t)r0 * m, resp + (size_t)r0 * m);

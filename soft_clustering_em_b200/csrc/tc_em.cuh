@@ -82,8 +82,16 @@ constexpr int kTcRows = 128;      // rows per tile (= tensor-memory lanes)
 constexpr int kTcComps = 128;     // components per CTA
 constexpr int kTcChunk = 64;      // features per operand chunk (one swizzled 128-byte row)
 constexpr int kTcStages = 3;      // depth of the W ring
-constexpr int kTcMaxChunks = 4;   // 2D <= 256
-constexpr int kTcMaxD = 128;
+constexpr int kTcMaxChunks = 4;   // features resident in shared memory: 2D <= 256
+constexpr int kTcMaxD = 128;      // the largest D with resident features
+// Beyond D = 128 the features stream through shared memory: kTcRoundChunks
+// feature chunks (hi and lo) at a time, for the E-step and again for the
+// statistics, which accumulate kTcGroupChunks chunks per pass in tensor memory
+// (128 logit + 320 statistic + 16 N_k columns), one pass per feature group.
+constexpr int kTcMaxDStream = 1024;
+static_assert(kTcMaxDStream < 2048, "split and direct counts are packed in 11 bits");
+constexpr int kTcRoundChunks = 2;
+constexpr int kTcGroupChunks = 5;
 constexpr int kTcMaxCluster = 16;
 constexpr int kTcThreads = 320;          // 8 compute warps + MMA warp + TMA warp
 constexpr int kTcComputeThreads = 256;
@@ -168,7 +176,9 @@ constexpr int kTcMaxGroups = 64;
 // Largest cluster of a component group when there are several (G > 1): the
 // grid must hold a whole number of clusters per group, and smaller clusters
 // pack more of the SMs into it (8-CTA clusters left a third of a B200 idle).
-constexpr int kTcGroupClusterMax = 16;
+// Measured at D = 96, K = 4096 per 1e6 rows: 8-CTA clusters (4 groups) 119 ms,
+// 4 (8 groups) 92 ms, 2 (16 groups) 94 ms, 1 (32 groups) 106 ms.
+constexpr int kTcGroupClusterMax = 4;
 constexpr int64_t kTcChunkRowsMax = 1 << 18;       // rows per pass with component groups
 constexpr size_t kTcChunkFBytesMax = 256u << 20;   // cap on the chunk's feature buffer
 
@@ -190,6 +200,7 @@ __device__ unsigned long long g_phase_trace[64 * 16];
 
 inline int tc_nchunks(int D) { return (2 * D + kTcChunk - 1) / kTcChunk; }
 inline int tc_cluster(int K) { return (K + kTcComps - 1) / kTcComps; }
+__host__ __device__ inline bool tc_streamed(int nchunks) { return nchunks > kTcMaxChunks; }
 
 // Byte offsets of the kernel's shared-memory regions (from a 1024-aligned base).
 // nfb F buffers of fbytes each: two when they fit (small D), so that a tile's
@@ -198,6 +209,7 @@ inline int tc_cluster(int K) { return (K + kTcComps - 1) / kTcComps; }
 struct TcSmem {
   uint32_t F, W, R, ONES, msm, iscs, csm, cis, wscs, shl, precs, xchg, bars, tslot, total;
   uint32_t nfb, fbytes;
+  uint32_t nr;  // feature chunks an F buffer holds: all of them, or a round when streamed
 };
 
 constexpr uint32_t kTcMaxSmem = 232448;  // 227 KB per CTA
@@ -205,14 +217,18 @@ constexpr uint32_t kTcMaxSmem = 232448;  // 227 KB per CTA
 __host__ __device__ inline TcSmem tc_smem_layout_n(int D, int C, int nchunks, uint32_t nfb) {
   TcSmem L;
   uint32_t off = 0;
+  const bool streamed = tc_streamed(nchunks);
   L.nfb = nfb;
-  L.fbytes = 2u * nchunks * kTcChunkBytes;
+  L.nr = streamed ? (uint32_t)kTcRoundChunks : (uint32_t)nchunks;
+  L.fbytes = 2u * L.nr * kTcChunkBytes;
   L.F = off;
   off += nfb * L.fbytes;
   L.W = off;
   off += kTcStages * kTcChunkBytes;
   L.R = off;
-  off += 2u * kTcChunkBytes;
+  // r^ hi | lo: one 64-row half at a time, or all 128 rows when the statistics
+  // run in several rounds over the features
+  off += (streamed ? 4u : 2u) * kTcChunkBytes;
   L.ONES = off;
   off += 4096;
   L.msm = off;
@@ -240,6 +256,7 @@ __host__ __device__ inline TcSmem tc_smem_layout_n(int D, int C, int nchunks, ui
 }
 
 __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
+  if (tc_streamed(nchunks)) return tc_smem_layout_n(D, C, nchunks, 1);
   const TcSmem two = tc_smem_layout_n(D, C, nchunks, 2);
   return two.total <= kTcMaxSmem ? two : tc_smem_layout_n(D, C, nchunks, 1);
 }
@@ -257,12 +274,12 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //          them (nsplit: C*128 int32) also leave the contraction for the logits
 //   pmask: [C*128 x Fpad/32] u32 per feature of each component, 1 if it is
 //          drained after every tile with mass (see tc_prep_w_kernel)
-//   perm : [C*128 x D] u8 dimensions of each component by decreasing
+//   perm : [C*128 x D] u16 dimensions of each component by decreasing
 //          (mu^^2 + 1)/var^
 //   muh, ph : [C*128 x D] f32 mu and 1/var (data units) in perm order
 //   mhp, php : [C*128 x D] f32 mu^ and 1/var^ in perm order
 //   whi, wlo : [C*128 x 64*nchunks] fp16 operand W (hi and lo parts)
-//   rank : [C*128 x D] u8 position of each dimension in perm
+//   rank : [C*128 x D] u16 position of each dimension in perm
 //   dirq : [4D x C*128] u64 direct-form moments of split dimensions about the
 //          input means, by perm position i, as 64-bit fixed-point words (see
 //          kTcDirScale): rows i / D+i hold the high / low words of
@@ -284,7 +301,8 @@ struct TcLayout {
   size_t m, isc, sc, c, ci, wsc, ndir, nsplit, precise, pmask, muh, ph, perm, rank, mhp, php, whi,
       wlo, dirq, slots, fhi, flo, part, cand, rowst, total, slot_stride;
   int C, G, nchunks, Kpad, Fpad, P;
-  int64_t R;   // rows per chunk (G > 1)
+  int nfg, NFG;  // feature chunks per statistics group, and groups (1 unless streamed)
+  int64_t R;   // rows per chunk (G > 1, or streamed features)
   int64_t Rt;  // rows per chunk of the top-m assignment
 };
 
@@ -294,7 +312,7 @@ struct TcLayout {
 // can hold one cluster each.  False if none does (or D is not a multiple of 4
 // up to 128): such shapes run on the CUDA cores.
 inline bool tc_shape(int D, int K, int num_sms, int* C_out, int* G_out) {
-  if (!(D >= 4 && D <= 128 && D % 4 == 0 && K >= 1)) return false;
+  if (!(D >= 4 && D <= kTcMaxDStream && D % 4 == 0 && K >= 1)) return false;
   const int cfull = tc_cluster(K);
   for (int G = 1; G <= kTcMaxGroups; G++) {
     const int C = (cfull + G - 1) / G;
@@ -329,7 +347,10 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   L.nchunks = tc_nchunks(D);
   L.Kpad = L.G * L.C * kTcComps;
   L.Fpad = L.nchunks * kTcChunk;
-  L.R = L.G > 1 ? tc_chunk_rows(L.Fpad) : 0;
+  const bool streamed = tc_streamed(L.nchunks);
+  L.nfg = streamed ? kTcGroupChunks : L.nchunks;
+  L.NFG = (L.nchunks + L.nfg - 1) / L.nfg;
+  L.R = (L.G > 1 || streamed) ? tc_chunk_rows(L.Fpad) : 0;
   size_t off = 256;
   L.m = off;
   off = align_up(off + (size_t)D * 4, 256);
@@ -352,9 +373,9 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   L.ph = off;
   off = align_up(off + (size_t)L.Kpad * D * 4, 256);
   L.perm = off;
-  off = align_up(off + (size_t)L.Kpad * D, 256);
+  off = align_up(off + (size_t)L.Kpad * D * 2, 256);
   L.rank = off;
-  off = align_up(off + (size_t)L.Kpad * D, 256);
+  off = align_up(off + (size_t)L.Kpad * D * 2, 256);
   L.mhp = off;
   off = align_up(off + (size_t)L.Kpad * D * 4, 256);
   L.php = off;
@@ -370,9 +391,9 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   L.dirq = off;
   off = align_up(off + (size_t)4 * D * L.Kpad * 8, 256);
   L.slot_stride = align_up((size_t)(2 * D + 1) * K + 1, 32);
-  // the chunk buffers of the two-pass form (G > 1), ahead of the slots
+  // the chunk buffers of pre-converted features (G > 1 or streamed), ahead of the slots
   L.fhi = L.flo = L.part = off;
-  if (L.G > 1) {
+  if (L.R > 0) {
     L.fhi = off;
     off = align_up(off + (size_t)L.R * L.Fpad * 2, 256);
     L.flo = off;
@@ -385,7 +406,7 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
     const size_t per_row = (size_t)L.G * L.C * 2 * kTcCand * 8 + 8;
     int64_t rt = (int64_t)((size_t)(64u << 20) / per_row) / kTcRows * kTcRows;
     rt = std::max<int64_t>(kTcRows, std::min<int64_t>(rt, kTcChunkRowsMax));
-    if (L.G > 1) rt = std::min<int64_t>(rt, L.R);
+    if (L.R > 0) rt = std::min<int64_t>(rt, L.R);
     L.Rt = rt;
     L.cand = off;
     off = align_up(off + (size_t)rt * (per_row - 8), 256);
@@ -419,7 +440,7 @@ struct TcArgs {
   const int* nsplit;    // how many of those also leave the contraction, C*128
   const float* muh;     // mu (data units) in perm order, C*128 x D
   const float* ph;      // 1/var (data units) in perm order, C*128 x D
-  const uint8_t* perm;  // dimensions by decreasing (mu^^2 + 1)/var^, C*128 x D
+  const uint16_t* perm;  // dimensions by decreasing (mu^^2 + 1)/var^, C*128 x D
   const float* mhp;     // mu^ in that order, C*128 x D
   const float* php;     // 1/var^ in that order, C*128 x D
   double* slots;        // per-cluster statistic slots
@@ -433,6 +454,8 @@ struct TcArgs {
   float2* cand;         // top-m: [rows x (G C 2) x kTcCand] (log-joint, index) candidates
   float2* rowst;        // top-m: [rows] the row's (max, sum-exp) over all components
   int ncand;            // top-m: candidates kept per (CTA, column half), <= kTcCand
+  int fg0, nfgc, nfg;   // streamed features: this pass's statistics group (first chunk,
+                        // chunks) and the group size that lays out tensor memory
   unsigned int* status;
   int drain_tiles;
   const int* precise;   // 1: some feature of the component is drained every tile, C*128
@@ -446,6 +469,14 @@ struct TcArgs {
 // A shared-memory descriptor advanced by `bytes` (start-address field only;
 // every operand lies within the first 256 KB of shared memory, so no carry).
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+// An entry of the CTA's list of components with direct-form dimensions: the
+// local column j (< 128), the split count ns and the direct count nd (each
+// <= D <= 1024) in 7 + 11 + 11 bits.
+__device__ __forceinline__ int shl_pack(int j, int ns, int nd) { return j | (ns << 7) | (nd << 18); }
+__device__ __forceinline__ int shl_j(int v) { return v & 127; }
+__device__ __forceinline__ int shl_ns(int v) { return (v >> 7) & 2047; }
+__device__ __forceinline__ int shl_nd(int v) { return (v >> 18) & 2047; }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
@@ -540,7 +571,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* csm = reinterpret_cast<float*>(sm + L.csm);
   float* cis = reinterpret_cast<float*>(sm + L.cis);
   float* wscs = reinterpret_cast<float*>(sm + L.wscs);
-  int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = j | nsplit << 8
+  int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = shl_pack entries
   int* precs = reinterpret_cast<int*>(sm + L.precs);
   float2* xchg = reinterpret_cast<float2*>(sm + L.xchg);  // [2][C][2][128] (max, sum-exp)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
@@ -619,12 +650,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     int n = 0;
     uint32_t mw[4] = {0u, 0u, 0u, 0u};
-    // every component with direct-form moments: local index | split count << 8
-    // | direct count << 16; the mask marks those with split dimensions
+    // every component with direct-form moments (shl_pack: local index, split
+    // count, direct count); the mask marks those with split dimensions
     for (int j = 0; j < kTcComps; j++)
       if (a.ndir[k0 + j] > 0) {
         const int ns = a.nsplit[k0 + j];
-        shl[1 + n++] = j | (ns << 8) | (a.ndir[k0 + j] << 16);
+        shl[1 + n++] = shl_pack(j, ns, a.ndir[k0 + j]);
         if (ns > 0) mw[j >> 5] |= 1u << (j & 31);
       }
     shl[0] = n;
@@ -651,7 +682,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t tmem = *tslot;
   const uint32_t tL = tmem;
   const uint32_t tS = tmem + 128;
-  const uint32_t tNK = tmem + 128 + 64 * (uint32_t)nch;
+  const uint32_t tNK = tmem + 128 + 64 * (uint32_t)(FSRC == 2 ? a.nfg : nch);
 
   if (warp == kTcTmaWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -686,10 +717,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           fissued++;
           return true;
         };
+        // FSRC = 2: the features stream through the one F buffer a round of
+        // chunks [c0, c0 + n) at a time (u counts the buffer's uses)
+        auto load_round = [&](int c0, int n) -> bool {
+          if (fissued > 0 && !mbar_wait_bounded(&f_free[0], (uint32_t)((fissued - 1) & 1),
+                                                status, kAbort, a.wait_ns))
+            return false;
+          const int y = (int)(((int64_t)cid + li * ncl) * kTcRows);
+          mbar_arrive_expect_tx(&f_tx[0], 2u * (uint32_t)n * kTcChunkBytes);
+          for (int c = 0; c < n; c++) {
+            tma_load_2d(sF + (uint32_t)c * kTcChunkBytes, &tm_fhi, (c0 + c) * kTcChunk, y,
+                        &f_tx[0]);
+            tma_load_2d(sF + (L.nr + (uint32_t)c) * kTcChunkBytes, &tm_flo, (c0 + c) * kTcChunk,
+                        y, &f_tx[0]);
+          }
+          fissued++;
+          return true;
+        };
         int wi = 0;  // W loads issued for this tile
         for (int c = 0; c < nch && ok; c++)
           for (int part = 0; part < 2 && ok; part++, wi++) {
-            if (FSRC && wi == (2 * nch < kTcStages ? 2 * nch : kTcStages)) ok = load_features();
+            if (FSRC == 2 && part == 0 && c % (int)L.nr == 0)
+              ok = load_round(c, min((int)L.nr, nch - c));
+            if (FSRC == 1 && wi == (2 * nch < kTcStages ? 2 * nch : kTcStages))
+              ok = load_features();
             if (!ok) break;
             ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, status, kAbort, a.wait_ns);
             if (!ok) break;
@@ -702,7 +753,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               phase ^= 1u;
             }
           }
-        if (ok && FSRC && wi <= kTcStages && wi == 2 * nch) ok = load_features();
+        if (ok && FSRC == 1 && wi <= kTcStages && wi == 2 * nch) ok = load_features();
+        // FSRC = 2: the statistics group's chunks once more, for the statistics MMAs
+        if (FSRC == 2 && kStats)
+          for (int c = a.fg0; c < a.fg0 + a.nfgc && ok; c += (int)L.nr)
+            ok = load_round(c, min((int)L.nr, a.fg0 + a.nfgc - c));
         if (!ok) break;
       }
       // every load issued must have landed before the CTA may exit
@@ -730,6 +785,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint64_t dR = sw128_desc(rb, 8192, 1024);      // r^ as the MN-major statistics A
       const uint64_t dOnes = sw128_desc(ob, 16, 1024);
       uint32_t stage = 0, phase = 0, ndrain = 0;
+      int64_t fu = 0;  // FSRC = 2: uses of the F buffer so far (rounds)
       const bool has_split = (shl[kTcComps + 1] | shl[kTcComps + 2] | shl[kTcComps + 3] |
                               shl[kTcComps + 4]) != 0;
       for (int64_t li = 0; li < my_tiles; li++) {
@@ -742,16 +798,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         } else if (!mbar_wait_bounded(f_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) {
           break;
         }
-        if (FSRC && !mbar_wait_bounded(&f_tx[li % L.nfb], (uint32_t)((li / L.nfb) & 1), status,
-                                       kAbort, a.wait_ns))
+        if (FSRC == 1 && !mbar_wait_bounded(&f_tx[li % L.nfb], (uint32_t)((li / L.nfb) & 1),
+                                            status, kAbort, a.wait_ns))
           break;
         SCEM_TRACE(li, 8);
         tc_fence_after_sync();
         bool ok = true;
         const uint32_t fofs = (uint32_t)(li % L.nfb) * L.fbytes;  // this tile's F buffer
         for (int c = 0; c < nch && ok; c++) {
-          const uint32_t fhi = fb + fofs + (uint32_t)c * kTcChunkBytes;
-          const uint32_t flo = fb + fofs + (uint32_t)(nch + c) * kTcChunkBytes;
+          // FSRC = 2: chunk c sits in slot c mod nr of the round buffer
+          const uint32_t cs = FSRC == 2 ? (uint32_t)c % L.nr : (uint32_t)c;
+          if (FSRC == 2 && cs == 0) {
+            ok = mbar_wait_bounded(&f_tx[0], (uint32_t)(fu & 1), status, kAbort, a.wait_ns);
+            if (!ok) break;
+            tc_fence_after_sync();
+          }
+          const uint32_t fhi = fb + fofs + cs * kTcChunkBytes;
+          const uint32_t flo = fb + fofs + (L.nr + cs) * kTcChunkBytes;
           for (int part = 0; part < 2; part++) {
             ok = mbar_wait_bounded(&full[stage], phase, status, kAbort, a.wait_ns);
             if (!ok) break;
@@ -770,17 +833,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               phase ^= 1u;
             }
           }
+          // FSRC = 2: the round's last chunk is issued; the buffer is free once it is done
+          if (FSRC == 2 && ok && (cs + 1 == L.nr || c + 1 == nch)) {
+            mma_commit(&f_free[0]);
+            fu++;
+          }
         }
         if (!ok) break;
         if (kOverlap) {
           mma_commit(&l_full2[lb]);
           // the F buffer is free once the E-step is done with it -- or, where
           // split dimensions' filter reads it, once both row halves' epilogues are
-          if (has_split &&
-              !(mbar_wait_bounded(r_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns) &&
-                mbar_wait_bounded(r_full1, (uint32_t)(li & 1), status, kAbort, a.wait_ns)))
-            break;
-          mma_commit(&f_free[li % L.nfb]);
+          if (FSRC == 1) {
+            if (has_split &&
+                !(mbar_wait_bounded(r_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns) &&
+                  mbar_wait_bounded(r_full1, (uint32_t)(li & 1), status, kAbort, a.wait_ns)))
+              break;
+            mma_commit(&f_free[li % L.nfb]);
+          }
           continue;
         }
         mma_commit(l_full);
@@ -789,7 +859,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         SCEM_TRACE(li, 10);
         tc_fence_after_sync();
         bool ok2 = true;
-        if (kStats) {
+        if (kStats && FSRC == 2) {
+          // both 64-row halves of r^ are written (the buffer holds all 128 rows)
+          if (!mbar_wait_bounded(r_full1, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) break;
+          if (li > 0) {
+            if (!mbar_wait_bounded(drained, ndrain & 1u, status, kAbort, a.wait_ns)) break;
+            ndrain++;
+          }
+          tc_fence_after_sync();
+          const bool first = li == 0;
+          for (int c0 = a.fg0; c0 < a.fg0 + a.nfgc && ok2; c0 += (int)L.nr) {
+            const int n = min((int)L.nr, a.fg0 + a.nfgc - c0);
+            ok2 = mbar_wait_bounded(&f_tx[0], (uint32_t)(fu & 1), status, kAbort, a.wait_ns);
+            if (!ok2) break;
+            tc_fence_after_sync();
+            const uint32_t idSr = idesc_f16_f32(128, 64 * n, true, true);
+            const uint32_t tSr = tS + 64u * (uint32_t)(c0 - a.fg0);
+#pragma unroll 1
+            for (int k8 = 0; k8 < 8; k8++) {  // 16-row K-steps over the 128 rows
+              const uint32_t hofs = 32768u * (uint32_t)(k8 >> 2);
+              const uint64_t ahi = desc_add(dR, hofs + 2048u * (k8 & 3));
+              const uint64_t alo = desc_add(dR, hofs + 16384u + 2048u * (k8 & 3));
+              const bool acc = !(first && k8 == 0);
+              const uint32_t kr = 2048u * (uint32_t)k8;  // F rows of this K-step
+              const uint64_t fhi = desc_add(dFs, kr);
+              const uint64_t flo = desc_add(dFs, L.nr * kTcChunkBytes + kr);
+              mma_bf16(tSr, ahi, fhi, idSr, acc);
+              mma_bf16(tSr, ahi, flo, idSr, true);
+              mma_bf16(tSr, alo, fhi, idSr, true);
+              if (c0 == a.fg0) {
+                mma_bf16(tNK, ahi, dOnes, idN, acc);
+                mma_bf16(tNK, alo, dOnes, idN, true);
+              }
+            }
+            mma_commit(&f_free[0]);
+            fu++;
+          }
+        } else if (kStats) {
           const bool first = li == 0;  // later tiles add onto whatever the drains left
           if (li > 0) {
             if (!mbar_wait_bounded(drained, ndrain & 1u, status, kAbort, a.wait_ns)) break;
@@ -824,7 +930,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         if (!ok2) break;
         mma_commit(s_done);
-        if (FSRC) mma_commit(&f_free[li % L.nfb]);
+        if (FSRC == 1) mma_commit(&f_free[li % L.nfb]);
         SCEM_TRACE(li, 11);
       }
       // every MMA issued must be complete before tensor memory is released
@@ -873,7 +979,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       double* sk = slot + k;
       if (hf == 0) {
         if (due) {
-          if (vn[0] != 0.f) atomicAdd(sk + (size_t)(2 * D) * K, (double)vn[0]);
+          // (streamed features: N_k is the same in every group's pass; the first adds it)
+          if (vn[0] != 0.f && (FSRC != 2 || a.fg0 == 0))
+            atomicAdd(sk + (size_t)(2 * D) * K, (double)vn[0]);
 #pragma unroll
           for (int j = 0; j < 32; j++) vn[j] = 0.f;
         }
@@ -881,21 +989,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (t == 0) SCEM_TRACE(li, 15);
       const uint32_t* pm = a.pmask + (size_t)(due ? k : 0) * (2 * nch);
-      uint32_t mw[kTcMaxChunks];
-#pragma unroll
-      for (int c = 0; c < kTcMaxChunks; c++)
-        mw[c] = (!due || c >= nch) ? 0u : (force ? 0xffffffffu : __ldg(pm + 2 * c + hf));
-      for (int c = 0; c < nch; c++) {
-        uint32_t mask = mw[0];
-#pragma unroll
-        for (int c2 = 1; c2 < kTcMaxChunks; c2++)
-          if (c == c2) mask = mw[c2];
+      // the feature chunks in tensor memory: all, or this pass's statistics group
+      const int cbase = FSRC == 2 ? a.fg0 : 0, nchl = FSRC == 2 ? a.nfgc : nch;
+      for (int c = 0; c < nchl; c++) {
+        const uint32_t mask =
+            !due ? 0u : (force ? 0xffffffffu : __ldg(pm + 2 * (cbase + c) + hf));
         if (!__any_sync(0xffffffffu, mask != 0u)) continue;  // nothing of this block is due
         float v[32];
         const uint32_t cc = tS + lane_base + 64u * c + 32u * hf;
         tmem_ld32(cc, v);
         if (mask) {
-          const int f0 = 64 * c + 32 * hf;
+          const int f0 = 64 * (cbase + c) + 32 * hf;
           const int nf = min(32, 2 * D - f0);  // features of this column block that exist
 #pragma unroll
           for (int j = 0; j < 32; j++)
@@ -1135,14 +1239,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // the filter tables of every split component head for L1 now (one lane
         // per component), so the per-component loop below meets L1, not L2
         for (int sj = lane; sj < nsh; sj += 32) {
-          if (((shl[1 + sj] >> 8) & 255) == 0) continue;
-          const size_t base = (size_t)(k0 + (shl[1 + sj] & 255)) * D;
+          if (shl_ns(shl[1 + sj]) == 0) continue;
+          const size_t base = (size_t)(k0 + shl_j(shl[1 + sj])) * D;
           prefetch_l1(a.perm + base);
           prefetch_l1(a.mhp + base);
           prefetch_l1(a.php + base);
         }
         for (int si = 0; si < nsh; si++) {
-          const int j = shl[1 + si] & 255, ns = (shl[1 + si] >> 8) & 255;
+          const int j = shl_j(shl[1 + si]), ns = shl_ns(shl[1 + si]);
           if ((j >> 6) != hf || ns == 0) continue;
           const size_t base = (size_t)(k0 + j) * D;
           const float v0 = tmem_ld1(tLc + lane_base + (uint32_t)j);
@@ -1156,16 +1260,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // exceeds qmax by more than that bound is below the floor, and its
           // exact sum is not needed.
           bool far = !rvalid || !(qmax >= 0.f);
-          if (!far) {
+          if (!far && FSRC != 2) {  // (streamed features are not resident: exact sums only)
             const float sq_max = sqrtf(qmax);
             float qa = 0.f, eb = 0.f;
             for (int i0 = 0; i0 < ns && !far; i0 += 16) {
-              uchar4 pp[4];
+              ushort4 pp[4];
               float4 m4[4], p4[4];
 #pragma unroll
               for (int g4 = 0; g4 < 4; g4++) {
                 const int i = min(i0 + 4 * g4, D - 4);  // in range; entries past ns are not summed
-                pp[g4] = __ldg(reinterpret_cast<const uchar4*>(a.perm + base + i));
+                pp[g4] = __ldg(reinterpret_cast<const ushort4*>(a.perm + base + i));
                 m4[g4] = __ldg(reinterpret_cast<const float4*>(a.mhp + base + i));
                 p4[g4] = __ldg(reinterpret_cast<const float4*>(a.php + base + i));
               }
@@ -1199,7 +1303,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int g4 = 0; g4 < 4; g4++) {
               const int i = min(i0 + 4 * g4, D - 4);
-              const uchar4 pp = __ldg(reinterpret_cast<const uchar4*>(a.perm + base + i));
+              const ushort4 pp = __ldg(reinterpret_cast<const ushort4*>(a.perm + base + i));
               x4[g4][0] = load1<XT>(xrow, min((int)pp.x, D - 1));
               x4[g4][1] = load1<XT>(xrow, min((int)pp.y, D - 1));
               x4[g4][2] = load1<XT>(xrow, min((int)pp.z, D - 1));
@@ -1322,7 +1426,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float lse = kHard ? M : M + __logf(S);
       if (MODE == kTcTopm && valid && rank == 0 && hf == 0 && grp == 0)
         a.rowst[row0 + row] = make_float2(M, S);
-      if (!kPartial && MODE != kTcTopm && valid && rank == 0 && hf == 0 && grp == 0) {
+      if (!kPartial && MODE != kTcTopm && valid && rank == 0 && hf == 0 && grp == 0 &&
+          (FSRC != 2 || a.fg0 == 0)) {
         ll += (double)lse;
         if (kHard && a.labels) a.labels[row0 + row] = win < K ? win : -1;
       }
@@ -1336,7 +1441,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int hr = row >> 6, rr = row & 63;  // which 64-row half of r^, row within it
       uint64_t rbits = 0;  // the thread's columns whose r exceeds kTcDirRmin
       if (kStats) {
-        if (hr == 1) {
+        if (FSRC != 2 && hr == 1) {
           // the first half's MMAs must be done with the buffer
           ok = __all_sync(0xffffffffu, mbar_wait_bounded(r_free, (uint32_t)(li & 1), status,
                                                          kAbort, a.wait_ns));
@@ -1349,8 +1454,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           split_half2(e[8 * q8 + 2] * scale, e[8 * q8 + 3] * scale, ph4.y, pl4.y);
           split_half2(e[8 * q8 + 4] * scale, e[8 * q8 + 5] * scale, ph4.z, pl4.z);
           split_half2(e[8 * q8 + 6] * scale, e[8 * q8 + 7] * scale, ph4.w, pl4.w);
-          const uint32_t off = (uint32_t)hf * 8192u + (uint32_t)rr * 128u +
-                               ((((uint32_t)q8) ^ ((uint32_t)rr & 7u)) << 4);
+          const uint32_t off = (FSRC == 2 ? 32768u * (uint32_t)hr : 0u) + (uint32_t)hf * 8192u +
+                               (uint32_t)rr * 128u + ((((uint32_t)q8) ^ ((uint32_t)rr & 7u)) << 4);
           *reinterpret_cast<uint4*>(sR + off) = ph4;
           *reinterpret_cast<uint4*>(sR + 16384u + off) = pl4;
         }
@@ -1371,13 +1476,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // hold the next tile once the statistics MMAs are done.)  They go into
       // the shared fixed-point area (kTcDirScale), so the order in which rows
       // and clusters add them does not change the sums.
-      if (kStats && shl[0] > 0) {
+      if (kStats && shl[0] > 0 && (FSRC != 2 || a.fg0 == 0)) {
         const int nsh = shl[0];
         const XT* xrow = reinterpret_cast<const XT*>(a.X) + (size_t)(valid ? row0 + row : 0) * D;
         const size_t kp = (size_t)a.Kpad;
         for (int si = 0; si < nsh; si++) {
-          const int j = shl[1 + si] & 255, ns = (shl[1 + si] >> 8) & 255, nd = shl[1 + si] >> 16;
-          if ((j >> 6) != hf || !((rbits >> (j & 63)) & 1ull)) continue;
+          const int j = shl_j(shl[1 + si]), ns = shl_ns(shl[1 + si]), nd = shl_nd(shl[1 + si]);
+          if ((j >> 6) != hf || nd == 0) continue;
+          // skipped only when no row of the warp needs it: the tensor-memory
+          // load below is a warp-collective (.sync.aligned) instruction
+          if (!__any_sync(0xffffffffu, (rbits >> (j & 63)) & 1ull)) continue;
           // the log-joint: finished in tensor memory for a component with split
           // dimensions, the raw accumulator (scaled as the epilogue scales it) otherwise
           const float v0 = tmem_ld1(tLc + lane_base + (uint32_t)j);
@@ -1482,7 +1590,11 @@ __global__ void __launch_bounds__(256) tc_center_kernel(int D, int K, const floa
   sc_out[d] = ldexpf(1.0f, e);
 }
 
-// One block per (padded) component, one thread per dimension (D <= 128).
+inline size_t tc_prep_smem_bytes(int D, int Fpad) {
+  return (size_t)(4 * D + 2 * Fpad) * sizeof(double) + (size_t)D * sizeof(int);
+}
+
+// One block of 128 threads per (padded) component, looping over the dimensions.
 //
 // Direct-form split.  The expanded form's fp32 error grows with
 // kappa_k = sum_d (mu^_kd^2 + 1)/var^_kd.  When kappa_k exceeds kTcSharpKappa (a
@@ -1517,13 +1629,19 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     __half* __restrict__ whi, __half* __restrict__ wlo, float* __restrict__ c_out,
     float* __restrict__ wsc_out, int* __restrict__ ndir_out, int* __restrict__ nsplit_out,
     float* __restrict__ muh, float* __restrict__ ph, int* __restrict__ precise_out,
-    float* __restrict__ ci_out, uint8_t* __restrict__ perm_out, float* __restrict__ mhp_out,
-    float* __restrict__ php_out, uint32_t* __restrict__ pmask_out, uint8_t* __restrict__ rank_out,
+    float* __restrict__ ci_out, uint16_t* __restrict__ perm_out, float* __restrict__ mhp_out,
+    float* __restrict__ php_out, uint32_t* __restrict__ pmask_out, uint16_t* __restrict__ rank_out,
     unsigned long long* __restrict__ dirq, unsigned int* status) {
-  __shared__ double mh_s[kTcMaxD], vh_s[kTcMaxD], kd_s[kTcMaxD], ksort[kTcMaxD];
-  __shared__ int rank_s[kTcMaxD];
-  __shared__ double wv[kTcChunk * kTcMaxChunks];  // Fpad <= 256
-  __shared__ double ef[kTcChunk * kTcMaxChunks];  // E[F] under the component
+  // dynamic shared memory (tc_prep_smem_bytes): per dimension mu^, var^, kappa_kd and
+  // kappa sorted (doubles) and the rank (int); per feature W and E[F] (doubles)
+  extern __shared__ double prep_sm[];
+  double* mh_s = prep_sm;
+  double* vh_s = mh_s + D;
+  double* kd_s = vh_s + D;
+  double* ksort = kd_s + D;
+  double* wv = ksort + D;    // Fpad
+  double* ef = wv + Fpad;    // Fpad: E[F] under the component
+  int* rank_s = reinterpret_cast<int*>(ef + Fpad);
   __shared__ double red[4][4];
   __shared__ int ns_s, nd_s;
   const int k = blockIdx.x;
@@ -1585,9 +1703,9 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     }
     rank_s[d] = r;
     ksort[r] = key;
-    rank_out[(size_t)k * D + d] = (uint8_t)r;
+    rank_out[(size_t)k * D + d] = (uint16_t)r;
     const size_t o = (size_t)k * D + r;
-    perm_out[o] = (uint8_t)d;
+    perm_out[o] = (uint16_t)d;
     mhp_out[o] = (float)mh_s[d];
     php_out[o] = (float)(1.0 / vh_s[d]);
     muh[o] = k < K ? mu[(size_t)k * D + d] : 0.f;
@@ -1690,7 +1808,7 @@ __device__ __forceinline__ double fixed_value(unsigned long long hi, unsigned lo
 // stored ph the fused pass divided by.
 __global__ void __launch_bounds__(256) tc_reduce_stats_kernel(
     int D, int K, int Kpad, const float* __restrict__ m, const float* __restrict__ sc,
-    const float* __restrict__ mu, const uint8_t* __restrict__ rank,
+    const float* __restrict__ mu, const uint16_t* __restrict__ rank,
     const int* __restrict__ ndir, const float* __restrict__ ph,
     const unsigned long long* __restrict__ dirq, const double* __restrict__ slots,
     size_t slot_stride, int nslots, int G, int group_comps, double* __restrict__ stats) {

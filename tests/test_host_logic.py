@@ -193,8 +193,8 @@ def test_tensor_core_shape_limits_and_f_buffers(tmp_path):
     assert [r[0] for r in rows] == list(range(4, 129, 4))
     for D, maxk, nfb256, nfb1024, nfbmax, c4096, g4096 in rows:
         assert maxk == (2048 if D <= 64 else 1280 if D <= 96 else 256), D
-        # K = 4096 takes component groups of one cluster each, the fewest that fit
-        assert (c4096, g4096) == ((16, 2) if D <= 64 else (8, 4) if D <= 96 else (2, 16)), D
+        # K = 4096 takes component groups of one cluster each, of at most 4 CTAs
+        assert (c4096, g4096) == ((4, 8) if D <= 96 else (2, 16)), D
         if D <= 32:  # two F buffers at every K
             assert (nfb256, nfb1024, nfbmax) == (2, 2, 2), D
         elif D <= 64:  # two only at small K, where the cluster is small enough
