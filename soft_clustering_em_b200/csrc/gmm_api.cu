@@ -197,8 +197,8 @@ gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const 
   tc_center_kernel<<<p->D, 256, 0, st>>>(p->D, p->K, w, mu, var, m,
                                                        (float*)(ws + T.isc), (float*)(ws + T.sc));
   const size_t psmem = tc_prep_smem_bytes(p->D, T.Fpad);
-  if (psmem > 48 * 1024 &&
-      cudaFuncSetAttribute(tc_prep_w_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  // (set every time: the static shared memory adds to the dynamic size)
+  if (cudaFuncSetAttribute(tc_prep_w_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)psmem) != cudaSuccess) {
     cudaGetLastError();
     return GMM_ERR_UNSUPPORTED;
@@ -207,7 +207,8 @@ gmm_status tc_prep(const gmm_problem* p, const float* w, const float* mu, const 
       p->N, p->D, p->K, T.Fpad, w, mu, var, m, (const float*)(ws + T.sc), (__half*)(ws + T.whi),
       (__half*)(ws + T.wlo), (float*)(ws + T.c), (float*)(ws + T.wsc), (int*)(ws + T.ndir),
       (int*)(ws + T.nsplit), (float*)(ws + T.muh), (float*)(ws + T.ph), (int*)(ws + T.precise),
-      (float*)(ws + T.ci), (uint16_t*)(ws + T.perm), (float*)(ws + T.mhp), (float*)(ws + T.php),
+      (float*)(ws + T.ci), (float*)(ws + T.cx), (float*)(ws + T.mg), (uint16_t*)(ws + T.perm),
+      (float*)(ws + T.mun), (float*)(ws + T.pn),
       (uint32_t*)(ws + T.pmask), (uint16_t*)(ws + T.rank), (unsigned long long*)(ws + T.dirq),
       (unsigned int*)ws);
   return launched(2);
@@ -310,8 +311,10 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, int64_t N, char* ws, c
   args.muh = (const float*)(ws + T.muh);
   args.ph = (const float*)(ws + T.ph);
   args.perm = (const uint16_t*)(ws + T.perm);
-  args.mhp = (const float*)(ws + T.mhp);
-  args.php = (const float*)(ws + T.php);
+  args.mun = (const float*)(ws + T.mun);
+  args.pn = (const float*)(ws + T.pn);
+  args.cx = (const float*)(ws + T.cx);
+  args.mg = (const float*)(ws + T.mg);
   args.slots = (double*)(ws + T.slots);
   args.slot_stride = T.slot_stride;
   args.dirq = (unsigned long long*)(ws + T.dirq);

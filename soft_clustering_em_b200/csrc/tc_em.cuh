@@ -133,12 +133,12 @@ constexpr float kTcXMax = 240.0f;                // |x^| beyond this cannot be s
 constexpr double kTcStartFrac = -0.625;
 // Fixed-point unit of the split dimensions' direct-form moments: each row's
 // r (x - mu) / sigma and r (x - mu)^2 / sigma^2 is rounded to a multiple of
-// 2^-32 and added as a signed 64-bit integer split into a high word
-// (q >> 32, signed) and a low word (q mod 2^32), each summed with a 64-bit
-// integer atomic.  Integer sums do not depend on the order of the additions,
-// so the result is deterministic whatever the scheduling; the rounding is
-// 2^-33 of a standard deviation per row, and the low-word sum stays exact for
-// up to 2^31 contributing rows per component.
+// 2^-32; a warp's sum of those integers is added as a high word (q >> 32,
+// signed) and a low word (q mod 2^32), each summed with a 64-bit integer
+// atomic.  Integer sums do not depend on the order of the additions, so the
+// result is deterministic whatever the scheduling; the rounding is 2^-33 of a
+// standard deviation per row, and the low-word sum stays exact for up to 2^31
+// contributing warps per component.
 constexpr double kTcDirScale = 4294967296.0;  // 2^32
 
 // kTcStats: E-step, responsibilities and statistics (with G > 1 component
@@ -207,7 +207,8 @@ __host__ __device__ inline bool tc_streamed(int nchunks) { return nchunks > kTcM
 // features can be written while the previous tile's statistics MMAs still
 // read the other buffer.
 struct TcSmem {
-  uint32_t F, W, R, ONES, msm, iscs, csm, cis, wscs, shl, precs, xchg, bars, tslot, total;
+  uint32_t F, W, R, ONES, msm, iscs, csm, cis, wscs, cxs, mgs, shl, precs, xchg, bars, tslot,
+      total;
   uint32_t nfb, fbytes;
   uint32_t nr;  // feature chunks an F buffer holds: all of them, or a round when streamed
 };
@@ -240,6 +241,10 @@ __host__ __device__ inline TcSmem tc_smem_layout_n(int D, int C, int nchunks, ui
   L.cis = off;
   off += kTcComps * 4;
   L.wscs = off;
+  off += kTcComps * 4;
+  L.cxs = off;
+  off += kTcComps * 4;
+  L.mgs = off;
   off += kTcComps * 4;
   L.shl = off;
   off += (kTcComps + 8) * 4;
@@ -277,13 +282,16 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //   perm : [C*128 x D] u16 dimensions of each component by decreasing
 //          (mu^^2 + 1)/var^
 //   muh, ph : [C*128 x D] f32 mu and 1/var (data units) in perm order
-//   mhp, php : [C*128 x D] f32 mu^ and 1/var^ in perm order
+//   mun, pn : [C*128 x D] f32 mu and 1/var (data units) in natural order
+//   cx   : C*128 f32 log pi_k - 1/2 sum_d log(2 pi var_kd): the direct form's constant
+//   mg   : C*128 f32 bound on the error of the contraction's log-joint of a
+//          component with exact log-joints (see tc_prep_w_kernel), 0 for the others
 //   whi, wlo : [C*128 x 64*nchunks] fp16 operand W (hi and lo parts)
 //   rank : [C*128 x D] u16 position of each dimension in perm
-//   dirq : [4D x C*128] u64 direct-form moments of split dimensions about the
+//   dirq : [C*128 x 4D] u64 direct-form moments of split dimensions about the
 //          input means, by perm position i, as 64-bit fixed-point words (see
-//          kTcDirScale): rows i / D+i hold the high / low words of
-//          sum r (x - mu) / sigma, rows 2D+i / 3D+i those of
+//          kTcDirScale): per component, words i / D+i hold the high / low
+//          words of sum r (x - mu) / sigma, words 2D+i / 3D+i those of
 //          sum r (x - mu)^2 / sigma^2.  One area for all clusters: integer
 //          additions commute, so the sums do not depend on the order in which
 //          rows or clusters add them.  Zeroed by tc_prep_w_kernel.
@@ -298,7 +306,8 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //   cand     : [Rt x (G C 2) x kTcCand] float2 (log-joint, index) candidates
 //   rowst    : [Rt] float2 (max, sum-exp) of each row
 struct TcLayout {
-  size_t m, isc, sc, c, ci, wsc, ndir, nsplit, precise, pmask, muh, ph, perm, rank, mhp, php, whi,
+  size_t m, isc, sc, c, ci, wsc, cx, mg, ndir, nsplit, precise, pmask, muh, ph, perm, rank, mun, pn,
+      whi,
       wlo, dirq, slots, fhi, flo, part, cand, rowst, total, slot_stride;
   int C, G, nchunks, Kpad, Fpad, P;
   int nfg, NFG;  // feature chunks per statistics group, and groups (1 unless streamed)
@@ -364,6 +373,10 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.wsc = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
+  L.cx = off;
+  off = align_up(off + (size_t)L.Kpad * 4, 256);
+  L.mg = off;
+  off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.ndir = off;
   off = align_up(off + (size_t)L.Kpad * 4, 256);
   L.nsplit = off;
@@ -376,9 +389,9 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   off = align_up(off + (size_t)L.Kpad * D * 2, 256);
   L.rank = off;
   off = align_up(off + (size_t)L.Kpad * D * 2, 256);
-  L.mhp = off;
+  L.mun = off;
   off = align_up(off + (size_t)L.Kpad * D * 4, 256);
-  L.php = off;
+  L.pn = off;
   off = align_up(off + (size_t)L.Kpad * D * 4, 256);
   L.whi = off;
   off = align_up(off + (size_t)L.Kpad * L.Fpad * 2, 256);
@@ -441,8 +454,10 @@ struct TcArgs {
   const float* muh;     // mu (data units) in perm order, C*128 x D
   const float* ph;      // 1/var (data units) in perm order, C*128 x D
   const uint16_t* perm;  // dimensions by decreasing (mu^^2 + 1)/var^, C*128 x D
-  const float* mhp;     // mu^ in that order, C*128 x D
-  const float* php;     // 1/var^ in that order, C*128 x D
+  const float* mun;     // mu (data units), C*128 x D
+  const float* pn;      // 1/var (data units), C*128 x D
+  const float* cx;      // direct-form constants, C*128
+  const float* mg;      // error bounds of the contraction's log-joints, C*128
   double* slots;        // per-cluster statistic slots
   size_t slot_stride;   // doubles per slot: (2D+1)*K statistics + LL
   unsigned long long* dirq;  // fixed-point direct-form moments of split dimensions, 4D x Kpad
@@ -484,14 +499,6 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 }
 
 __device__ __forceinline__ float round_half(float a) { return __half2float(__float2half_rn(a)); }
-
-// Adds v (already in units of 2^-32) to the fixed-point pair (hi, lo).
-__device__ __forceinline__ void fixed_add(unsigned long long* hi, unsigned long long* lo,
-                                          double v) {
-  const long long q = __double2ll_rn(v);
-  atomicAdd(hi, (unsigned long long)(q >> 32));
-  atomicAdd(lo, (unsigned long long)(q & 0xffffffffll));
-}
 
 // (a, b) -> fp16 pairs hi = fp16(a, b) and lo = fp16(a - hi_a, b - hi_b), packed:
 // three conversion instructions for two values.
@@ -571,6 +578,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* csm = reinterpret_cast<float*>(sm + L.csm);
   float* cis = reinterpret_cast<float*>(sm + L.cis);
   float* wscs = reinterpret_cast<float*>(sm + L.wscs);
+  float* cxs = reinterpret_cast<float*>(sm + L.cxs);
+  float* mgs = reinterpret_cast<float*>(sm + L.mgs);
   int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = shl_pack entries
   int* precs = reinterpret_cast<int*>(sm + L.precs);
   float2* xchg = reinterpret_cast<float2*>(sm + L.xchg);  // [2][C][2][128] (max, sum-exp)
@@ -645,6 +654,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     csm[i] = a.c[k0 + i];
     cis[i] = a.ci[k0 + i];
     wscs[i] = a.wsc[k0 + i];
+    cxs[i] = a.cx[k0 + i];
+    mgs[i] = a.mg[k0 + i];
     precs[i] = a.precise[k0 + i];
   }
   if (tid == 0) {
@@ -1203,9 +1214,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float e[64];
       float mx = -INFINITY;
       // first pass (final = false): every column is an accumulator value,
-      // scaled to a log-joint; columns in the mask (split components) stay out
-      // of the max.  Second pass (final = true): the masked columns already
-      // hold finished log-joints.
+      // scaled to a log-joint; the max is a lower bound of the half's best
+      // log-joint (columns in the mask, components with exact log-joints,
+      // count less their error bound mg).  Second pass (final = true): the
+      // masked columns already hold exact log-joints (or -inf).
       auto load_logits = [&](bool final, uint32_t m0, uint32_t m1) {
         mx = -INFINITY;
 #pragma unroll
@@ -1218,7 +1230,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int cidx = col0 + 32 * q + j;
             const bool masked = (mq >> j) & 1u;
             e[32 * q + j] = (final && masked) ? v[j] : fmaf(v[j], wscs[cidx], csm[cidx]);
-            if (final || !masked) mx = fmaxf(mx, e[32 * q + j]);
+            mx = fmaxf(mx, (final || !masked) ? e[32 * q + j] : e[32 * q + j] - mgs[cidx]);
           }
         }
       };
@@ -1226,105 +1238,51 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      sm1 = (uint32_t)shl[kTcComps + 2 + 2 * hf];
       load_logits(false, sm0, sm1);
       if (sm0 | sm1) {
-        // Components of this column half with split dimensions: the tensor
-        // cores gave the log-joint over their other dimensions; add
-        // -1/2 sum (x - mu)^2/var over the split ones, in data units.  A row
-        // whose log-joint falls 80 nats below the best component of the half
-        // without split dimensions has responsibility 0 and gets -inf.
+        // Components of this column half with exact log-joints.  A row whose
+        // contraction value, plus its error bound, falls 80 nats below the
+        // half's lower bound has responsibility 0 and gets -inf; for the rows
+        // near the component the warp computes the log-joint in direct form
+        // from X, one row at a time, its lanes over the dimensions, the
+        // per-lane sums added in a fixed butterfly order.
         const float floor_l = mx - 80.f;
         const int nsh = shl[0];
         const bool rvalid = row0 + row < a.N;
-        const XT* xrow = reinterpret_cast<const XT*>(a.X) + (size_t)(rvalid ? row0 + row : 0) * D;
-        const uint32_t lo_off = (uint32_t)nch * kTcChunkBytes;
-        // the filter tables of every split component head for L1 now (one lane
-        // per component), so the per-component loop below meets L1, not L2
-        for (int sj = lane; sj < nsh; sj += 32) {
-          if (shl_ns(shl[1 + sj]) == 0) continue;
-          const size_t base = (size_t)(k0 + shl_j(shl[1 + sj])) * D;
-          prefetch_l1(a.perm + base);
-          prefetch_l1(a.mhp + base);
-          prefetch_l1(a.php + base);
-        }
+        const XT* xw = reinterpret_cast<const XT*>(a.X) + (size_t)(row0 + 32 * qd) * D;
         for (int si = 0; si < nsh; si++) {
           const int j = shl_j(shl[1 + si]), ns = shl_ns(shl[1 + si]);
           if ((j >> 6) != hf || ns == 0) continue;
-          const size_t base = (size_t)(k0 + j) * D;
           const float v0 = tmem_ld1(tLc + lane_base + (uint32_t)j);
-          const float lr = fmaf(v0, wscs[j], csm[j]);  // log-joint over the kept dimensions
-          const float qmax = 2.f * (lr - floor_l);      // split sum beyond this: below the floor
-          // Filter: the row's own features x^ = F_hi + F_lo (shared memory).
-          // With a = x^ - mu^ and the feature's error |da_d| <= e_d =
-          // 2^-20 (|x^_d| + |mu^_d|) + 2^-24 (fp32 x^, the fp16 split, fp32
-          // mu^), the weighted norms obey |sqrt(q~) - sqrt(q)| <=
-          // sqrt(sum_d e_d^2 / var^_d); a row whose approximate split sum
-          // exceeds qmax by more than that bound is below the floor, and its
-          // exact sum is not needed.
-          bool far = !rvalid || !(qmax >= 0.f);
-          if (!far && FSRC != 2) {  // (streamed features are not resident: exact sums only)
-            const float sq_max = sqrtf(qmax);
-            float qa = 0.f, eb = 0.f;
-            for (int i0 = 0; i0 < ns && !far; i0 += 16) {
-              ushort4 pp[4];
-              float4 m4[4], p4[4];
-#pragma unroll
-              for (int g4 = 0; g4 < 4; g4++) {
-                const int i = min(i0 + 4 * g4, D - 4);  // in range; entries past ns are not summed
-                pp[g4] = __ldg(reinterpret_cast<const ushort4*>(a.perm + base + i));
-                m4[g4] = __ldg(reinterpret_cast<const float4*>(a.mhp + base + i));
-                p4[g4] = __ldg(reinterpret_cast<const float4*>(a.php + base + i));
-              }
-#pragma unroll
-              for (int g4 = 0; g4 < 4; g4++) {
-                const int fs[4] = {pp[g4].x, pp[g4].y, pp[g4].z, pp[g4].w};
-                const float ms[4] = {m4[g4].x, m4[g4].y, m4[g4].z, m4[g4].w};
-                const float ps[4] = {p4[g4].x, p4[g4].y, p4[g4].z, p4[g4].w};
-#pragma unroll
-                for (int u = 0; u < 4; u++) {
-                  if (i0 + 4 * g4 + u >= ns) break;
-                  const int f = min(fs[u], D - 1);
-                  const uint32_t o = (uint32_t)(f >> 6) * kTcChunkBytes + sw128_offset(row, f & 63);
-                  const float xh = __half2float(*reinterpret_cast<const __half*>(sFc + o)) +
-                                   __half2float(*reinterpret_cast<const __half*>(sFc + lo_off + o));
-                  const float dd = xh - ms[u];
-                  qa = fmaf(dd * dd, ps[u], qa);
-                  const float ed = 9.6e-7f * (fabsf(xh) + fabsf(ms[u])) + 6.0e-8f;
-                  eb = fmaf(ed * ed, ps[u], eb);
-                  if (fabsf(xh) >= kTcXMax) eb = INFINITY;  // clamped feature: no bound
-                }
-              }
-              far = sqrtf(qa) * 0.99999f > sq_max + 1.01f * sqrtf(eb) + 1e-3f;
+          const float la = fmaf(v0, wscs[j], csm[j]);  // the contraction's log-joint
+          const bool near = rvalid && la > -INFINITY && la + mgs[j] >= floor_l;
+          uint32_t nm = __ballot_sync(0xffffffffu, near);
+          const float* muk = a.mun + (size_t)(k0 + j) * D;
+          const float* pk = a.pn + (size_t)(k0 + j) * D;
+          float lx = -INFINITY;
+          while (nm != 0u) {
+            // two rows at a time, so that their loads overlap
+            const int s0 = __ffs(nm) - 1;
+            nm &= nm - 1u;
+            const int s1 = nm != 0u ? __ffs(nm) - 1 : -1;
+            if (s1 >= 0) nm &= nm - 1u;
+            const XT* x0 = xw + (size_t)s0 * D;
+            const XT* x1 = xw + (size_t)(s1 >= 0 ? s1 : s0) * D;
+            float q0 = 0.f, q1 = 0.f;
+            for (int d = lane; d < D; d += 32) {
+              const float mu_d = __ldg(muk + d), p_d = __ldg(pk + d);
+              const float e0 = load1<XT>(x0, d) - mu_d, e1 = load1<XT>(x1, d) - mu_d;
+              q0 = fmaf(e0 * e0, p_d, q0);
+              q1 = fmaf(e1 * e1, p_d, q1);
             }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              q0 += __shfl_xor_sync(0xffffffffu, q0, o);
+              q1 += __shfl_xor_sync(0xffffffffu, q1, o);
+            }
+            if (lane == s0) lx = cxs[j] - 0.5f * q0;
+            if (lane == s1) lx = cxs[j] - 0.5f * q1;
           }
-          // exact split sum in data units from X, 16 dimensions per step
-          float q = far ? INFINITY : 0.f;
-          for (int i0 = 0; i0 < ns && q <= qmax; i0 += 16) {
-            float x4[4][4];
-            float4 m4[4], p4[4];
-#pragma unroll
-            for (int g4 = 0; g4 < 4; g4++) {
-              const int i = min(i0 + 4 * g4, D - 4);
-              const ushort4 pp = __ldg(reinterpret_cast<const ushort4*>(a.perm + base + i));
-              x4[g4][0] = load1<XT>(xrow, min((int)pp.x, D - 1));
-              x4[g4][1] = load1<XT>(xrow, min((int)pp.y, D - 1));
-              x4[g4][2] = load1<XT>(xrow, min((int)pp.z, D - 1));
-              x4[g4][3] = load1<XT>(xrow, min((int)pp.w, D - 1));
-              m4[g4] = __ldg(reinterpret_cast<const float4*>(a.muh + base + i));
-              p4[g4] = __ldg(reinterpret_cast<const float4*>(a.ph + base + i));
-            }
-#pragma unroll
-            for (int g4 = 0; g4 < 4; g4++) {
-              const float ms[4] = {m4[g4].x, m4[g4].y, m4[g4].z, m4[g4].w};
-              const float ps[4] = {p4[g4].x, p4[g4].y, p4[g4].z, p4[g4].w};
-#pragma unroll
-              for (int u = 0; u < 4; u++) {
-                if (i0 + 4 * g4 + u >= ns) break;
-                const float e0 = x4[g4][u] - ms[u];
-                q = fmaf(e0 * e0, ps[u], q);
-              }
-            }
-          }
-          // the finished log-joint (the second load_logits takes it as is)
-          tmem_st1(tLc + lane_base + (uint32_t)j, q <= qmax ? lr - 0.5f * q : -INFINITY);
+          // the exact log-joint (the second load_logits takes it as is)
+          tmem_st1(tLc + lane_base + (uint32_t)j, lx);
         }
         load_logits(true, sm0, sm1);
       }
@@ -1471,15 +1429,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (t == 0) SCEM_TRACE(li, 7);
       // Moments of split dimensions in direct form, about the input means, in
       // data units from X (no cancellation however narrow the dimension),
-      // while the statistics MMAs run.  Only rows with a finite log-joint for
-      // the component contribute: the few near it.  (X, not F: F may already
-      // hold the next tile once the statistics MMAs are done.)  They go into
-      // the shared fixed-point area (kTcDirScale), so the order in which rows
-      // and clusters add them does not change the sums.
+      // while the statistics MMAs run.  Only rows whose responsibility exceeds
+      // kTcDirRmin contribute: the few near the component.  (X, not F: F may
+      // already hold the next tile once the statistics MMAs are done.)  Each
+      // row's terms are rounded to the fixed-point unit kTcDirScale; a warp
+      // takes one component at a time, its lanes over 32 of the component's
+      // dimensions, sums the terms of its active rows as 64-bit integers and
+      // adds the sums to the shared fixed-point area with one coalesced
+      // atomic per word.  Integer sums do not depend on the order in which
+      // rows, warps and clusters add them.
       if (kStats && shl[0] > 0 && (FSRC != 2 || a.fg0 == 0)) {
         const int nsh = shl[0];
-        const XT* xrow = reinterpret_cast<const XT*>(a.X) + (size_t)(valid ? row0 + row : 0) * D;
-        const size_t kp = (size_t)a.Kpad;
         for (int si = 0; si < nsh; si++) {
           const int j = shl_j(shl[1 + si]), ns = shl_ns(shl[1 + si]), nd = shl_nd(shl[1 + si]);
           if ((j >> 6) != hf || nd == 0) continue;
@@ -1493,16 +1453,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const double r = !(valid && l > -INFINITY) ? 0.0
                            : kHard ? (k0 + j == win ? 1.0 : 0.0)
                                    : (double)__expf(l - lse);
-          if (r > (double)kTcDirRmin) {
-            const size_t base = (size_t)(k0 + j) * D;
-            unsigned long long* q = a.dirq + (k0 + j);
-            for (int i = 0; i < nd; i++) {
-              const int d = min((int)a.perm[base + i], D - 1);
-              const double p = (double)a.ph[base + i];  // 1/var of this dimension
-              const double u = ((double)load1<XT>(xrow, d) - (double)a.muh[base + i]) * sqrt(p);
-              const double ru = r * u * kTcDirScale;
-              fixed_add(q + (size_t)i * kp, q + (size_t)(D + i) * kp, ru);
-              fixed_add(q + (size_t)(2 * D + i) * kp, q + (size_t)(3 * D + i) * kp, ru * u);
+          const uint32_t active = __ballot_sync(0xffffffffu, r > (double)kTcDirRmin);
+          if (active == 0u) continue;
+          const size_t base = (size_t)(k0 + j) * D;
+          unsigned long long* q = a.dirq + (size_t)(k0 + j) * (4 * D);
+          for (int i0 = 0; i0 < nd; i0 += 32) {
+            const int i = i0 + lane;
+            const bool has = i < nd;
+            const int d = has ? min((int)a.perm[base + i], D - 1) : 0;
+            const double mu_i = has ? (double)a.muh[base + i] : 0.0;
+            const double isd = has ? sqrt((double)a.ph[base + i]) : 0.0;  // 1/sigma
+            long long sa = 0, sb = 0;
+            for (uint32_t m = active; m != 0u; m &= m - 1u) {
+              const int src = __ffs(m) - 1;
+              const double rs = __shfl_sync(0xffffffffu, r, src);
+              if (has) {
+                const XT* xs = reinterpret_cast<const XT*>(a.X) +
+                               (size_t)(row0 + 32 * qd + src) * D;  // a valid row: r > 0
+                const double u = ((double)load1<XT>(xs, d) - mu_i) * isd;
+                const double ru = rs * u * kTcDirScale;
+                sa += __double2ll_rn(ru);
+                sb += __double2ll_rn(ru * u);
+              }
+            }
+            if (has) {
+              atomicAdd(q + i, (unsigned long long)(sa >> 32));
+              atomicAdd(q + D + i, (unsigned long long)(sa & 0xffffffffll));
+              atomicAdd(q + 2 * D + i, (unsigned long long)(sb >> 32));
+              atomicAdd(q + 3 * D + i, (unsigned long long)(sb & 0xffffffffll));
             }
           }
         }
@@ -1591,49 +1569,54 @@ __global__ void __launch_bounds__(256) tc_center_kernel(int D, int K, const floa
 }
 
 inline size_t tc_prep_smem_bytes(int D, int Fpad) {
-  return (size_t)(4 * D + 2 * Fpad) * sizeof(double) + (size_t)D * sizeof(int);
+  return (size_t)(4 * D + 2 * Fpad) * sizeof(double);
 }
 
 // One block of 128 threads per (padded) component, looping over the dimensions.
 //
-// Direct-form split.  The expanded form's fp32 error grows with
+// Exact log-joints.  The expanded form's fp32 error grows with
 // kappa_k = sum_d (mu^_kd^2 + 1)/var^_kd.  When kappa_k exceeds kTcSharpKappa (a
 // component collapsed onto a few points in some dimensions), or kTcSmallKappa
-// for a component expecting fewer than kTcSmallPoints points, its dimensions
-// are ranked by their share kappa_kd and the leading ones -- just enough that
-// the rest sum below the threshold -- are taken out of the contraction: their
-// W entries are zero, and the kernel adds -1/2 sum (x - mu)^2/var over them in
-// data units on the CUDA cores ("split" dimensions, nsplit_k of them, first in
-// perm).  The tensor cores keep the rest.
+// for a component expecting fewer than kTcSmallPoints points, the contraction's
+// log-joint serves only to find the rows near the component: it is within
+// mg_k = 1 + 2^-14 kappa_k nats of the exact one (the accumulated fp32 error is
+// about 4e-8 kappa_k; the bound allows well over a hundred times that), and a
+// row whose contraction value lies more than 80 + mg_k nats below the row's
+// best lower bound has responsibility 0.  For the others the kernel computes
+// log pi_k - 1/2 sum_d [log(2 pi var_kd) + (x_d - mu_kd)^2/var_kd] in data units
+// on the CUDA cores (cx_k the constant part; mun, pn the tables).  nsplit_k > 0
+// marks these components: the count of leading dimensions (by kappa_kd) that
+// bring the rest below the threshold, which also take their moments in direct
+// form.
 //
-// W = [mu^/var^, -1/(2 var^)] over the remaining dimensions, scaled by a power
-// of two 2^-g_k so its largest entry lies in [2^13, 2^14), split into fp16
-// hi/lo rows of Fpad features (padding rows and features zero).
+// W = [mu^/var^, -1/(2 var^)] over all dimensions, scaled by a power of two
+// 2^-g_k so its largest entry lies in [2^13, 2^14), split into fp16 hi/lo rows
+// of Fpad features (padding rows and features zero).
 //
 // The expanded-form constant c_k = log pi_k - (1/2) sum_d log(2 pi var_kd)
-// - (1/2) sum_{d kept} mu^_kd^2 / var^_kd is corrected for the part of W that
+// - (1/2) sum_d mu^_kd^2 / var^_kd is corrected for the part of W that
 // the fp16 hi/lo split drops: the MMA sums F (W_hi + W_lo) 2^g, short of F W 2^g
 // by F dW 2^g with dW = W 2^-g - W_hi - W_lo, known exactly here.  For the
 // points the component explains F is near its expectation E[F] = [mu^,
 // mu^^2 + var^], so 2^g E[F] . dW is added to c_k: that removes the split's
 // systematic error on those points (what remains is (F - E[F]) . dW, of either
 // sign from point to point).  The accumulator starts from ci_k = kTcStartFrac
-// sum_{d kept} mu^^2/var^ (fp32, in 2^g units); the fp32 remainder
-// c_k - 2^g ci_k is added after the MMAs.
+// sum_d mu^^2/var^ (fp32, in 2^g units); the fp32 remainder c_k - 2^g ci_k is
+// added after the MMAs.
 //
-// Tables for the split dimensions, in perm order: mu^ and 1/var^ (the filter on
-// the tile's features) and mu and 1/var in data units (the exact sum).
+// Tables for the direct-form moments, in perm order: mu and 1/var in data units.
 __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     int64_t N, int D, int K, int Fpad, const float* __restrict__ w, const float* __restrict__ mu,
     const float* __restrict__ var, const float* __restrict__ m, const float* __restrict__ sc,
     __half* __restrict__ whi, __half* __restrict__ wlo, float* __restrict__ c_out,
     float* __restrict__ wsc_out, int* __restrict__ ndir_out, int* __restrict__ nsplit_out,
     float* __restrict__ muh, float* __restrict__ ph, int* __restrict__ precise_out,
-    float* __restrict__ ci_out, uint16_t* __restrict__ perm_out, float* __restrict__ mhp_out,
-    float* __restrict__ php_out, uint32_t* __restrict__ pmask_out, uint16_t* __restrict__ rank_out,
+    float* __restrict__ ci_out, float* __restrict__ cx_out, float* __restrict__ mg_out,
+    uint16_t* __restrict__ perm_out, float* __restrict__ mun_out, float* __restrict__ pn_out,
+    uint32_t* __restrict__ pmask_out, uint16_t* __restrict__ rank_out,
     unsigned long long* __restrict__ dirq, unsigned int* status) {
   // dynamic shared memory (tc_prep_smem_bytes): per dimension mu^, var^, kappa_kd and
-  // kappa sorted (doubles) and the rank (int); per feature W and E[F] (doubles)
+  // kappa sorted; per feature W and E[F] (doubles)
   extern __shared__ double prep_sm[];
   double* mh_s = prep_sm;
   double* vh_s = mh_s + D;
@@ -1641,14 +1624,13 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
   double* ksort = kd_s + D;
   double* wv = ksort + D;    // Fpad
   double* ef = wv + Fpad;    // Fpad: E[F] under the component
-  int* rank_s = reinterpret_cast<int*>(ef + Fpad);
   __shared__ double red[4][4];
   __shared__ int ns_s, nd_s;
   const int k = blockIdx.x;
   const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
   const float wk = k < K ? w[k] : 0.f;
   // the fused pass adds this component's split-dimension moments onto zero
-  for (int q = threadIdx.x; q < 4 * D; q += blockDim.x) dirq[(size_t)q * gridDim.x + k] = 0ull;
+  for (int q = threadIdx.x; q < 4 * D; q += blockDim.x) dirq[(size_t)k * (4 * D) + q] = 0ull;
   const bool live = k < K && wk > 0.f;
   auto block_sum = [&](double v) -> double {
     v = warp_sum(v);
@@ -1684,6 +1666,8 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     }
     mh_s[d] = mh;
     vh_s[d] = vh;
+    mun_out[(size_t)k * D + d] = k < K ? mu[(size_t)k * D + d] : 0.f;
+    pn_out[(size_t)k * D + d] = k < K ? (float)(1.0 / (double)var[(size_t)k * D + d]) : 0.f;
     kd_s[d] = kd >= 0.0 ? fmin(kd, 1e300) : 0.0;  // NaN -> 0: the ranks stay a permutation
   }
   const double S_log = block_sum(s_log);
@@ -1701,13 +1685,10 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
       const double o = kd_s[e2];
       r += (o > key || (o == key && e2 < d)) ? 1 : 0;
     }
-    rank_s[d] = r;
     ksort[r] = key;
     rank_out[(size_t)k * D + d] = (uint16_t)r;
     const size_t o = (size_t)k * D + r;
     perm_out[o] = (uint16_t)d;
-    mhp_out[o] = (float)mh_s[d];
-    php_out[o] = (float)(1.0 / vh_s[d]);
     muh[o] = k < K ? mu[(size_t)k * D + d] : 0.f;
     ph[o] = k < K ? (float)(1.0 / (double)var[(size_t)k * D + d]) : 0.f;
   }
@@ -1728,22 +1709,20 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
   __syncthreads();
   const int ns = ns_s;
 
-  // ---- pass 2: the contraction's features, without the split dimensions
+  // ---- pass 2: the contraction's features
   double s_q = 0.0, amax = 0.0;
   for (int f = threadIdx.x; f < Fpad; f += blockDim.x) {
     double v = 0.0, e = 0.0;
     if (k < K && f < 2 * D) {
       const int d = f < D ? f : f - D;
-      if (rank_s[d] >= ns) {
-        const double mh = mh_s[d], vh = vh_s[d];
-        if (f < D) {
-          v = mh / vh;
-          e = mh;
-          s_q += mh * mh / vh;
-        } else {
-          v = -0.5 / vh;
-          e = mh * mh + vh;
-        }
+      const double mh = mh_s[d], vh = vh_s[d];
+      if (f < D) {
+        v = mh / vh;
+        e = mh;
+        s_q += mh * mh / vh;
+      } else {
+        v = -0.5 / vh;
+        e = mh * mh + vh;
       }
     }
     wv[f] = v;
@@ -1785,6 +1764,8 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
     const float cstart = live ? (float)ldexp(kTcStartFrac * S_q, -g) : 0.f;
     ci_out[k] = cstart;
     c_out[k] = live ? (float)(cfull - ldexp((double)cstart, g)) : -INFINITY;
+    cx_out[k] = live ? (float)(lw - 0.5 * S_log) : -INFINITY;
+    mg_out[k] = ns > 0 ? (float)(1.0 + ldexp(Kap, -14)) : 0.f;
     wsc_out[k] = ldexpf(1.0f, g);
     ndir_out[k] = nd_s;
     nsplit_out[k] = ns;
@@ -1836,11 +1817,10 @@ __global__ void __launch_bounds__(256) tc_reduce_stats_kernel(
   if (d == 0) stats[k] = n;
   const int r = rank[(size_t)k * D + d];
   if (r < ndir[k]) {
-    const size_t kp = (size_t)Kpad;
     const double p = (double)ph[(size_t)k * D + r];  // 1/var, perm order
-    const double a1 = fixed_value(dirq[(size_t)r * kp + k], dirq[(size_t)(D + r) * kp + k]);
-    const double b1 =
-        fixed_value(dirq[(size_t)(2 * D + r) * kp + k], dirq[(size_t)(3 * D + r) * kp + k]);
+    const unsigned long long* q = dirq + (size_t)k * (4 * D);
+    const double a1 = fixed_value(q[r], q[D + r]);
+    const double b1 = fixed_value(q[2 * D + r], q[3 * D + r]);
     stats[K + (size_t)k * D + d] = a1 / kTcDirScale / sqrt(p);
     stats[K + KD + (size_t)k * D + d] = b1 / kTcDirScale / p;
     return;
