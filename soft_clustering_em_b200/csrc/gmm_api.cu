@@ -262,7 +262,7 @@ gmm_status tc_clusters(const TcLayout& T, int64_t ntiles, size_t smem, int* ncl_
 template <typename XT, int MODE, int FSRC>
 gmm_status tc_launch(const gmm_problem* p, const void* X, int64_t N, char* ws, const TcLayout& T,
                      int ncl, int accumulate, cudaStream_t st, int32_t* labels = nullptr,
-                     int ncand = 0, int fg0 = 0, int nfgc = 0) {
+                     int ncand = 0, int fg0 = 0, int nfgc = 0, int rmode = 0) {
   CUtensorMap mhi, mlo, fhi, flo;
   memset(&mhi, 0, sizeof(mhi));
   memset(&mlo, 0, sizeof(mlo));
@@ -329,6 +329,8 @@ gmm_status tc_launch(const gmm_problem* p, const void* X, int64_t N, char* ws, c
   args.fg0 = fg0;
   args.nfgc = nfgc > 0 ? nfgc : T.nfg;
   args.nfg = T.nfg;
+  args.rbuf = (uint8_t*)(ws + T.rbuf);
+  args.rmode = rmode;
   args.status = (unsigned int*)ws;
   args.drain_tiles = kTcDrainTiles;
   args.precise = (const int*)(ws + T.precise);
@@ -389,11 +391,13 @@ gmm_status tc_pass_chunked(const gmm_problem* p, const void* X, char* ws, const 
     if (T.G > 1 && (s = tc_launch<XT, PART, FS>(p, Xc, n, ws, T, ncl, 0, st)) != GMM_OK)
       return s;
     if (tc_mode_stats(MODE)) {
+      // several feature groups: the first pass stores r^, the others load it
       for (int fg = 0; fg < T.NFG; fg++) {
         const int fg0 = fg * T.nfg;
+        const int rmode = T.NFG == 1 ? 0 : fg == 0 ? 1 : 2;
         if ((s = tc_launch<XT, MODE, FS>(p, Xc, n, ws, T, ncl, !(i == 0 && fg == 0), st,
                                          labels ? labels + r0 : nullptr, 0, fg0,
-                                         std::min(T.nfg, T.nchunks - fg0))) != GMM_OK)
+                                         std::min(T.nfg, T.nchunks - fg0), rmode)) != GMM_OK)
           return s;
       }
     } else if (T.G > 1) {

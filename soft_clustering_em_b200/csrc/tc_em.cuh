@@ -91,6 +91,7 @@ constexpr int kTcMaxD = 128;      // the largest D with resident features
 constexpr int kTcMaxDStream = 1024;
 static_assert(kTcMaxDStream < 2048, "split and direct counts are packed in 11 bits");
 constexpr int kTcRoundChunks = 2;
+constexpr uint32_t kTcRBytes = 65536;  // r^ hi | lo of a 128-row tile, streamed layout
 constexpr int kTcGroupChunks = 5;
 constexpr int kTcMaxCluster = 16;
 constexpr int kTcThreads = 320;          // 8 compute warps + MMA warp + TMA warp
@@ -101,11 +102,15 @@ constexpr double kTcRhoPrecise = 64.0;  // mu^^2/var^ of a dimension above which
                                         // drain after every tile with mass
 constexpr uint32_t kTcChunkBytes = 128u * 128u;  // one [128 x 64] 16-bit operand chunk
 constexpr float kTcRScale = 32768.0f;            // r is stored as fp16(r * 2^15)
-// Split dimensions above this kappa_k: the expanded form's logit bias, about
-// 4e-8 kappa_k nats with the accumulator start value below, stays under the
-// 4e-3 nats the weight tolerance allows ...
-constexpr double kTcSharpKappa = 1e5;
-constexpr double kTcSmallKappa = 2.0e4;          // ... or above this one for a component
+// Exact log-joints above this kappa_k: below it the expanded form's logit
+// bias, about 4e-8 kappa_k nats with the accumulator start value below (for
+// D <= 128; it grows as D / 128 beyond, and so the thresholds shrink as
+// 128 / D), stays near 1e-3 nats: under the 4e-3 nats the weight tolerance
+// allows, and small enough that a component's variance, which a wrong
+// responsibility for a distant row shifts by that row's squared distance,
+// stays within its 1e-3 tolerance ...
+constexpr double kTcSharpKappa = 3e4;
+constexpr double kTcSmallKappa = 6.0e3;          // ... or above this one for a component
 constexpr double kTcSmallPoints = 50.0;          //     expecting fewer points than this
 // Dimensions whose kappa_kd = (mu^^2 + 1)/var^ exceeds this take their moments
 // in direct form (exact, fixed point) even when the contraction keeps them for
@@ -275,8 +280,8 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //          units of the W row scale
 //   wsc  : C*128 f32 power-of-two scale of each W row
 //   ndir : C*128 int32 how many of the component's leading dimensions (in perm
-//          order) take their moments in direct form; the first nsplit of
-//          them (nsplit: C*128 int32) also leave the contraction for the logits
+//          order) take their moments in direct form
+//   nsplit: C*128 int32, > 0 for a component with exact log-joints
 //   pmask: [C*128 x Fpad/32] u32 per feature of each component, 1 if it is
 //          drained after every tile with mass (see tc_prep_w_kernel)
 //   perm : [C*128 x D] u16 dimensions of each component by decreasing
@@ -302,13 +307,16 @@ __host__ __device__ inline TcSmem tc_smem_layout(int D, int C, int nchunks) {
 //   fhi, flo : [R x Fpad] fp16 features [x^, x^^2] (hi and lo parts) of one
 //              chunk of R rows, written by tc_convert_kernel, read by TMA
 //   part     : [R x G] float2 (max, sum-exp) of each row over each group
+//   rbuf     : streamed features with several statistics groups: [R/128 x G C]
+//              r^ images (kTcRBytes) of a chunk's tiles, written by the first
+//              group's pass and read by the others
 //   Top-m assignment, for chunks of Rt rows:
 //   cand     : [Rt x (G C 2) x kTcCand] float2 (log-joint, index) candidates
 //   rowst    : [Rt] float2 (max, sum-exp) of each row
 struct TcLayout {
   size_t m, isc, sc, c, ci, wsc, cx, mg, ndir, nsplit, precise, pmask, muh, ph, perm, rank, mun, pn,
       whi,
-      wlo, dirq, slots, fhi, flo, part, cand, rowst, total, slot_stride;
+      wlo, dirq, slots, fhi, flo, part, rbuf, cand, rowst, total, slot_stride;
   int C, G, nchunks, Kpad, Fpad, P;
   int nfg, NFG;  // feature chunks per statistics group, and groups (1 unless streamed)
   int64_t R;   // rows per chunk (G > 1, or streamed features)
@@ -360,6 +368,10 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   L.nfg = streamed ? kTcGroupChunks : L.nchunks;
   L.NFG = (L.nchunks + L.nfg - 1) / L.nfg;
   L.R = (L.G > 1 || streamed) ? tc_chunk_rows(L.Fpad) : 0;
+  if (streamed && L.NFG > 1) {  // the r^ images of a chunk (4 Kpad bytes a row) at most 256 MiB
+    const int64_t rr = (int64_t)(kTcChunkFBytesMax / (4u * (size_t)L.Kpad)) / kTcRows * kTcRows;
+    L.R = std::max<int64_t>(kTcRows, std::min<int64_t>(L.R, rr));
+  }
   size_t off = 256;
   L.m = off;
   off = align_up(off + (size_t)D * 4, 256);
@@ -414,6 +426,11 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
     L.part = off;
     off = align_up(off + (size_t)L.R * L.G * 8, 256);
   }
+  // streamed features with several statistics groups: the r^ image of every
+  // (tile, CTA) of a chunk, stored by the first group's pass
+  L.rbuf = off;
+  if (streamed && L.NFG > 1)
+    off = align_up(off + (size_t)(L.R / kTcRows) * (L.Kpad / kTcComps) * kTcRBytes, 256);
   // top-m candidates: at most 64 MiB, at most 2^18 rows (and R with groups)
   {
     const size_t per_row = (size_t)L.G * L.C * 2 * kTcCand * 8 + 8;
@@ -450,7 +467,7 @@ struct TcArgs {
   const float* ci;      // accumulator start values (W-row-scale units), C*128
   const float* wsc;     // W row scales, C*128
   const int* ndir;      // leading perm dimensions with direct-form moments, C*128
-  const int* nsplit;    // how many of those also leave the contraction, C*128
+  const int* nsplit;    // > 0: the component takes exact log-joints, C*128
   const float* muh;     // mu (data units) in perm order, C*128 x D
   const float* ph;      // 1/var (data units) in perm order, C*128 x D
   const uint16_t* perm;  // dimensions by decreasing (mu^^2 + 1)/var^, C*128 x D
@@ -471,6 +488,10 @@ struct TcArgs {
   int ncand;            // top-m: candidates kept per (CTA, column half), <= kTcCand
   int fg0, nfgc, nfg;   // streamed features: this pass's statistics group (first chunk,
                         // chunks) and the group size that lays out tensor memory
+  uint8_t* rbuf;        // streamed features with several statistics groups: the r^
+                        // image of every (tile, CTA) of the chunk, kTcRBytes each
+  int rmode;            // 0; 1: the first group's pass stores r^ to rbuf; 2: a later
+                        // group's pass loads it instead of repeating the E-step
   unsigned int* status;
   int drain_tiles;
   const int* precise;   // 1: some feature of the component is drained every tile, C*128
@@ -561,9 +582,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // logit buffers in tensor memory (columns [0, 128) and [128, 256), free of
   // statistics here), so the E-step of tile i+1 runs while the epilogue of
   // tile i reads the other buffer; the F buffer is released as soon as the
-  // E-step is done with it (after the epilogue when split dimensions' filter
-  // reads it too).
+  // E-step is done with it.
   constexpr bool kOverlap = !kStats && FSRC;
+  // Streamed features with several statistics groups: the first group's pass
+  // stores each tile's r^ image, the later groups' passes load it instead of
+  // repeating the E-step and its epilogue.
+  const bool rstore = kStats && FSRC == 2 && a.rmode == 1;
+  const bool rload = kStats && FSRC == 2 && a.rmode == 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -600,6 +625,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* f_tx = f_full + 13;    // [2] FSRC = 1: an F buffer's TMA loads have landed
   uint64_t* f_full2 = f_full + 15;  // [2] overlap: start values in logit buffer b stored
   uint64_t* l_full2 = f_full + 17;  // [2] overlap: E-step into logit buffer b done
+  uint64_t* r_tx = f_full + 19;     // rmode 2: a tile's r^ loaded from rbuf
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tslot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -630,6 +656,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&f_full2[b], kTcComputeThreads);
       mbar_init(&l_full2[b], 1);
     }
+    mbar_init(r_tx, 1);
     mbar_init(l_full, 1);
     mbar_init(r_full, kTcComputeThreads / 2);
     mbar_init(r_full1, kTcComputeThreads / 2);
@@ -661,10 +688,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     int n = 0;
     uint32_t mw[4] = {0u, 0u, 0u, 0u};
-    // every component with direct-form moments (shl_pack: local index, split
-    // count, direct count); the mask marks those with split dimensions
+    // every component with exact log-joints or direct-form moments (shl_pack:
+    // local index, split count, direct count); the mask marks the former
     for (int j = 0; j < kTcComps; j++)
-      if (a.ndir[k0 + j] > 0) {
+      if (a.ndir[k0 + j] > 0 || a.nsplit[k0 + j] > 0) {
         const int ns = a.nsplit[k0 + j];
         shl[1 + n++] = shl_pack(j, ns, a.ndir[k0 + j]);
         if (ns > 0) mw[j >> 5] |= 1u << (j & 31);
@@ -705,7 +732,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tma_prefetch_desc(&tm_flo);
       }
       uint32_t stage = 0, phase = 0;
-      int64_t issued = 0, fissued = 0;
+      int64_t issued = 0, fissued = 0, rissued = 0;
       for (int64_t li = 0; li < my_tiles; li++) {
         bool ok = true;
         // FSRC = 1: this tile's features into F buffer b, once the tile that
@@ -745,6 +772,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           fissued++;
           return true;
         };
+        if (rload) {
+          // the tile's r^ image, once the previous tile's statistics MMAs are
+          // done with the buffer, then the statistics group's feature rounds
+          if (li > 0 && !mbar_wait_bounded(s_done, (uint32_t)((li - 1) & 1), status, kAbort,
+                                           a.wait_ns))
+            break;
+          const uint8_t* src =
+              a.rbuf + ((size_t)(((int64_t)cid + li * ncl) * ngrp + grp) * C + rank) * kTcRBytes;
+          mbar_arrive_expect_tx(r_tx, kTcRBytes);
+          for (uint32_t q = 0; q < kTcRBytes; q += 16384u)
+            bulk_load(sR + q, src + q, 16384u, r_tx);
+          rissued++;
+          for (int c = a.fg0; c < a.fg0 + a.nfgc && ok; c += (int)L.nr)
+            ok = load_round(c, min((int)L.nr, a.fg0 + a.nfgc - c));
+          if (!ok) break;
+          continue;
+        }
         int wi = 0;  // W loads issued for this tile
         for (int c = 0; c < nch && ok; c++)
           for (int part = 0; part < 2 && ok; part++, wi++) {
@@ -780,6 +824,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int64_t uses = (fissued - b + L.nfb - 1) / L.nfb;  // feature loads into buffer b
         mbar_wait_bounded(&f_tx[b], (uint32_t)((uses - 1) & 1), status, 0u, a.drain_ns);
       }
+      if (rissued > 0) mbar_wait_bounded(r_tx, (uint32_t)((rissued - 1) & 1), status, 0u, a.drain_ns);
     }
   } else if (warp == kTcMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -797,9 +842,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint64_t dOnes = sw128_desc(ob, 16, 1024);
       uint32_t stage = 0, phase = 0, ndrain = 0;
       int64_t fu = 0;  // FSRC = 2: uses of the F buffer so far (rounds)
-      const bool has_split = (shl[kTcComps + 1] | shl[kTcComps + 2] | shl[kTcComps + 3] |
-                              shl[kTcComps + 4]) != 0;
+      // FSRC = 2: the statistics MMAs of tile li over this pass's feature
+      // group, a round of chunks at a time, once the previous tile's drain is done
+      auto stats_streamed = [&](int64_t li) -> bool {
+        if (li > 0) {
+          if (!mbar_wait_bounded(drained, ndrain & 1u, status, kAbort, a.wait_ns)) return false;
+          ndrain++;
+        }
+        tc_fence_after_sync();
+        const bool first = li == 0;
+        for (int c0 = a.fg0; c0 < a.fg0 + a.nfgc; c0 += (int)L.nr) {
+          const int n = min((int)L.nr, a.fg0 + a.nfgc - c0);
+          if (!mbar_wait_bounded(&f_tx[0], (uint32_t)(fu & 1), status, kAbort, a.wait_ns))
+            return false;
+          tc_fence_after_sync();
+          const uint32_t idSr = idesc_f16_f32(128, 64 * n, true, true);
+          const uint32_t tSr = tS + 64u * (uint32_t)(c0 - a.fg0);
+#pragma unroll 1
+          for (int k8 = 0; k8 < 8; k8++) {  // 16-row K-steps over the 128 rows
+            const uint32_t hofs = 32768u * (uint32_t)(k8 >> 2);
+            const uint64_t ahi = desc_add(dR, hofs + 2048u * (k8 & 3));
+            const uint64_t alo = desc_add(dR, hofs + 16384u + 2048u * (k8 & 3));
+            const bool acc = !(first && k8 == 0);
+            const uint32_t kr = 2048u * (uint32_t)k8;  // F rows of this K-step
+            const uint64_t fhi = desc_add(dFs, kr);
+            const uint64_t flo = desc_add(dFs, L.nr * kTcChunkBytes + kr);
+            mma_bf16(tSr, ahi, fhi, idSr, acc);
+            mma_bf16(tSr, ahi, flo, idSr, true);
+            mma_bf16(tSr, alo, fhi, idSr, true);
+            if (c0 == a.fg0) {
+              mma_bf16(tNK, ahi, dOnes, idN, acc);
+              mma_bf16(tNK, alo, dOnes, idN, true);
+            }
+          }
+          mma_commit(&f_free[0]);
+          fu++;
+        }
+        return true;
+      };
       for (int64_t li = 0; li < my_tiles; li++) {
+        if (rload) {
+          // r^ from the first group's pass: the statistics MMAs only
+          if (!mbar_wait_bounded(r_tx, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) break;
+          if (!stats_streamed(li)) break;
+          mma_commit(s_done);
+          continue;
+        }
         const uint32_t lb = kOverlap ? (uint32_t)(li & 1) : 0u;  // logit buffer
         const uint32_t tLb = tL + 128u * lb;
         if (kOverlap) {
@@ -853,15 +941,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!ok) break;
         if (kOverlap) {
           mma_commit(&l_full2[lb]);
-          // the F buffer is free once the E-step is done with it -- or, where
-          // split dimensions' filter reads it, once both row halves' epilogues are
-          if (FSRC == 1) {
-            if (has_split &&
-                !(mbar_wait_bounded(r_full, (uint32_t)(li & 1), status, kAbort, a.wait_ns) &&
-                  mbar_wait_bounded(r_full1, (uint32_t)(li & 1), status, kAbort, a.wait_ns)))
-              break;
-            mma_commit(&f_free[li % L.nfb]);
-          }
+          // the F buffer is free once the E-step is done with it (the epilogue
+          // reads X, not F)
+          if (FSRC == 1) mma_commit(&f_free[li % L.nfb]);
           continue;
         }
         mma_commit(l_full);
@@ -873,39 +955,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (kStats && FSRC == 2) {
           // both 64-row halves of r^ are written (the buffer holds all 128 rows)
           if (!mbar_wait_bounded(r_full1, (uint32_t)(li & 1), status, kAbort, a.wait_ns)) break;
-          if (li > 0) {
-            if (!mbar_wait_bounded(drained, ndrain & 1u, status, kAbort, a.wait_ns)) break;
-            ndrain++;
-          }
           tc_fence_after_sync();
-          const bool first = li == 0;
-          for (int c0 = a.fg0; c0 < a.fg0 + a.nfgc && ok2; c0 += (int)L.nr) {
-            const int n = min((int)L.nr, a.fg0 + a.nfgc - c0);
-            ok2 = mbar_wait_bounded(&f_tx[0], (uint32_t)(fu & 1), status, kAbort, a.wait_ns);
-            if (!ok2) break;
-            tc_fence_after_sync();
-            const uint32_t idSr = idesc_f16_f32(128, 64 * n, true, true);
-            const uint32_t tSr = tS + 64u * (uint32_t)(c0 - a.fg0);
-#pragma unroll 1
-            for (int k8 = 0; k8 < 8; k8++) {  // 16-row K-steps over the 128 rows
-              const uint32_t hofs = 32768u * (uint32_t)(k8 >> 2);
-              const uint64_t ahi = desc_add(dR, hofs + 2048u * (k8 & 3));
-              const uint64_t alo = desc_add(dR, hofs + 16384u + 2048u * (k8 & 3));
-              const bool acc = !(first && k8 == 0);
-              const uint32_t kr = 2048u * (uint32_t)k8;  // F rows of this K-step
-              const uint64_t fhi = desc_add(dFs, kr);
-              const uint64_t flo = desc_add(dFs, L.nr * kTcChunkBytes + kr);
-              mma_bf16(tSr, ahi, fhi, idSr, acc);
-              mma_bf16(tSr, ahi, flo, idSr, true);
-              mma_bf16(tSr, alo, fhi, idSr, true);
-              if (c0 == a.fg0) {
-                mma_bf16(tNK, ahi, dOnes, idN, acc);
-                mma_bf16(tNK, alo, dOnes, idN, true);
-              }
-            }
-            mma_commit(&f_free[0]);
-            fu++;
+          if (rstore) {
+            // the tile's r^ image for the later statistics groups' passes
+            uint8_t* dst =
+                a.rbuf + ((size_t)(((int64_t)cid + li * ncl) * ngrp + grp) * C + rank) * kTcRBytes;
+            for (uint32_t q = 0; q < kTcRBytes; q += 16384u) bulk_store(dst + q, sR + q, 16384u);
+            bulk_commit();
           }
+          ok2 = stats_streamed(li);
+          if (rstore) bulk_wait_read();  // before s_done lets the next tile overwrite r^
         } else if (kStats) {
           const bool first = li == 0;  // later tiles add onto whatever the drains left
           if (li > 0) {
@@ -944,6 +1003,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (FSRC == 1) mma_commit(&f_free[li % L.nfb]);
         SCEM_TRACE(li, 11);
       }
+      if (rstore) bulk_wait_all();  // the r^ images are in global memory
       // every MMA issued must be complete before tensor memory is released
       mma_commit(final_bar);
       mbar_wait_bounded(final_bar, 0, status, 0u, a.drain_ns);
@@ -1068,6 +1128,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_after_sync();
         return r;
       };
+      if (rload) {
+        // r^ comes from the first group's pass: the previous tile's drain only
+        if (li > 0) {
+          ok = wait_prev_stats();
+          if (ok) ok = drain((li % a.drain_tiles) == 0, li);
+          if (!ok) break;
+          tc_fence_before_sync();
+          mbar_arrive(drained);
+        }
+        continue;
+      }
       if (!FSRC && li > 0 && L.nfb == 1) {
         ok = wait_prev_stats();
         if (!ok) break;
@@ -1216,9 +1287,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // first pass (final = false): every column is an accumulator value,
       // scaled to a log-joint; the max is a lower bound of the half's best
       // log-joint (columns in the mask, components with exact log-joints,
-      // count less their error bound mg).  Second pass (final = true): the
-      // masked columns already hold exact log-joints (or -inf).
-      auto load_logits = [&](bool final, uint32_t m0, uint32_t m1) {
+      // count less their error bound mg).  Second pass (final = true): a
+      // masked column holds the exact log-joint where the row is near the
+      // component (bit set in nb) and is -inf elsewhere.
+      auto load_logits = [&](bool final, uint32_t m0, uint32_t m1, uint64_t nb) {
         mx = -INFINITY;
 #pragma unroll
         for (int q = 0; q < 2; q++) {
@@ -1229,14 +1301,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int j = 0; j < 32; j++) {
             const int cidx = col0 + 32 * q + j;
             const bool masked = (mq >> j) & 1u;
-            e[32 * q + j] = (final && masked) ? v[j] : fmaf(v[j], wscs[cidx], csm[cidx]);
+            const bool nr = (nb >> (32 * q + j)) & 1ull;
+            e[32 * q + j] = (final && masked) ? (nr ? v[j] : -INFINITY)
+                                              : fmaf(v[j], wscs[cidx], csm[cidx]);
             mx = fmaxf(mx, (final || !masked) ? e[32 * q + j] : e[32 * q + j] - mgs[cidx]);
           }
         }
       };
       const uint32_t sm0 = (uint32_t)shl[kTcComps + 1 + 2 * hf],
                      sm1 = (uint32_t)shl[kTcComps + 2 + 2 * hf];
-      load_logits(false, sm0, sm1);
+      load_logits(false, sm0, sm1, 0ull);
+      uint64_t nearb = 0;  // masked columns of this half that the row is near
       if (sm0 | sm1) {
         // Components of this column half with exact log-joints.  A row whose
         // contraction value, plus its error bound, falls 80 nats below the
@@ -1245,16 +1320,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // from X, one row at a time, its lanes over the dimensions, the
         // per-lane sums added in a fixed butterfly order.
         const float floor_l = mx - 80.f;
-        const int nsh = shl[0];
         const bool rvalid = row0 + row < a.N;
+#pragma unroll
+        for (int j = 0; j < 64; j++) {
+          const bool masked = ((j < 32 ? sm0 : sm1) >> (j & 31)) & 1u;
+          if (masked && rvalid && e[j] > -INFINITY && e[j] + mgs[col0 + j] >= floor_l)
+            nearb |= 1ull << j;
+        }
+        const int nsh = shl[0];
         const XT* xw = reinterpret_cast<const XT*>(a.X) + (size_t)(row0 + 32 * qd) * D;
         for (int si = 0; si < nsh; si++) {
           const int j = shl_j(shl[1 + si]), ns = shl_ns(shl[1 + si]);
           if ((j >> 6) != hf || ns == 0) continue;
-          const float v0 = tmem_ld1(tLc + lane_base + (uint32_t)j);
-          const float la = fmaf(v0, wscs[j], csm[j]);  // the contraction's log-joint
-          const bool near = rvalid && la > -INFINITY && la + mgs[j] >= floor_l;
-          uint32_t nm = __ballot_sync(0xffffffffu, near);
+          uint32_t nm = __ballot_sync(0xffffffffu, (nearb >> (j & 63)) & 1ull);
+          if (nm == 0u) continue;  // no row of the warp: the column is not read again
           const float* muk = a.mun + (size_t)(k0 + j) * D;
           const float* pk = a.pn + (size_t)(k0 + j) * D;
           float lx = -INFINITY;
@@ -1281,10 +1360,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (lane == s0) lx = cxs[j] - 0.5f * q0;
             if (lane == s1) lx = cxs[j] - 0.5f * q1;
           }
-          // the exact log-joint (the second load_logits takes it as is)
+          // the exact log-joint (the second load_logits takes it where the row is near)
           tmem_st1(tLc + lane_base + (uint32_t)j, lx);
         }
-        load_logits(true, sm0, sm1);
+        load_logits(true, sm0, sm1, nearb);
       }
       if (t == 0) SCEM_TRACE(li, 5);
       float se = 0.f;
@@ -1446,10 +1525,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // skipped only when no row of the warp needs it: the tensor-memory
           // load below is a warp-collective (.sync.aligned) instruction
           if (!__any_sync(0xffffffffu, (rbits >> (j & 63)) & 1ull)) continue;
-          // the log-joint: finished in tensor memory for a component with split
-          // dimensions, the raw accumulator (scaled as the epilogue scales it) otherwise
+          // the log-joint: exact in tensor memory for a component with exact
+          // log-joints where the row is near it (-inf elsewhere), the raw
+          // accumulator (scaled as the epilogue scales it) otherwise
           const float v0 = tmem_ld1(tLc + lane_base + (uint32_t)j);
-          const float l = ns > 0 ? v0 : fmaf(v0, wscs[j], csm[j]);
+          const float l = ns == 0 ? fmaf(v0, wscs[j], csm[j])
+                          : ((nearb >> (j & 63)) & 1ull) ? v0 : -INFINITY;
           const double r = !(valid && l > -INFINITY) ? 0.0
                            : kHard ? (k0 + j == win ? 1.0 : 0.0)
                                    : (double)__expf(l - lse);
@@ -1585,9 +1666,9 @@ inline size_t tc_prep_smem_bytes(int D, int Fpad) {
 // best lower bound has responsibility 0.  For the others the kernel computes
 // log pi_k - 1/2 sum_d [log(2 pi var_kd) + (x_d - mu_kd)^2/var_kd] in data units
 // on the CUDA cores (cx_k the constant part; mun, pn the tables).  nsplit_k > 0
-// marks these components: the count of leading dimensions (by kappa_kd) that
-// bring the rest below the threshold, which also take their moments in direct
-// form.
+// marks these components (the count of leading dimensions, by kappa_kd, that
+// bring the rest below the threshold).  Independently, the leading ndir_k
+// dimensions with kappa_kd > kTcDirectKappa take their moments in direct form.
 //
 // W = [mu^/var^, -1/(2 var^)] over all dimensions, scaled by a power of two
 // 2^-g_k so its largest entry lies in [2^13, 2^14), split into fp16 hi/lo rows
@@ -1674,7 +1755,9 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
   const double Kap = block_sum(kap);
   const double Rho = block_max(rho);
   const bool small = (double)wk * (double)N < kTcSmallPoints;
-  const double thr = small ? kTcSmallKappa : kTcSharpKappa;
+  // the fp32 error grows with the number of accumulation steps, 2D / 16 per
+  // operand pair: the thresholds hold for D <= 128 and scale as 128 / D beyond
+  const double thr = (small ? kTcSmallKappa : kTcSharpKappa) * fmin(1.0, 128.0 / (double)D);
   const bool sharp = live && Kap > thr;
 
   // ---- dimensions by decreasing kappa_kd (ties to the lower index)
@@ -1700,8 +1783,8 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
       while (ns < D && rem > thr) rem -= ksort[ns++];
     }
     ns_s = ns;
-    // and the further leading dimensions whose moments are taken in direct form
-    int nd = ns;
+    // the leading dimensions whose moments are taken in direct form
+    int nd = 0;
     if (live)
       while (nd < D && ksort[nd] > kTcDirectKappa) nd++;
     nd_s = nd;
@@ -1733,12 +1816,15 @@ __global__ void __launch_bounds__(128) tc_prep_w_kernel(
   const double Amax = block_max(amax);
   // Precise features: both features of a dimension with mu^^2/var^ > kTcRhoPrecise
   // (the variance S2/N - (S1/N)^2 magnifies their fp32 rounding by that ratio),
-  // every feature of a component expecting fewer than kTcSmallPoints points.
+  // every feature of a component expecting fewer than kTcSmallPoints points --
+  // except the dimensions whose moments are taken in direct form (the first
+  // nd in perm order), whose tensor-core sums are not used.
   for (int f = threadIdx.x; f < Fpad; f += blockDim.x) {  // warp w: features 32w.. of each 128
     bool pf = false;
     if (live && f < 2 * D) {
       const int d = f < D ? f : f - D;
-      pf = small || mh_s[d] * mh_s[d] / vh_s[d] > kTcRhoPrecise;
+      pf = (small || mh_s[d] * mh_s[d] / vh_s[d] > kTcRhoPrecise) &&
+           (int)rank_out[(size_t)k * D + d] >= nd_s;
     }
     const uint32_t word = __ballot_sync(0xffffffffu, pf);
     if (lane == 0) pmask_out[(size_t)k * (Fpad / 32) + f / 32] = word;

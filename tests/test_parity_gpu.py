@@ -80,6 +80,7 @@ CASES = [
     ("gauss8", 10_007, 8, 3),
     ("uint8img", 20_011, 256, 3),
     ("sphere768", 3_001, 1024, 2),
+    ("sphere768", 50_000, 1024, 1),  # D = 768 streamed: 5 statistics groups, two row chunks
     ("gauss4096", 20_000, 4096, 2),  # two passes over 4 component groups of 8-CTA clusters
     ("gauss4096", 300_007, 1536, 1),  # two groups of 6 CTAs; two row chunks (2^18 + ragged)
     ("gauss4096", 20_000, 512, 2),  # D = 96 on the tensor cores: 3 feature chunks, 4-CTA clusters
@@ -485,10 +486,12 @@ def test_split_dimensions_match_oracle(G):
     np.testing.assert_allclose(got[2][0][:4], 1e-6, rtol=1e-6)
 
 
-@pytest.mark.parametrize("D,K", [(48, 200), (96, 300)])
+@pytest.mark.parametrize("D,K", [(48, 200), (96, 300), (260, 200), (1024, 130)])
 def test_padded_and_odd_feature_chunks(G, D, K):
-    """2D not a multiple of 64 (D = 48: two chunks, the second half padding) and an odd
-    chunk count (D = 96: three chunks), with ragged K and N."""
+    """2D not a multiple of 64 (D = 48: two chunks, the second half padding), an odd
+    chunk count (D = 96: three chunks), and streamed features (D = 260: nine chunks in
+    statistics groups of five and four; D = 1024, the largest: 32 chunks in seven
+    groups), with ragged K and N."""
     rng = np.random.default_rng(D)
     N = 5_003
     centers = rng.uniform(-6, 6, size=(K, D))
