@@ -1314,12 +1314,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint64_t nearb = 0;  // masked columns of this half that the row is near
       if (sm0 | sm1) {
         // Components of this column half with exact log-joints.  A row whose
-        // contraction value, plus its error bound, falls 80 nats below the
-        // half's lower bound has responsibility 0 and gets -inf; for the rows
-        // near the component the warp computes the log-joint in direct form
-        // from X, one row at a time, its lanes over the dimensions, the
-        // per-lane sums added in a fixed butterfly order.
-        const float floor_l = mx - 80.f;
+        // contraction value, plus its error bound, falls 32 nats below a lower
+        // bound of its best log-joint (this half's, or with component groups
+        // the exact row max from the partial pass) has responsibility below
+        // e^-32: its r^ (fp16 of r 2^15) is 0 and it takes no direct-form
+        // moments (kTcDirRmin), so it gets -inf.  For the rows near the
+        // component the warp computes the log-joint in direct form from X,
+        // one row at a time, its lanes over the dimensions, the per-lane sums
+        // added in a fixed butterfly order.
+        const float floor_l = fmaxf(mx, M) - 32.f;
         const bool rvalid = row0 + row < a.N;
 #pragma unroll
         for (int j = 0; j < 64; j++) {
