@@ -461,9 +461,7 @@ def ours(args):
                       f"{plan['chunk_rows']} rows tc_convert_kernel (features to HBM), the "
                       "partial (max, sum-exp) pass and the statistics pass, features TMA-loaded")
     else:
-        dtype = "f32"
-        precision = "fp32 direct form on the CUDA cores, fp64 reductions and M-step"
-        kernel = "simt_fused_kernel (CUDA cores, direct form; the shape has no tensor-core plan)"
+        raise SystemExit(f"{wl.name}: no tensor-core plan for this shape")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

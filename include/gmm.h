@@ -91,8 +91,10 @@ typedef struct {
 
 /* How the library runs a problem on the current device (see gmm_plan). */
 typedef struct {
-  int32_t tensor_cores; /* 1: the tcgen05 tensor-core kernel; 0: the CUDA-core kernel
-                           (D > 128, D not a multiple of 4, or no cluster shape fits) */
+  int32_t tensor_cores; /* 1: the tcgen05 tensor-core kernel runs the problem; 0: no
+                           tensor-core plan (D > 1024, D not a multiple of 4, or no
+                           cluster shape fits), and the EM calls return
+                           GMM_ERR_UNSUPPORTED */
   int32_t cluster_ctas; /* tensor cores: CTAs per thread-block cluster, 128 components each */
   int32_t groups;       /* tensor cores: component groups.  1: one fused pass, the row
                            normalisation exchanged inside the cluster.  > 1: per chunk of
@@ -151,6 +153,8 @@ gmm_status gmm_init_rows(const gmm_problem* p, const void* X, const int64_t* row
  * loglik (device, 1 double, may be NULL) receives LL of the INPUT parameters,
  * sum_n log p(x_n), including the -D/2 log(2 pi) term.
  * The N x K responsibilities exist only on chip (review page, sections 2-3).
+ * Runs on the tensor cores; a shape without a tensor-core plan (gmm_plan)
+ * returns GMM_ERR_UNSUPPORTED before any launch.
  */
 gmm_status gmm_em_step(const gmm_problem* p, const void* X, float* w, float* mu, float* var,
                        double* loglik, void* ws, size_t ws_bytes, void* stream);
@@ -198,12 +202,10 @@ gmm_status gmm_mstep(const gmm_problem* p, const double* stats, int32_t nshards,
  * before any stream capture.  When the statistics slots of the regular
  * workspace do not all fit, fewer CTAs (or clusters) run the fused pass, one
  * slot each, which is slower but gives the same result up to summation order.
- * A tensor-core slot holds K*(2D+1)+1 doubles beside the parameter tables;
- * when not even one fits (and for shapes whose tensor-core plan has more than
- * one component group, whose row-chunk buffers exceed the scratch), the call
- * runs the CUDA-core kernel, whose slot holds K*(2D+1)+1.  A problem for which
- * not even that fits is rejected with GMM_ERR_UNSUPPORTED and a message on
- * stderr.
+ * A tensor-core slot holds K*(2D+1)+1 doubles beside the parameter tables.
+ * A problem for which not even one fits, or whose plan's row-chunk buffers
+ * (several component groups, or D > 128) exceed the scratch, is rejected with
+ * GMM_ERR_UNSUPPORTED and a message on stderr.
  *
  * Every call on a device uses the same array and it keeps the previous call's
  * contents; each call resets the status word and rewrites everything else it

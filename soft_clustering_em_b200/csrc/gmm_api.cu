@@ -15,7 +15,7 @@
 #include "common.cuh"
 #include "gmm.h"
 #include "ivf.cuh"
-#include "simt_em.cuh"
+#include "mstep_init.cuh"
 #include "small_fit.cuh"
 #include "tc_em.cuh"
 #include "tma_host.h"
@@ -57,12 +57,12 @@ gmm_status device_sms(int* sms) {
   return GMM_OK;
 }
 
-// Which kernels a problem runs and where their data sits in the workspace.
-// The CUDA-core layout always exists (top-m and init use it); the tensor-core
-// layout exists when the shape fits that kernel.  Both start at offset 256,
-// after the shared status word, and the workspace covers the larger one.
+// Where a problem's data sits in the workspace.  The init scratch always
+// exists; the tensor-core layout exists when the shape has a tensor-core plan
+// (every EM call needs one).  Both start at offset 256, after the shared
+// status word, and the workspace covers the larger one.
 struct Plan {
-  WsLayout simt;
+  InitLayout init;
   TcLayout tc;
   bool use_tc;
   size_t stats;  // canonical statistics buffer: K(2D+1)+1 doubles
@@ -76,13 +76,13 @@ Plan make_plan(const gmm_problem* p, int sms, size_t cap) {
   Plan P;
   const size_t sbytes = align_up(stats_doubles(p) * 8, 256);
   const size_t c = cap ? (cap > sbytes ? cap - sbytes : 1) : 0;
-  P.simt = c ? ws_layout_capped(p->D, p->K, sms, c) : ws_layout(p->D, p->K, sms);
+  P.init = init_layout(p->D, p->K, sms);
   P.use_tc = tc_shape_ok(p->D, p->K, sms);
   if (P.use_tc) {
     P.tc = tc_layout(p->D, p->K, sms, c);
     if (P.tc.P < 1) P.use_tc = false;
   }
-  size_t body = P.simt.P >= 1 ? P.simt.total : 0;
+  size_t body = P.init.total;
   if (P.use_tc) body = std::max(body, P.tc.total);
   P.stats = align_up(body, 256);
   P.aux = P.stats + sbytes;
@@ -152,37 +152,6 @@ void ivf_walk(int m, bool fill, int64_t N, int K, const int32_t* idx, const floa
     case 7: return ivf_walk_m<7>(fill, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
     default: return ivf_walk_m<8>(fill, N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
   }
-}
-
-template <typename XT, int MODE>
-gmm_status launch_simt(const gmm_problem* p, const void* X, const WsPtrs& w, int m, int32_t* idx,
-                       float* resp, cudaStream_t st) {
-  const size_t smem = simt_smem_bytes(p->D);
-  auto kern = simt_fused_kernel<XT, MODE>;
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return GMM_ERR_UNSUPPORTED;
-    }
-  }
-  trace_begin(st);
-  kern<<<w.P, kSimtThreads, smem, st>>>((const XT*)X, p->N, p->D, p->K, w, m, idx, resp);
-  trace_end(st);
-  return launched(1);
-}
-
-template <int MODE>
-gmm_status fused_pass(const gmm_problem* p, const void* X, const WsPtrs& w, int m, int32_t* idx,
-                      float* resp, cudaStream_t st) {
-  if (p->xdtype == GMM_BF16) return launch_simt<__nv_bfloat16, MODE>(p, X, w, m, idx, resp, st);
-  return launch_simt<float, MODE>(p, X, w, m, idx, resp, st);
-}
-
-gmm_status prep(const gmm_problem* p, const float* w, const float* mu, const float* var,
-                const WsPtrs& ws, cudaStream_t st) {
-  prep_kernel<<<p->K, 128, 0, st>>>(p->D, p->K, w, mu, var, ws);
-  return launched(1);
 }
 
 // ---------------------------------------------------------------------------
@@ -455,8 +424,8 @@ gmm_status estep_stats_impl(const gmm_problem* p, const void* X, const float* w,
   gmm_status s;
   const size_t KD = (size_t)p->K * p->D;
   const unsigned blocks = (unsigned)((KD + 255) / 256);
-  if (hard && !P.use_tc) return GMM_ERR_UNSUPPORTED;
-  if (P.use_tc) {
+  if (!P.use_tc) return GMM_ERR_UNSUPPORTED;  // no tensor-core plan for this shape
+  {
     const TcLayout& T = P.tc;
     gmm_problem pp = *p;
     pp.N = n_prep;
@@ -472,11 +441,6 @@ gmm_status estep_stats_impl(const gmm_problem* p, const void* X, const float* w,
         nslots, T.G, T.C * kTcComps, stats);
     return launched(1);
   }
-  const WsPtrs wp = ws_ptrs(ws_base, P.simt);
-  if ((s = prep(p, w, mu, var, wp, st)) != GMM_OK) return s;
-  if ((s = fused_pass<kModeStats>(p, X, wp, 0, nullptr, nullptr, st)) != GMM_OK) return s;
-  simt_reduce_stats_kernel<<<blocks, 256, 0, st>>>(p->D, p->K, wp, stats);
-  return launched(1);
 }
 
 // One chunk of the top-m pass over pre-converted features (FS = 1 or 2).
@@ -797,10 +761,12 @@ gmm_status gmm_init_rows(const gmm_problem* p, const void* X, const int64_t* row
     if (rows_host[k] < 0 || rows_host[k] >= p->N) return GMM_ERR_INVALID_ARG;
   Plan P;
   if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
-  WsPtrs wp = ws_ptrs(ws, P.simt);
+  int64_t* rows = (int64_t*)((char*)ws + P.init.rows);
+  double* part = (double*)((char*)ws + P.init.part);
+  const int nparts = P.init.P;
   cudaStream_t st = (cudaStream_t)stream;
   // the K row indices travel to the workspace (the one host->device copy of this call)
-  if (cudaMemcpyAsync(wp.scratch, rows_host, sizeof(int64_t) * p->K, cudaMemcpyHostToDevice, st) !=
+  if (cudaMemcpyAsync(rows, rows_host, sizeof(int64_t) * p->K, cudaMemcpyHostToDevice, st) !=
       cudaSuccess) {
     launch_status();
     return GMM_ERR_CUDA;
@@ -808,22 +774,22 @@ gmm_status gmm_init_rows(const gmm_problem* p, const void* X, const int64_t* row
   const bool bf = p->xdtype == GMM_BF16;
   if (bf)
     init_gather_kernel<__nv_bfloat16><<<p->K, 128, 0, st>>>((const __nv_bfloat16*)X, p->D, p->K,
-                                                           wp.scratch, init_var, w, mu, var);
+                                                           rows, init_var, w, mu, var);
   else
-    init_gather_kernel<float><<<p->K, 128, 0, st>>>((const float*)X, p->D, p->K, wp.scratch,
-                                                    init_var, w, mu, var);
+    init_gather_kernel<float><<<p->K, 128, 0, st>>>((const float*)X, p->D, p->K, rows, init_var,
+                                                    w, mu, var);
   if ((s = launched(1)) != GMM_OK) return s;
   if (init_var == GMM_INIT_VAR_DATA) {
-    double* part = wp.slots;
-    double* mean = part + (size_t)wp.P * p->D;
+    double* mean = part + (size_t)nparts * p->D;
     for (int pass = 0; pass < 2; pass++) {
       const double* mptr = pass == 0 ? nullptr : mean;
       if (bf)
-        col_partial_kernel<__nv_bfloat16><<<wp.P, 256, 0, st>>>((const __nv_bfloat16*)X, p->N,
-                                                                p->D, mptr, part);
+        col_partial_kernel<__nv_bfloat16><<<nparts, 256, 0, st>>>((const __nv_bfloat16*)X, p->N,
+                                                                  p->D, mptr, part);
       else
-        col_partial_kernel<float><<<wp.P, 256, 0, st>>>((const float*)X, p->N, p->D, mptr, part);
-      col_finish_kernel<<<(p->D + 127) / 128, 128, 0, st>>>(p->N, p->D, p->K, wp.P, part, pass,
+        col_partial_kernel<float><<<nparts, 256, 0, st>>>((const float*)X, p->N, p->D, mptr,
+                                                          part);
+      col_finish_kernel<<<(p->D + 127) / 128, 128, 0, st>>>(p->N, p->D, p->K, nparts, part, pass,
                                                             p->var_floor, mean, var);
       if ((s = launched(2)) != GMM_OK) return s;
     }
@@ -900,11 +866,11 @@ gmm_status gmm_em_step_noalloc(const gmm_problem* p, const void* X, float* w, fl
   int sms = 0;
   if ((s = device_sms(&sms)) != GMM_OK) return s;
   const Plan P = make_plan(p, sms, kNoallocScratchBytes);
-  if (!P.use_tc && P.simt.P < 1) {
+  if (!P.use_tc || P.aux > kNoallocScratchBytes) {  // (the step uses no region past stats)
     fprintf(stderr,
-            "gmm_em_step_noalloc: K=%d, D=%d needs %zu bytes of scratch for one statistics "
-            "slot; the built-in scratch holds %zu bytes\n",
-            p->K, p->D, P.simt.slots + P.simt.slot_stride * 8, kNoallocScratchBytes);
+            "gmm_em_step_noalloc: K=%d, D=%d has no tensor-core plan whose one statistics "
+            "slot fits the built-in scratch of %zu bytes\n",
+            p->K, p->D, kNoallocScratchBytes);
     return GMM_ERR_UNSUPPORTED;
   }
   void* ws = nullptr;
@@ -1016,8 +982,9 @@ gmm_status gmm_loglik(const gmm_problem* p, const void* X, const float* w, const
   if (!w || !mu || !var || !loglik) return GMM_ERR_INVALID_ARG;
   Plan P;
   if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  if (!P.use_tc) return GMM_ERR_UNSUPPORTED;  // no tensor-core plan for this shape
   cudaStream_t st = (cudaStream_t)stream;
-  if (P.use_tc) {
+  {
     char* wsb = (char*)ws;
     const TcLayout& T = P.tc;
     if ((s = tc_prep(p, w, mu, var, wsb, T, st)) != GMM_OK) return s;
@@ -1028,11 +995,6 @@ gmm_status gmm_loglik(const gmm_problem* p, const void* X, const float* w, const
                                              T.slot_stride, nslots, loglik);
     return launched(1);
   }
-  const WsPtrs wp = ws_ptrs(ws, P.simt);
-  if ((s = prep(p, w, mu, var, wp, st)) != GMM_OK) return s;
-  if ((s = fused_pass<kModeLoglik>(p, X, wp, 0, nullptr, nullptr, st)) != GMM_OK) return s;
-  reduce_loglik_kernel<<<1, 1, 0, st>>>(p->D, p->K, wp, loglik);
-  return launched(1);
 }
 
 gmm_status gmm_assign_topm(const gmm_problem* p, const void* X, const float* w, const float* mu,
@@ -1045,15 +1007,11 @@ gmm_status gmm_assign_topm(const gmm_problem* p, const void* X, const float* w, 
   if (m < 1 || m > kMaxTopM || m > p->K) return GMM_ERR_INVALID_ARG;
   Plan P;
   if ((s = get_plan(p, ws, ws_bytes, &P)) != GMM_OK) return s;
+  if (!P.use_tc) return GMM_ERR_UNSUPPORTED;  // no tensor-core plan for this shape
   cudaStream_t st = (cudaStream_t)stream;
-  if (P.use_tc) {
-    if (p->xdtype == GMM_BF16)
-      return tc_topm_t<__nv_bfloat16>(p, X, w, mu, var, m, idx, resp, (char*)ws, P, st);
-    return tc_topm_t<float>(p, X, w, mu, var, m, idx, resp, (char*)ws, P, st);
-  }
-  const WsPtrs wp = ws_ptrs(ws, P.simt);
-  if ((s = prep(p, w, mu, var, wp, st)) != GMM_OK) return s;
-  return fused_pass<kModeTopm>(p, X, wp, m, idx, resp, st);
+  if (p->xdtype == GMM_BF16)
+    return tc_topm_t<__nv_bfloat16>(p, X, w, mu, var, m, idx, resp, (char*)ws, P, st);
+  return tc_topm_t<float>(p, X, w, mu, var, m, idx, resp, (char*)ws, P, st);
 }
 
 gmm_status gmm_ivf_workspace_size(int64_t N, int32_t K, size_t* bytes) {

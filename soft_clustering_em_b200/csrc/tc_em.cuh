@@ -212,8 +212,8 @@ __host__ __device__ inline bool tc_streamed(int nchunks) { return nchunks > kTcM
 // features can be written while the previous tile's statistics MMAs still
 // read the other buffer.
 struct TcSmem {
-  uint32_t F, W, R, ONES, msm, iscs, csm, cis, wscs, cxs, mgs, shl, precs, xchg, bars, tslot,
-      total;
+  uint32_t F, W, R, ONES, msm, iscs, csm, cis, wscs, cxs, mgs, shl, shs, ndc, precs, xchg, bars,
+      tslot, total;
   uint32_t nfb, fbytes;
   uint32_t nr;  // feature chunks an F buffer holds: all of them, or a round when streamed
 };
@@ -253,6 +253,10 @@ __host__ __device__ inline TcSmem tc_smem_layout_n(int D, int C, int nchunks, ui
   off += kTcComps * 4;
   L.shl = off;
   off += (kTcComps + 8) * 4;
+  L.shs = off;  // per column half: the count, then the local columns with exact log-joints
+  off += 2 * (kTcComps / 2 + 1) * 4;
+  L.ndc = off;  // per local component its direct dimensions, then 4 words: those with any
+  off += (kTcComps + 4) * 4;
   L.precs = off;
   off += kTcComps * 4;
   L.xchg = off;
@@ -606,6 +610,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* cxs = reinterpret_cast<float*>(sm + L.cxs);
   float* mgs = reinterpret_cast<float*>(sm + L.mgs);
   int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = shl_pack entries
+  int* shs = reinterpret_cast<int*>(sm + L.shs);  // [half][0] = count, [half][1..] = columns
+  int* ndc = reinterpret_cast<int*>(sm + L.ndc);  // [128] direct dimensions, [128..131] mask
   int* precs = reinterpret_cast<int*>(sm + L.precs);
   float2* xchg = reinterpret_cast<float2*>(sm + L.xchg);  // [2][C][2][128] (max, sum-exp)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L.bars);
@@ -626,6 +632,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* f_full2 = f_full + 15;  // [2] overlap: start values in logit buffer b stored
   uint64_t* l_full2 = f_full + 17;  // [2] overlap: E-step into logit buffer b done
   uint64_t* r_tx = f_full + 19;     // rmode 2: a tile's r^ loaded from rbuf
+
   uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + L.tslot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -657,6 +664,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&l_full2[b], 1);
     }
     mbar_init(r_tx, 1);
+
     mbar_init(l_full, 1);
     mbar_init(r_full, kTcComputeThreads / 2);
     mbar_init(r_full1, kTcComputeThreads / 2);
@@ -699,6 +707,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     shl[0] = n;
     // after the list (entries 1..128): bit j of word q is local component 32q + j
     for (int q = 0; q < 4; q++) shl[kTcComps + 1 + q] = (int)mw[q];
+    // per column half, the columns with exact log-joints
+    for (int h = 0; h < 2; h++) {
+      int c = 0;
+      for (int j = 64 * h; j < 64 * h + 64; j++)
+        if ((mw[j >> 5] >> (j & 31)) & 1u) shs[h * (kTcComps / 2 + 1) + 1 + c++] = j;
+      shs[h * (kTcComps / 2 + 1)] = c;
+    }
+    // per local component its direct dimensions, and which have any
+    uint32_t dw[4] = {0u, 0u, 0u, 0u};
+    for (int j = 0; j < kTcComps; j++) {
+      ndc[j] = a.ndir[k0 + j];
+      if (ndc[j] > 0) dw[j >> 5] |= 1u << (j & 31);
+    }
+    for (int q = 0; q < 4; q++) ndc[kTcComps + q] = (int)dw[q];
   }
   for (int i = tid; i < 2048; i += kTcThreads)
     reinterpret_cast<__half*>(sOnes)[i] = __float2half_rn(1.0f);
@@ -1285,11 +1307,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float e[64];
       float mx = -INFINITY;
       // first pass (final = false): every column is an accumulator value,
-      // scaled to a log-joint; the max is a lower bound of the half's best
-      // log-joint (columns in the mask, components with exact log-joints,
-      // count less their error bound mg).  Second pass (final = true): a
-      // masked column holds the exact log-joint where the row is near the
-      // component (bit set in nb) and is -inf elsewhere.
+      // scaled to a log-joint; a masked column (a component with exact
+      // log-joints) holds that value plus its error bound mg, an upper bound,
+      // and counts at the value less mg in the max, a lower bound of the
+      // half's best log-joint.  Second pass (final = true): a masked column
+      // holds the exact log-joint where the row is near the component (bit
+      // set in nb) and is -inf elsewhere.
       auto load_logits = [&](bool final, uint32_t m0, uint32_t m1, uint64_t nb) {
         mx = -INFINITY;
 #pragma unroll
@@ -1302,15 +1325,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int cidx = col0 + 32 * q + j;
             const bool masked = (mq >> j) & 1u;
             const bool nr = (nb >> (32 * q + j)) & 1ull;
-            e[32 * q + j] = (final && masked) ? (nr ? v[j] : -INFINITY)
-                                              : fmaf(v[j], wscs[cidx], csm[cidx]);
-            mx = fmaxf(mx, (final || !masked) ? e[32 * q + j] : e[32 * q + j] - mgs[cidx]);
+            if (final) {
+              e[32 * q + j] = masked ? (nr ? v[j] : -INFINITY) : fmaf(v[j], wscs[cidx], csm[cidx]);
+              mx = fmaxf(mx, e[32 * q + j]);
+            } else {
+              const float l = fmaf(v[j], wscs[cidx], csm[cidx]);
+              const float mg = masked ? mgs[cidx] : 0.f;
+              e[32 * q + j] = l + mg;
+              mx = fmaxf(mx, l - mg);
+            }
           }
         }
       };
       const uint32_t sm0 = (uint32_t)shl[kTcComps + 1 + 2 * hf],
                      sm1 = (uint32_t)shl[kTcComps + 2 + 2 * hf];
       load_logits(false, sm0, sm1, 0ull);
+      // a lower bound of the row's best log-joint: this half's or, with
+      // component groups, the exact row max from the partial pass
+      const float mlb = fmaxf(mx, M);
       uint64_t nearb = 0;  // masked columns of this half that the row is near
       if (sm0 | sm1) {
         // Components of this column half with exact log-joints.  A row whose
@@ -1322,19 +1354,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // component the warp computes the log-joint in direct form from X,
         // one row at a time, its lanes over the dimensions, the per-lane sums
         // added in a fixed butterfly order.
-        const float floor_l = fmaxf(mx, M) - 32.f;
+        const float floor_l = mlb - 32.f;
         const bool rvalid = row0 + row < a.N;
+        if (rvalid) {
+          const uint64_t msk = (uint64_t)sm0 | ((uint64_t)sm1 << 32);
 #pragma unroll
-        for (int j = 0; j < 64; j++) {
-          const bool masked = ((j < 32 ? sm0 : sm1) >> (j & 31)) & 1u;
-          if (masked && rvalid && e[j] > -INFINITY && e[j] + mgs[col0 + j] >= floor_l)
-            nearb |= 1ull << j;
+          for (int j = 0; j < 64; j++)
+            if (e[j] > -INFINITY && e[j] >= floor_l) nearb |= 1ull << j;  // e: the upper bound
+          nearb &= msk;
         }
-        const int nsh = shl[0];
+        const int* hs = shs + hf * (kTcComps / 2 + 1);
+        const int nhs = hs[0];
         const XT* xw = reinterpret_cast<const XT*>(a.X) + (size_t)(row0 + 32 * qd) * D;
-        for (int si = 0; si < nsh; si++) {
-          const int j = shl_j(shl[1 + si]), ns = shl_ns(shl[1 + si]);
-          if ((j >> 6) != hf || ns == 0) continue;
+        for (int si = 0; si < nhs; si++) {
+          const int j = hs[1 + si];
           uint32_t nm = __ballot_sync(0xffffffffu, (nearb >> (j & 63)) & 1ull);
           if (nm == 0u) continue;  // no row of the warp: the column is not read again
           const float* muk = a.mun + (size_t)(k0 + j) * D;
@@ -1521,19 +1554,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // atomic per word.  Integer sums do not depend on the order in which
       // rows, warps and clusters add them.
       if (kStats && shl[0] > 0 && (FSRC != 2 || a.fg0 == 0)) {
-        const int nsh = shl[0];
-        for (int si = 0; si < nsh; si++) {
-          const int j = shl_j(shl[1 + si]), ns = shl_ns(shl[1 + si]), nd = shl_nd(shl[1 + si]);
-          if ((j >> 6) != hf || nd == 0) continue;
-          // skipped only when no row of the warp needs it: the tensor-memory
-          // load below is a warp-collective (.sync.aligned) instruction
-          if (!__any_sync(0xffffffffu, (rbits >> (j & 63)) & 1ull)) continue;
+        // the components of this half with direct dimensions that some row
+        // of the warp needs (a warp-uniform set: the tensor-memory load below
+        // is a warp-collective .sync.aligned instruction)
+        const uint64_t exact = (uint64_t)sm0 | ((uint64_t)sm1 << 32);
+        const uint64_t direct =
+            (uint64_t)(uint32_t)ndc[kTcComps + 2 * hf] |
+            ((uint64_t)(uint32_t)ndc[kTcComps + 2 * hf + 1] << 32);
+        const uint64_t need =
+            (((uint64_t)__reduce_or_sync(0xffffffffu, (uint32_t)(rbits >> 32)) << 32) |
+             (uint64_t)__reduce_or_sync(0xffffffffu, (uint32_t)rbits)) & direct;
+        for (uint64_t todo = need; todo != 0ull; todo &= todo - 1ull) {
+          const int jj = __ffsll((long long)todo) - 1, j = col0 + jj;
+          const int nd = ndc[j];
           // the log-joint: exact in tensor memory for a component with exact
           // log-joints where the row is near it (-inf elsewhere), the raw
           // accumulator (scaled as the epilogue scales it) otherwise
           const float v0 = tmem_ld1(tLc + lane_base + (uint32_t)j);
-          const float l = ns == 0 ? fmaf(v0, wscs[j], csm[j])
-                          : ((nearb >> (j & 63)) & 1ull) ? v0 : -INFINITY;
+          const float l = !((exact >> jj) & 1ull) ? fmaf(v0, wscs[j], csm[j])
+                          : ((nearb >> jj) & 1ull) ? v0 : -INFINITY;
           const double r = !(valid && l > -INFINITY) ? 0.0
                            : kHard ? (k0 + j == win ? 1.0 : 0.0)
                                    : (double)__expf(l - lse);

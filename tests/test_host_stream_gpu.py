@@ -50,7 +50,7 @@ def _setup(G, name, N, K):
     ("gauss8", 1_001, 8, 7),             # 143 chunks of 7 rows
     ("gauss8", 1_000, 8, 1_000),         # exactly one chunk
     ("gauss8", 999, 8, 5_000),           # chunk larger than N
-    ("sphere768", 2_003, 1024, 500),     # the CUDA-core kernel
+    ("sphere768", 2_003, 1024, 500),     # D = 768: streamed features, 5 statistics groups
     ("gauss4096", 20_000, 4096, 6_000),  # component groups: two passes per host chunk
 ])
 def test_host_streamed_step_matches_oracle(G, name, N, K, chunk):

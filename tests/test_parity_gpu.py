@@ -466,9 +466,9 @@ def test_split_dimensions_deterministic(G):
 def test_split_dimensions_match_oracle(G):
     """A component collapsed onto rows that share exact values in some dimensions
     (variance at the floor there: kappa far above 1e7), and a tight component
-    expecting 20 points (kappa between 2e4 and 1e7): both have dimensions summed in
-    direct form on the CUDA cores next to the tensor-core contraction of the rest,
-    and the split dimensions' moments summed in direct form too.  (The tight
+    expecting 20 points (kappa between 6e3 and 1e7): both take exact log-joints in
+    direct form for the rows near them, and the moments of their dimensions with
+    kappa_kd > 500 in direct form too.  (The tight
     component sits 0.1 from the centring point in x^ units: far from it, mu^^2/var^ of
     its kept dimensions would bound its variance's precision at about that ratio times
     2^-22; right at it, x^^2 of its points would fall below fp16's normal range -- the
