@@ -67,6 +67,9 @@ def parse():
     ap.add_argument("--host-stream", action="store_true",
                     help="time EM with X in pinned host memory (gmm_em_step_host)")
     ap.add_argument("--chunk-rows", type=int, default=1 << 17)
+    ap.add_argument("--all", action="store_true",
+                    help="one GPU: run every workload in turn (a process each), one JSON line "
+                         "per workload")
     return ap.parse_args()
 
 
@@ -651,8 +654,29 @@ def host_stream_bench(args):
     print(json.dumps(line), flush=True)
 
 
+def all_workloads(args):
+    """One line per workload, each from its own process (bench.py --workload W)."""
+    rc = 0
+    for name in sorted(synth.WORKLOADS):
+        cmd = [sys.executable, os.path.abspath(__file__), "--workload", name,
+               "--steps", str(args.steps), "--warmup", str(args.warmup)]
+        if args.no_cpu_baseline:
+            cmd.append("--no-cpu-baseline")
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+        if r.returncode != 0 or not lines:
+            rc = r.returncode or 1
+            print(json.dumps({"workload": name, "error": (r.stderr.strip().splitlines() or
+                                                          ["no output"])[-1]}), flush=True)
+        else:
+            print(lines[-1], flush=True)
+    return rc
+
+
 def main():
     args = parse()
+    if args.all:
+        raise SystemExit(all_workloads(args))
     if args.impl == "reference":
         reference_arm(args)
         return
