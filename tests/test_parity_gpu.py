@@ -178,6 +178,33 @@ def test_ragged_k_and_dead_component(G):
     assert compare.compare_step(ref[:4], got, ref[4])["ok"]
 
 
+def test_shapes_without_a_tensor_core_plan_are_rejected(G):
+    """One backend: a shape the tensor-core kernel has no plan for is refused before any
+    launch (D beyond 1024 at the argument check; K beyond what component groups of
+    2-CTA clusters hold at D = 128), not run elsewhere."""
+    import torch
+
+    assert G.gmm_plan(G.problem(1000, 128, 16384))["tensor_cores"] == 1
+    p = G.problem(1000, 128, 20000)
+    assert G.gmm_plan(p)["tensor_cores"] == 0
+    X = torch.zeros(1000, 128, device="cuda")
+    K = 20000
+    w = torch.full((K,), 1.0 / K, device="cuda")
+    mu = torch.zeros(K, 128, device="cuda")
+    var = torch.ones(K, 128, device="cuda")
+    ll = torch.zeros(1, dtype=torch.float64, device="cuda")
+    for call in (lambda: G.gmm_em_step(X, w, mu, var, ll),
+                 lambda: G.gmm_loglik(X, w, mu, var)):
+        with pytest.raises(G.GmmError) as e:
+            call()
+        assert e.value.status == G.GMM_ERR_UNSUPPORTED
+    Xw = torch.zeros(100, 1028, device="cuda")
+    with pytest.raises(G.GmmError) as e:
+        G.gmm_em_step(Xw, w[:4] * 0 + 0.25, torch.zeros(4, 1028, device="cuda"),
+                      torch.ones(4, 1028, device="cuda"), ll)
+    assert e.value.status == G.GMM_ERR_UNSUPPORTED
+
+
 def test_workspace_does_not_depend_on_n(G):
     for D, K, dt in ((128, 256, 0), (96, 4096, 0), (32, 1024, 1), (768, 1024, 0)):
         sizes = {G.gmm_workspace_size(G.problem(N, D, K, dt)) for N in (10_000, 10**6, 10**8)}
