@@ -75,7 +75,8 @@ size_t stats_doubles(const gmm_problem* p) { return (size_t)p->K * (2 * (size_t)
 Plan make_plan(const gmm_problem* p, int sms, size_t cap) {
   Plan P;
   const size_t sbytes = align_up(stats_doubles(p) * 8, 256);
-  const size_t c = cap ? (cap > sbytes ? cap - sbytes : 1) : 0;
+  // (less 256 bytes: the regions below start on 256-byte boundaries)
+  const size_t c = cap ? (cap > sbytes + 256 ? cap - sbytes - 256 : 1) : 0;
   P.init = init_layout(p->D, p->K, sms);
   P.use_tc = tc_shape_ok(p->D, p->K, sms);
   if (P.use_tc) {

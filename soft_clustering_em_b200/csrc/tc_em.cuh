@@ -435,12 +435,14 @@ inline TcLayout tc_layout(int D, int K, int num_sms, size_t cap = 0) {
   L.rbuf = off;
   if (streamed && L.NFG > 1)
     off = align_up(off + (size_t)(L.R / kTcRows) * (L.Kpad / kTcComps) * kTcRBytes, 256);
-  // top-m candidates: at most 64 MiB, at most 2^18 rows (and R with groups)
+  // top-m candidates: at most 64 MiB, at most 2^18 rows (and R with groups);
+  // one tile's worth under a byte cap (the no-allocation step runs no top-m)
   {
     const size_t per_row = (size_t)L.G * L.C * 2 * kTcCand * 8 + 8;
     int64_t rt = (int64_t)((size_t)(64u << 20) / per_row) / kTcRows * kTcRows;
     rt = std::max<int64_t>(kTcRows, std::min<int64_t>(rt, kTcChunkRowsMax));
     if (L.R > 0) rt = std::min<int64_t>(rt, L.R);
+    if (cap) rt = kTcRows;
     L.Rt = rt;
     L.cand = off;
     off = align_up(off + (size_t)rt * (per_row - 8), 256);
