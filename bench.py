@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--ivf", action="store_true",
                     help="time the IVF list build (gmm_ivf_build) instead of the EM step")
     ap.add_argument("--ivf-tau", type=float, default=0.1)
+    ap.add_argument("--topm", action="store_true",
+                    help="time the top-2 assignment (gmm_assign_topm) instead of the EM step")
     ap.add_argument("--host-stream", action="store_true",
                     help="time EM with X in pinned host memory (gmm_em_step_host)")
     ap.add_argument("--chunk-rows", type=int, default=1 << 17)
@@ -583,6 +585,68 @@ def ivf_bench(args):
     print(json.dumps(line), flush=True)
 
 
+def topm_bench(args):
+    """One GPU: the top-m assignment (m = 2) of a workload's rows after a short fit.
+
+    A step is one gmm_assign_topm: the E-step on the tensor cores (the groups'
+    partial pass first where K spans several clusters), each (CTA, column half)'s
+    best candidates, then the direct-form refinement of each row's candidates.
+    The parameters come from the seeded init and 3 EM steps.  Algorithmic work:
+    the E-step's 4*N*K*D flop.
+    """
+    import torch
+
+    from soft_clustering_em_b200 import gmm as G
+
+    wl = synth.WORKLOADS[args.workload]
+    N = args.rows or wl.N
+    dev = torch.device("cuda", 0)
+    X_np, _ = synth.make_data(wl, N)
+    Xd = torch.from_numpy(X_np.view(np.int16) if wl.dtype == "bf16" else X_np)
+    if wl.dtype == "bf16":
+        Xd = Xd.view(torch.bfloat16)
+    Xd = Xd.to(dev)
+    mode = G.GMM_INIT_VAR_ONE if wl.var_init == "one" else G.GMM_INIT_VAR_DATA
+    p = G.problem_for(Xd, wl.K, wl.var_floor)
+    ws = G.workspace(p, dev)
+    w, mu, var = G.gmm_init(Xd, wl.init_seed, wl.K, mode, wl.var_floor, ws=ws)
+    ll = torch.zeros(1, dtype=torch.float64, device=dev)
+    for _ in range(3):
+        G.gmm_em_step(Xd, w, mu, var, ll, wl.var_floor, ws=ws)
+    m = 2
+    stream = torch.cuda.current_stream(dev)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else None)
+    for _ in range(max(3, args.warmup)):
+        G.gmm_assign_topm(Xd, w, mu, var, m, wl.var_floor, ws=ws)
+    torch.cuda.synchronize(dev)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = G.gmm_launch_count()
+    start.record(stream)
+    for _ in range(args.steps):
+        G.gmm_assign_topm(Xd, w, mu, var, m, wl.var_floor, ws=ws)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = G.gmm_launch_count() - launches0
+    clocks = sampler.stop()
+    ms = start.elapsed_time(stop) / args.steps
+    rc, flags = G.gmm_device_status(ws)
+    pk, kind = peaks()
+    achieved = 4.0 * N * wl.K * wl.D / (ms * 1e-3) / 1e12
+    line = {
+        "metric": "top-2 assignment, points/s on 1 B200", "value": N / (ms * 1e-3),
+        "unit": "points/s", "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16", "data": "synthetic",
+        "config": dict(workload_config(wl, N), m=m, params="seeded init + 3 EM steps"),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                     "algorithmic": "4*N*K*D flop (the E-step)", "peak_kind": kind},
+        "gpu_launches": launches, "device_status": rc, "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def host_stream_bench(args):
     """One GPU: EM iterations with X in pinned host memory, streamed in chunks.
 
@@ -685,6 +749,9 @@ def main():
         return
     if args.host_stream:
         host_stream_bench(args)
+        return
+    if args.topm:
+        topm_bench(args)
         return
     ours(args)
 
