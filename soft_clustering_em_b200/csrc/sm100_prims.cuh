@@ -72,10 +72,24 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
                : "memory");
 }
 
-// Arrive on the mbarrier at shared::cluster address `addr` (possibly another CTA's).
+// Arrive on the mbarrier at shared::cluster address `addr` (possibly another
+// CTA's), releasing the thread's earlier writes at cluster scope.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
                : "memory");
+}
+
+// Arrive, without ordering of its own, on the mbarrier at shared::cluster
+// address `addr` (possibly another CTA's): after one fence_acq_rel_cluster, a
+// thread's arrives on several CTAs' barriers release its earlier writes once,
+// instead of one release fence per arrive.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel_cluster() {
+  asm volatile("fence.acq_rel.cluster;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
