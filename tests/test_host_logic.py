@@ -201,3 +201,24 @@ def test_tensor_core_shape_limits_and_f_buffers(tmp_path):
             assert (nfb256, nfb1024, nfbmax) == (2, 1, 1), D
         else:
             assert nfb256 == 1 and nfbmax == 1 and nfb1024 == (1 if D <= 96 else 0), D
+    # streamed features (D > 128): every case has a plan that fits 227 KB of shared
+    # memory, statistics groups of five chunks, chunk buffers within 256 MiB, and
+    # r^ images only where there is more than one statistics group
+    out = subprocess.run([exe, "streamed"], check=True, capture_output=True, text=True).stdout
+    for ln in out.strip().split("\n"):
+        D, K, C, G, nch, nfg, NFG, R, smem, fhi, rbuf = map(int, ln.split())
+        assert C > 0 and G > 0, (D, K)
+        assert nch == (2 * D + 63) // 64 and nfg == 5 and NFG == (nch + 4) // 5, (D, K)
+        assert smem <= 232448, (D, K, smem)
+        assert R >= 128 and R % 128 == 0, (D, K, R)
+        assert 2 * fhi <= (256 << 20) + 512, (D, K, fhi)  # hi and lo feature planes
+        if NFG == 1:
+            assert rbuf == 0, (D, K)
+        else:
+            assert (R // 128) * G * C * 65536 <= rbuf <= (256 << 20) + 256, (D, K, rbuf)
+    # the largest K with a tensor-core plan: 37 groups of 4-CTA clusters (one cluster
+    # per group at least on 148 SMs), or 64 groups of 2 at D = 100..128
+    out = subprocess.run([exe, "maxk"], check=True, capture_output=True, text=True).stdout
+    for ln in out.strip().split("\n"):
+        D, maxk = map(int, ln.split())
+        assert maxk == (16384 if 100 <= D <= 128 else 18944), (D, maxk)
