@@ -127,17 +127,34 @@ gmm_status launched(int n) {
 }
 
 // One walk of gmm_ivf_build over all chunks, for m candidates per point.
+template <int kM, bool kFill, bool kShared>
+void ivf_walk_launch(int64_t N, int K, const int32_t* idx, const float* resp, float tau,
+                     const IvfLayout& L, int64_t* cnt, const int64_t* offsets, int64_t* ids,
+                     unsigned int* status, cudaStream_t st) {
+  const int ctas = (L.B + kIvfWarps - 1) / kIvfWarps;
+  const size_t smem = kShared ? (size_t)K * kIvfWarps * 4 : 0;
+  auto kern = ivf_walk_kernel<kM, kFill, kShared>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess)
+    return;  // the launch below fails and the caller's launch check reports it
+  kern<<<ctas, kIvfWarps * 32, smem, st>>>(N, K, idx, resp, tau, L.B, L.R, cnt, offsets, ids,
+                                           status);
+}
+
 template <int kM>
 void ivf_walk_m(bool fill, int64_t N, int K, const int32_t* idx, const float* resp, float tau,
                 const IvfLayout& L, int64_t* cnt, const int64_t* offsets, int64_t* ids,
                 unsigned int* status, cudaStream_t st) {
-  const int ctas = (L.B + kIvfWarps - 1) / kIvfWarps;
-  if (fill)
-    ivf_walk_kernel<kM, true><<<ctas, kIvfWarps * 32, 0, st>>>(N, K, idx, resp, tau, L.B, L.R,
-                                                               cnt, offsets, ids, status);
+  const bool sh = ivf_shared_counters(K, L.R, kM);
+  if (fill && sh)
+    ivf_walk_launch<kM, true, true>(N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+  else if (fill)
+    ivf_walk_launch<kM, true, false>(N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
+  else if (sh)
+    ivf_walk_launch<kM, false, true>(N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
   else
-    ivf_walk_kernel<kM, false><<<ctas, kIvfWarps * 32, 0, st>>>(N, K, idx, resp, tau, L.B, L.R,
-                                                                cnt, offsets, ids, status);
+    ivf_walk_launch<kM, false, false>(N, K, idx, resp, tau, L, cnt, offsets, ids, status, st);
 }
 
 void ivf_walk(int m, bool fill, int64_t N, int K, const int32_t* idx, const float* resp,

@@ -27,7 +27,8 @@
 // point's m components are distinct, so each list takes at most one entry per
 // point); the lane holding a list's last entry in the group advances that
 // list's counter.  One warp owns each counter column, so the counters need no
-// global atomics and the order is fixed.
+// global atomics and the order is fixed.  Where K is small the running counts
+// live in the warp's shared memory and reach cnt once per chunk.
 #pragma once
 #include <algorithm>
 
@@ -83,7 +84,14 @@ constexpr int ivf_table_log2(int m) { return m <= 1 ? 6 : m <= 2 ? 7 : m <= 4 ? 
 // lanes holding that list; the entry's rank is the count of mask bits below
 // its lane.  The masks do not depend on the order of the atomics, so neither
 // does the result.
-template <int kM, bool kFill>
+//
+// kShared (K small enough, see ivf_shared_counters): each warp keeps its
+// chunk's running count of every list in shared memory (int32, from 0) instead
+// of in cnt, so no global load and store sits on the per-group chain.  The
+// count pass writes the final counts to cnt once at the end; the fill pass
+// reads each entry's chunk prefix from cnt (read-only there) and adds the
+// shared count.
+template <int kM, bool kFill, bool kShared>
 __global__ void __launch_bounds__(kIvfWarps * 32, kM <= 4 ? 4 : 2)
     ivf_walk_kernel(int64_t N, int K, const int32_t* __restrict__ idx,
                     const float* __restrict__ resp, float tau, int B, int64_t R, int64_t* cnt,
@@ -93,6 +101,7 @@ __global__ void __launch_bounds__(kIvfWarps * 32, kM <= 4 ? 4 : 2)
   constexpr int kT = 1 << kLog;
   __shared__ int s_key[kIvfWarps][kT];
   __shared__ unsigned int s_lanes[kIvfWarps][kT];
+  extern __shared__ int ivf_counts[];  // kShared: [kIvfWarps][K]
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int c = blockIdx.x * kIvfWarps + w;
   if (c >= B) return;  // c is the same for the whole warp; the tables are per warp
@@ -102,6 +111,9 @@ __global__ void __launch_bounds__(kIvfWarps * 32, kM <= 4 ? 4 : 2)
     key[i] = -1;
     lanes[i] = 0u;
   }
+  int* scnt = ivf_counts + (size_t)w * K;
+  if (kShared)
+    for (int k = lane; k < K; k += 32) scnt[k] = 0;
   __syncwarp();
   const unsigned int below = (1u << lane) - 1u;
   const unsigned int above = ~below & ~(1u << lane);
@@ -162,22 +174,38 @@ __global__ void __launch_bounds__(kIvfWarps * 32, kM <= 4 ? 4 : 2)
       const unsigned int mask = e[j] >= 0 ? lanes[slot[j]] : 0u;
       before[j] = __popc(mask & below);
       last[j] = (mask & above) == 0u;
-      base[j] = e[j] >= 0 ? cnt[(int64_t)e[j] * B + c] : 0;
+      base[j] = e[j] < 0 ? 0 : kShared ? (int64_t)scnt[e[j]] : cnt[(int64_t)e[j] * B + c];
     }
     __syncwarp();  // every lane has read its mask and counter
 #pragma unroll
     for (int j = 0; j < kM; ++j) {
       if (e[j] >= 0) {
         const int64_t rel = base[j] + before[j];
-        if (kFill) ids[offsets[e[j]] + rel] = n;
-        if (last[j]) cnt[(int64_t)e[j] * B + c] = rel + 1;
+        if (kFill) {
+          const int64_t pre = kShared ? cnt[(int64_t)e[j] * B + c] : 0;  // the chunk's prefix
+          ids[offsets[e[j]] + pre + rel] = n;
+        }
+        if (last[j]) {
+          if (kShared)
+            scnt[e[j]] = (int)(rel + 1);
+          else
+            cnt[(int64_t)e[j] * B + c] = rel + 1;
+        }
         key[slot[j]] = -1;
         lanes[slot[j]] = 0u;
       }
     }
     __syncwarp();  // counters advanced and the table empty for the next group
   }
+  if (kShared && !kFill)
+    for (int k = lane; k < K; k += 32) cnt[(int64_t)k * B + c] = scnt[k];
   if (bad) atomicOr(status, GMM_DEVFLAG_BAD_INDEX);
+}
+
+// Shared-memory counters: one int32 per list per warp, at most 64 KB per CTA,
+// and a chunk's entries (R points times m) within int32.
+inline bool ivf_shared_counters(int K, int64_t R, int m) {
+  return (size_t)K * kIvfWarps * 4 <= (64u << 10) && R * m < ((int64_t)1 << 31);
 }
 
 // Step 2a: one warp per list; exclusive prefix of cnt[k * B + 0 .. B) in place,
