@@ -38,7 +38,7 @@ namespace scem {
 
 constexpr int kIvfWarps = 8;                          // warps (chunks) per CTA
 constexpr int64_t kIvfMinPoints = 256;                // points per chunk, at least
-constexpr int64_t kIvfMaxChunks = 148 * 32;           // 4 CTAs of 8 warps on 148 SMs
+constexpr int64_t kIvfMaxChunks = 148 * 8;            // one CTA of 8 warps per SM (measured)
 constexpr size_t kIvfCountBytes = (size_t)64 << 20;   // bound on the count matrix
 
 // Workspace of gmm_ivf_build:
