@@ -89,7 +89,6 @@ constexpr int kTcMaxD = 128;      // the largest D with resident features
 // statistics, which accumulate kTcGroupChunks chunks per pass in tensor memory
 // (128 logit + 320 statistic + 16 N_k columns), one pass per feature group.
 constexpr int kTcMaxDStream = 1024;
-static_assert(kTcMaxDStream < 2048, "split and direct counts are packed in 11 bits");
 constexpr int kTcRoundChunks = 2;
 constexpr uint32_t kTcRBytes = 65536;  // r^ hi | lo of a 128-row tile, streamed layout
 constexpr int kTcGroupChunks = 5;
@@ -512,14 +511,6 @@ struct TcArgs {
 // every operand lies within the first 256 KB of shared memory, so no carry).
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
-// An entry of the CTA's list of components with direct-form dimensions: the
-// local column j (< 128), the split count ns and the direct count nd (each
-// <= D <= 1024) in 7 + 11 + 11 bits.
-__device__ __forceinline__ int shl_pack(int j, int ns, int nd) { return j | (ns << 7) | (nd << 18); }
-__device__ __forceinline__ int shl_j(int v) { return v & 127; }
-__device__ __forceinline__ int shl_ns(int v) { return (v >> 7) & 2047; }
-__device__ __forceinline__ int shl_nd(int v) { return (v >> 18) & 2047; }
-
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -611,7 +602,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   float* wscs = reinterpret_cast<float*>(sm + L.wscs);
   float* cxs = reinterpret_cast<float*>(sm + L.cxs);
   float* mgs = reinterpret_cast<float*>(sm + L.mgs);
-  int* shl = reinterpret_cast<int*>(sm + L.shl);  // [0] = count, [1..] = shl_pack entries
+  // [0]: how many local components take exact log-joints or direct-form
+  // moments; [129..132]: bit j of word q marks local component 32q + j as one
+  // with exact log-joints
+  int* shl = reinterpret_cast<int*>(sm + L.shl);
   int* shs = reinterpret_cast<int*>(sm + L.shs);  // [half][0] = count, [half][1..] = columns
   int* ndc = reinterpret_cast<int*>(sm + L.ndc);  // [128] direct dimensions, [128..131] mask
   int* precs = reinterpret_cast<int*>(sm + L.precs);
@@ -698,16 +692,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     int n = 0;
     uint32_t mw[4] = {0u, 0u, 0u, 0u};
-    // every component with exact log-joints or direct-form moments (shl_pack:
-    // local index, split count, direct count); the mask marks the former
     for (int j = 0; j < kTcComps; j++)
       if (a.ndir[k0 + j] > 0 || a.nsplit[k0 + j] > 0) {
-        const int ns = a.nsplit[k0 + j];
-        shl[1 + n++] = shl_pack(j, ns, a.ndir[k0 + j]);
-        if (ns > 0) mw[j >> 5] |= 1u << (j & 31);
+        n++;
+        if (a.nsplit[k0 + j] > 0) mw[j >> 5] |= 1u << (j & 31);
       }
     shl[0] = n;
-    // after the list (entries 1..128): bit j of word q is local component 32q + j
     for (int q = 0; q < 4; q++) shl[kTcComps + 1 + q] = (int)mw[q];
     // per column half, the columns with exact log-joints
     for (int h = 0; h < 2; h++) {
